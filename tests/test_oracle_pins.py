@@ -1,0 +1,472 @@
+"""Pins for the CPU oracle: closed forms, brute force, library routines and invariants.
+
+Each test checks the oracle against something other than itself, chosen so that a
+plausible slip (a dropped term, a wrong index, a transposed operand, a wrong divisor) fails.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import bsa_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(shape, seed, dtype=np.float64):
+    return np.random.default_rng(seed).standard_normal(shape).astype(dtype)
+
+
+GRIDS = [(4, 8, 8), (6, 10, 9), (5, 7, 3), (8, 16, 16), (1, 1, 1), (9, 4, 5)]
+
+
+# ------------------------------------------------------------------------------ reorder
+@pytest.mark.parametrize("grid", GRIDS)
+def test_reorder_forward_formula(grid):
+    """Every token lands at the tile/slot given by the forward formula; padding is zero."""
+    T, Hs, Ws = grid
+    B, H, d = 2, 3, 5
+    x = _rand((B, T * Hs * Ws, H, d), 1) + 10.0
+    xt = O.reorder(x, T, Hs, Ws)
+    nT, nY, nX = -(-T // 4), -(-Hs // 4), -(-Ws // 4)
+    assert xt.shape == (B, H, nT * nY * nX, 64, d)
+    seen = np.zeros(xt.shape[2:4], dtype=bool)
+    for t in range(T):
+        for y in range(Hs):
+            for xx in range(Ws):
+                n = (t * Hs + y) * Ws + xx
+                j = ((t // 4) * nY + y // 4) * nX + xx // 4
+                r = ((t % 4) * 4 + y % 4) * 4 + xx % 4
+                assert np.array_equal(xt[:, :, j, r, :], x[:, n, :, :])
+                seen[j, r] = True
+    assert np.all(xt[:, :, ~seen, :] == 0.0)
+    assert seen.sum() == T * Hs * Ws
+
+
+@pytest.mark.parametrize("grid", GRIDS)
+def test_reorder_round_trip_bitwise(grid):
+    T, Hs, Ws = grid
+    x = torch.randn(1, T * Hs * Ws, 2, 8, generator=torch.Generator().manual_seed(3))
+    xb = x.to(torch.bfloat16).view(torch.int16).numpy()
+    back = O.unreorder(O.reorder(xb, T, Hs, Ws), T, Hs, Ws)
+    assert back.dtype == xb.dtype and np.array_equal(back, xb)
+
+
+# ------------------------------------------------------------------------------ pooling
+@pytest.mark.parametrize("grid", [(6, 10, 9), (8, 16, 16), (5, 7, 3)])
+def test_pool_matches_raster_block_mean(grid):
+    """Mean over the raster block of each tile, computed by slicing the raster grid."""
+    T, Hs, Ws = grid
+    B, H, d = 1, 2, 4
+    x = _rand((B, T * Hs * Ws, H, d), 5)
+    xb = O.pool(O.reorder(x, T, Hs, Ws), T, Hs, Ws)
+    g = x.reshape(B, T, Hs, Ws, H, d)
+    nT, nY, nX = O.tile_grid(T, Hs, Ws)
+    for tt in range(nT):
+        for ty in range(nY):
+            for tx in range(nX):
+                blk = g[:, 4 * tt:4 * tt + 4, 4 * ty:4 * ty + 4, 4 * tx:4 * tx + 4]
+                ref = blk.reshape(B, -1, H, d).mean(axis=1)             # [B, H, d]
+                j = (tt * nY + ty) * nX + tx
+                np.testing.assert_allclose(xb[:, :, j, :], ref, rtol=1e-13, atol=1e-13)
+
+
+def test_pool_constant_tiles_exact():
+    T, Hs, Ws = 6, 10, 9                       # ragged: partial tiles everywhere at edges
+    NT = np.prod(O.tile_grid(T, Hs, Ws))
+    vals = np.arange(NT, dtype=np.float64) * 0.375 - 3.0
+    src = O.slot_tokens(T, Hs, Ws)
+    x = np.zeros((1, T * Hs * Ws, 1, 3))
+    for j in range(NT):
+        for r in range(64):
+            if src[j, r] >= 0:
+                x[0, src[j, r], 0, :] = vals[j]
+    xb = O.pool(O.reorder(x, T, Hs, Ws), T, Hs, Ws)
+    assert np.array_equal(xb[0, 0, :, 0], vals)
+
+
+# ------------------------------------------------------------------------------ windows
+def _golden_windows():
+    rows = []
+    with open(os.path.join(GOLDEN, "window_sizes.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            kind, r, size = line.split()
+            rows.append((0 if kind == "cube" else 1, int(r), int(size)))
+    return rows
+
+
+@pytest.mark.parametrize("kind,r,size", _golden_windows())
+def test_window_interior_size(kind, r, size):
+    T = Hs = Ws = 4 * (2 * r + 3)              # big enough that the centre tile is interior
+    nT, nY, nX = O.tile_grid(T, Hs, Ws)
+    c = ((nT // 2) * nY + nY // 2) * nX + nX // 2
+    assert int(O.window_row(kind, r, c, T, Hs, Ws).sum()) == size
+    assert int(O.window(kind, r, T, Hs, Ws)[c].sum()) == size
+
+
+@pytest.mark.parametrize("kind", [0, 1])
+@pytest.mark.parametrize("r", [0, 1, 2, 3])
+@pytest.mark.parametrize("grid", [(8, 16, 16), (6, 10, 9), (21, 30, 52)])
+def test_window_brute_force_and_clipped_counts(kind, r, grid):
+    """Brute-force loops (small grids) and per-axis clipped counts (all grids)."""
+    T, Hs, Ws = grid
+    nT, nY, nX = O.tile_grid(T, Hs, Ws)
+    W = O.window(kind, r, T, Hs, Ws)
+
+    def clip_count(c, s, n):
+        return max(0, min(c + s, n - 1) - max(c - s, 0) + 1) if s >= 0 else 0
+
+    for i in range(W.shape[0]):
+        tt, rem = divmod(i, nY * nX)
+        ty, tx = divmod(rem, nX)
+        if kind == 0:
+            expect = clip_count(tt, r, nT) * clip_count(ty, r, nY) * clip_count(tx, r, nX)
+        else:
+            expect = sum(clip_count(ty, r - abs(dt), nY) * clip_count(tx, r - abs(dt), nX)
+                         for dt in range(-r, r + 1) if 0 <= tt + dt < nT)
+        assert int(W[i].sum()) == expect
+    if W.shape[0] <= 64:
+        for i in range(W.shape[0]):
+            ti, rem = divmod(i, nY * nX)
+            yi, xi = divmod(rem, nX)
+            for j in range(W.shape[1]):
+                tj, rem = divmod(j, nY * nX)
+                yj, xj = divmod(rem, nX)
+                dt, dy, dx = abs(ti - tj), abs(yi - yj), abs(xi - xj)
+                inside = max(dt, dy, dx) <= r if kind == 0 else (dt <= r and max(dy, dx) <= r - dt)
+                assert W[i, j] == inside
+
+
+# ------------------------------------------------------------------------------ routing
+@pytest.mark.parametrize("rho", [0.0, 0.1, 0.2, 0.25, 0.5, 1.0])
+def test_route_count_and_order(rho):
+    rng = np.random.default_rng(7)
+    d = rng.random((3, 37)).astype(np.float32)
+    d[1, 5] = d[1, 9] = d[1, 30] = 0.999     # planted ties: lower index wins
+    dense = O.route_dense(d, rho)
+    nd = int(math.floor(float(np.float32(rho)) * 37 + 0.5))
+    assert np.all(dense.sum(axis=1) == nd)
+    for b in range(3):
+        order = sorted(range(37), key=lambda i: (-float(d[b, i]), i))
+        assert set(np.nonzero(dense[b])[0]) == set(order[:nd])
+    if rho == 0.0:
+        assert not dense.any()
+    if rho == 1.0:
+        assert dense.all()
+
+
+# ------------------------------------------------------------------------------ selection
+def _planted(T, Hs, Ws, H, d, kvals, qvec):
+    """Tiled Q/K whose every valid slot of tile j holds qvec (Q) and kvals[j] (K)."""
+    NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
+    valid = O.slot_valid(T, Hs, Ws)
+    qt = np.zeros((1, H, NT, 64, d))
+    kt = np.zeros((1, H, NT, 64, d))
+    for j in range(NT):
+        qt[0, :, j, valid[j]] = qvec
+        kt[0, :, j, valid[j]] = kvals[j]
+    return qt, kt
+
+
+@pytest.mark.parametrize("kind", [0, 1])
+def test_topk_planted_increasing_scores(kind):
+    """kbar_j = c*j*e1, qbar = e1: the extra tiles are the highest-indexed outside the window."""
+    T, Hs, Ws, d, k = 8, 16, 16, 8, 3
+    NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
+    e1 = np.zeros(d); e1[0] = 1.0
+    qt, kt = _planted(T, Hs, Ws, 2, d, [0.25 * (j + 1) * e1 for j in range(NT)], e1)
+    diff = np.zeros((1, NT), np.float32)
+    res = O.build_mask(qt, kt, diff, T=T, Hs=Hs, Ws=Ws, window_kind=kind, radius=1, topk=k,
+                       dense_fraction=0.0)
+    W = O.window(kind, 1, T, Hs, Ws)
+    for i in range(NT):
+        outside = [j for j in range(NT) if not W[i, j]]
+        expect = set(np.nonzero(W[i])[0]) | set(outside[-k:])
+        assert set(np.nonzero(res["mask"][0, 0, i])[0]) == expect
+        assert res["count"][0, 0, i] == W[i].sum() + min(k, len(outside))
+
+
+def test_topk_ties_go_to_lower_index():
+    T, Hs, Ws, d, k = 8, 16, 16, 4, 2
+    NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
+    e1 = np.zeros(d); e1[0] = 1.0
+    qt, kt = _planted(T, Hs, Ws, 1, d, [e1 for _ in range(NT)], e1)   # all scores equal
+    res = O.build_mask(qt, kt, np.zeros((1, NT), np.float32), T=T, Hs=Hs, Ws=Ws,
+                       window_kind=0, radius=0, topk=k, dense_fraction=0.0)
+    for i in range(NT):
+        outside = [j for j in range(NT) if j != i]
+        assert set(np.nonzero(res["mask"][0, 0, i])[0]) == {i, *outside[:k]}
+        assert res["near_tie"][0, 0, i]                   # equal scores are flagged
+
+
+def test_dense_rows_and_mask_invariants():
+    from bsa_synth import WORKLOADS, generate_qkv, generate_difficulty
+    w = WORKLOADS["tiny_ragged"]
+    q, k, v = generate_qkv(w)
+    diff = generate_difficulty(w).numpy()
+    qt, kt = O.reorder(O.to_f64(q), w.T, w.Hs, w.Ws), O.reorder(O.to_f64(k), w.T, w.Hs, w.Ws)
+    res = O.build_mask(qt, kt, diff, T=w.T, Hs=w.Hs, Ws=w.Ws, window_kind=0, radius=1,
+                       topk=2, dense_fraction=0.25)
+    NT = w.NT
+    W = O.window(0, 1, w.T, w.Hs, w.Ws)
+    assert res["dense"].sum() == O.n_dense(0.25, NT)
+    for i in range(NT):
+        for h in range(w.H):
+            row = res["mask"][0, h, i]
+            if res["dense"][0, i]:
+                assert row.all()
+            else:
+                assert np.all(row[W[i]])
+                assert row.sum() == W[i].sum() + min(2, NT - W[i].sum())
+    # dense routing is shared by every head
+    assert np.all(res["mask"][0, 0][res["dense"][0]] == res["mask"][0, 1][res["dense"][0]])
+
+
+def test_pooled_scores_against_direct_sum():
+    qbar = _rand((1, 2, 5, 16), 11)
+    kbar = _rand((1, 2, 7, 16), 12)
+    S = O.pooled_scores(qbar, kbar)
+    for h in range(2):
+        for i in range(5):
+            for j in range(7):
+                ref = sum(qbar[0, h, i, c] * kbar[0, h, j, c] for c in range(16)) / 4.0
+                assert abs(S[0, h, i, j] - ref) < 1e-12
+
+
+# ------------------------------------------------------------------------------ entropy budget
+def test_entropy_matches_scipy():
+    from scipy.special import softmax
+    from scipy.stats import entropy
+    s = _rand((3, 50), 13) * 3
+    ref = np.array([entropy(softmax(row)) for row in s])
+    np.testing.assert_allclose(O.row_entropy(s), ref, rtol=1e-12)
+
+
+def test_entropy_budget_uniform_scores():
+    """Identical kbar: every row's entropy is ln NKT and every budget is round(tau*NKT)."""
+    T, Hs, Ws, d = 8, 16, 16, 4
+    NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
+    e1 = np.zeros(d); e1[0] = 1.0
+    qt, kt = _planted(T, Hs, Ws, 1, d, [e1] * NT, 0.3 * e1)
+    for tau in (0.09, 0.14, 0.19, 0.5):
+        res = O.build_mask(qt, kt, np.zeros((1, NT), np.float32), T=T, Hs=Hs, Ws=Ws,
+                           window_kind=1, radius=0, topk=0, dense_fraction=0.0,
+                           budget_mode=1, budget_target=tau)
+        H = O.row_entropy(res["scores"][0, 0])
+        np.testing.assert_allclose(H, math.log(NT), rtol=1e-12)
+        expect = min(max(int(math.floor(float(np.float32(tau)) * NT + 0.5)), 1), NT)
+        assert np.all(res["budget"][0, 0] == expect)
+        assert np.all(res["count"][0, 0] == expect)
+
+
+def test_entropy_one_hot_dominant():
+    s = np.zeros((1, 20)); s[0, 3] = 60.0
+    assert O.row_entropy(s)[0] < 1e-20
+    b, x = O.entropy_budgets(np.array([0.0, math.log(20.0)]), 0.5, 20)
+    # budgets proportional to exp(H): 1 : 20, total tau*NKT*NQT = 20
+    np.testing.assert_allclose(x, [20.0 / 21.0, 400.0 / 21.0], rtol=1e-12)
+    assert list(b) == [1, 19]
+
+
+@pytest.mark.parametrize("grid", [(8, 16, 16), (33, 45, 80)])
+def test_radius_for_budget_brute(grid):
+    T, Hs, Ws = grid
+    NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
+    rng = np.random.default_rng(4)
+    for _ in range(12):
+        i = int(rng.integers(NT))
+        b = int(rng.integers(1, NT + 1))
+        r = O.radius_for_budget(b, i, T, Hs, Ws)
+        sizes = [int(O.window_row(1, rr, i, T, Hs, Ws).sum()) for rr in range(r + 2)]
+        assert sizes[r] <= b
+        assert sizes[r + 1] > b or sizes[r] == NT
+
+
+# ------------------------------------------------------------------------------ bitmask
+def test_bitmask_layout():
+    m = np.zeros((2, 70), dtype=bool)
+    m[0, [0, 31, 32, 69]] = True
+    m[1, 33] = True
+    bits = O.pack_bitmask(m)
+    assert bits.shape == (2, 3) and bits.dtype == np.uint32
+    assert bits[0, 0] == (1 | (1 << 31)) and bits[0, 1] == 1 and bits[0, 2] == (1 << 5)
+    assert bits[1, 1] == 2
+    assert np.array_equal(O.unpack_bitmask(bits, 70), m)
+
+
+# ------------------------------------------------------------------------------ attention
+def _qkv(grid, B=1, H=2, d=8, seed=21):
+    T, Hs, Ws = grid
+    N = T * Hs * Ws
+    return [_rand((B, N, H, d), seed + i) for i in range(3)]
+
+
+@pytest.mark.parametrize("grid", [(4, 8, 8), (6, 10, 9)])
+def test_all_retained_equals_dense_sdpa(grid):
+    """All tiles retained == textbook dense softmax attention on the raster sequence."""
+    T, Hs, Ws = grid
+    q, k, v = _qkv(grid)
+    qt, kt, vt = (O.reorder(a, T, Hs, Ws) for a in (q, k, v))
+    NT = qt.shape[2]
+    mask = np.ones((1, 2, NT, NT), dtype=bool)
+    Ot, L = O.attention(qt, kt, vt, mask, T=T, Hs=Hs, Ws=Ws)
+    tq, tk, tv = (torch.from_numpy(a).permute(0, 2, 1, 3) for a in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv).permute(0, 2, 1, 3)
+    np.testing.assert_allclose(Ot, ref.numpy(), rtol=1e-11, atol=1e-12)
+    s = np.einsum("bnhd,bmhd->bhnm", q, k) / math.sqrt(8)
+    lse_ref = np.log(np.exp(s).sum(-1))
+    np.testing.assert_allclose(L, lse_ref, rtol=1e-12)
+
+
+def test_sparse_equals_sdpa_with_token_mask():
+    """A random tile mask expanded to tokens and fed to SDPA in raster order."""
+    grid = (6, 10, 9)
+    T, Hs, Ws = grid
+    q, k, v = _qkv(grid, B=2, H=3, d=8, seed=31)
+    qt, kt, vt = (O.reorder(a, T, Hs, Ws) for a in (q, k, v))
+    NT = qt.shape[2]
+    rng = np.random.default_rng(9)
+    mask = rng.random((2, 3, NT, NT)) < 0.3
+    mask[..., np.arange(NT), np.arange(NT)] = True
+    Ot, L = O.attention(qt, kt, vt, mask, T=T, Hs=Hs, Ws=Ws)
+    N = T * Hs * Ws
+    tile_of = np.zeros(N, dtype=np.int64)
+    src = O.slot_tokens(T, Hs, Ws)
+    for j in range(NT):
+        for r in range(64):
+            if src[j, r] >= 0:
+                tile_of[src[j, r]] = j
+    tok_mask = mask[:, :, tile_of][:, :, :, tile_of]                     # [B,H,N,N]
+    tq, tk, tv = (torch.from_numpy(a).permute(0, 2, 1, 3) for a in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk, tv, attn_mask=torch.from_numpy(tok_mask)).permute(0, 2, 1, 3)
+    np.testing.assert_allclose(Ot, ref.numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_brute_force_per_query_softmax():
+    """Plain loops over tokens, membership by tile lookup, on a tiny ragged grid."""
+    T, Hs, Ws = 5, 6, 5
+    q, k, v = _qkv((T, Hs, Ws), H=1, d=3, seed=41)
+    qt, kt, vt = (O.reorder(a, T, Hs, Ws) for a in (q, k, v))
+    nT, nY, nX = O.tile_grid(T, Hs, Ws)
+    NT = nT * nY * nX
+    mask = np.random.default_rng(2).random((1, 1, NT, NT)) < 0.5
+    mask[..., np.arange(NT), np.arange(NT)] = True
+    Ot, L = O.attention(qt, kt, vt, mask, T=T, Hs=Hs, Ws=Ws)
+
+    def tile(n):
+        t, rem = divmod(n, Hs * Ws)
+        y, x = divmod(rem, Ws)
+        return ((t // 4) * nY + y // 4) * nX + x // 4
+
+    N = T * Hs * Ws
+    for n in range(N):
+        s = []
+        for m in range(N):
+            if mask[0, 0, tile(n), tile(m)]:
+                s.append((sum(q[0, n, 0, c] * k[0, m, 0, c] for c in range(3)) / math.sqrt(3), m))
+        mx = max(a for a, _ in s)
+        z = sum(math.exp(a - mx) for a, _ in s)
+        o = [sum(math.exp(a - mx) / z * v[0, m, 0, c] for a, m in s) for c in range(3)]
+        assert np.allclose(Ot[0, n, 0], o, rtol=1e-12, atol=1e-13)
+        assert abs(L[0, 0, n] - (mx + math.log(z))) < 1e-12
+
+
+def test_weights_cover_exactly_retained_valid_keys():
+    T, Hs, Ws = 6, 10, 9
+    q, k, v = _qkv((T, Hs, Ws), H=1, d=4, seed=51)
+    qt, kt, vt = (O.reorder(a, T, Hs, Ws) for a in (q, k, v))
+    NT = qt.shape[2]
+    mask = np.random.default_rng(3).random((1, 1, NT, NT)) < 0.4
+    mask[..., np.arange(NT), np.arange(NT)] = True
+    valid = O.slot_valid(T, Hs, Ws)
+    rows = [(0, 0, i) for i in range(NT)]
+    res = O.attention_tiles(qt, kt, vt, mask, rows, T=T, Hs=Hs, Ws=Ws, return_weights=True)
+    for (b, h, i), e in res.items():
+        ids = {tuple(x) for x in e["key_ids"]}
+        expect = {(j, r) for j in np.nonzero(mask[0, 0, i])[0] for r in range(64) if valid[j, r]}
+        assert ids == expect
+        w = e["weights"][e["valid"]]
+        np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=1e-13)
+        assert np.all(w > 0)
+
+
+def test_zero_query_gives_mean_of_retained_values():
+    T, Hs, Ws = 6, 10, 9
+    q, k, v = _qkv((T, Hs, Ws), H=1, d=4, seed=61)
+    q[:] = 0.0
+    qt, kt, vt = (O.reorder(a, T, Hs, Ws) for a in (q, k, v))
+    NT = qt.shape[2]
+    mask = np.random.default_rng(5).random((1, 1, NT, NT)) < 0.4
+    mask[..., np.arange(NT), np.arange(NT)] = True
+    valid = O.slot_valid(T, Hs, Ws)
+    res = O.attention_tiles(qt, kt, vt, mask, [(0, 0, i) for i in range(NT)], T=T, Hs=Hs, Ws=Ws)
+    for (b, h, i), e in res.items():
+        keep = np.nonzero(mask[0, 0, i])[0]
+        vals = np.concatenate([vt[0, 0, j][valid[j]] for j in keep])
+        np.testing.assert_allclose(e["o"][e["valid"]], np.broadcast_to(vals.mean(0), (e["valid"].sum(), 4)),
+                                   rtol=1e-12)
+        np.testing.assert_allclose(e["lse"][e["valid"]], math.log(len(vals)), rtol=1e-13)
+
+
+def test_single_valid_key_returns_its_value():
+    T, Hs, Ws = 5, 5, 5                        # tile (1,1,1) holds exactly one token
+    q, k, v = _qkv((T, Hs, Ws), H=1, d=4, seed=71)
+    qt, kt, vt = (O.reorder(a, T, Hs, Ws) for a in (q, k, v))
+    NT = qt.shape[2]
+    last = NT - 1
+    assert O.slot_valid(T, Hs, Ws)[last].sum() == 1
+    mask = np.zeros((1, 1, NT, NT), dtype=bool)
+    mask[0, 0, :, last] = True
+    Ot, _ = O.attention(qt, kt, vt, mask, T=T, Hs=Hs, Ws=Ws)
+    n_last = T * Hs * Ws - 1
+    np.testing.assert_allclose(Ot[0, :, 0, :], np.broadcast_to(v[0, n_last, 0], (T * Hs * Ws, 4)),
+                               rtol=1e-14)
+
+
+def test_full_forward_tiny_is_dense():
+    """The 4x8x8 grid has 4 tiles, all inside a radius-1 cube: the path is dense attention."""
+    from bsa_synth import WORKLOADS, generate_qkv, generate_difficulty
+    w = WORKLOADS["tiny"]
+    q, k, v = (O.to_f64(t) for t in generate_qkv(w))
+    res = O.forward(q, k, v, generate_difficulty(w).numpy(), T=w.T, Hs=w.Hs, Ws=w.Ws,
+                    window_kind=0, radius=1, topk=1, dense_fraction=0.25)
+    assert res["mask"].all()
+    tq, tk, tv = (torch.from_numpy(a).permute(0, 2, 1, 3) for a in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv).permute(0, 2, 1, 3)
+    np.testing.assert_allclose(res["O"], ref.numpy(), rtol=1e-11, atol=1e-12)
+
+
+# ------------------------------------------------------------------------------ planted mistakes
+def test_pins_catch_planted_pool_divisor(monkeypatch):
+    """Dividing by 64 instead of the valid count must break the raster-mean pin."""
+    def bad_pool(xt, T, Hs, Ws):
+        valid = O.slot_valid(T, Hs, Ws).astype(np.float64)
+        return np.einsum("bhjrd,jr->bhjd", np.asarray(xt, np.float64), valid) / 64.0
+    monkeypatch.setattr(O, "pool", bad_pool)
+    with pytest.raises(AssertionError):
+        test_pool_matches_raster_block_mean((6, 10, 9))
+
+
+def test_pins_catch_planted_transpose(monkeypatch):
+    """Scoring K against Q (transposed operands) must break the top-k pin."""
+    real = O.pooled_scores
+    monkeypatch.setattr(O, "pooled_scores", lambda a, b: real(b, a))
+    with pytest.raises(AssertionError):
+        test_topk_planted_increasing_scores(0)
+
+
+def test_pins_catch_planted_tie_break(monkeypatch):
+    """Breaking ties toward the higher index must break the tie pin."""
+    def bad_top(scores_row, excluded, m):
+        cand = np.nonzero(~excluded)[0]
+        order = np.lexsort((-cand, -scores_row[cand]))
+        return cand[order[:m]]
+    monkeypatch.setattr(O, "top_outside", bad_top)
+    with pytest.raises(AssertionError):
+        test_topk_ties_go_to_lower_index()
