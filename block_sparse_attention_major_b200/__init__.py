@@ -1,0 +1,294 @@
+"""Python binding of libbsa, the B200 block-sparse video attention library.
+
+Argument marshalling only: every step of the path runs in the library's CUDA kernels.
+PyTorch supplies device memory and the current stream. There is no CPU fallback: if
+libbsa.so is missing or the device is not a B200, the calls raise.
+
+Entry points (same names as the C ABI in include/bsa.h):
+    reorder(g, x)                   raster [B,N,H,d] -> tile-major [B,H,NT,64,d]
+    unreorder(g, xt)                the inverse
+    build_mask(g, p, qt, kt, difficulty)     -> (mask uint32 [B,H,NQT,W], kv_count int32)
+    sparse_attn_fwd(g, qt, kt, vt, mask, kv_count)  -> (out bf16 [B,N,H,d], lse fp32 [B,H,N])
+    forward(g, p, q, k, v, difficulty)       the whole path, raster in, raster out
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbsa.so")
+
+BSA_OK = 0
+STATUS_NAMES = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_WORKSPACE",
+                3: "BSA_ERR_UNSUPPORTED_DEVICE", 4: "BSA_ERR_CUDA"}
+KERR_WAIT_TIMEOUT, KERR_BAD_UNIT, KERR_BAD_MASK = 1, 2, 4
+
+
+class bsa_geom(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
+                ("T", ctypes.c_int), ("Hs", ctypes.c_int), ("Ws", ctypes.c_int)]
+
+
+class bsa_mask_params(ctypes.Structure):
+    _fields_ = [("window_kind", ctypes.c_int), ("radius", ctypes.c_int), ("topk", ctypes.c_int),
+                ("dense_fraction", ctypes.c_float), ("budget_mode", ctypes.c_int),
+                ("budget_target", ctypes.c_float)]
+
+
+class BsaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+_lib_lock = threading.Lock()
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load libbsa.so (built in-tree by _build.py); raises if it is missing."""
+    global _lib
+    with _lib_lock:
+        if _lib is not None and path is None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(f"libbsa.so not found at {p}: run `python -m "
+                               "block_sparse_attention_major_b200._build` first")
+        lib = ctypes.CDLL(p)
+        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        G, P = ctypes.POINTER(bsa_geom), ctypes.POINTER(bsa_mask_params)
+        lib.bsa_status_string.restype = ctypes.c_char_p
+        lib.bsa_status_string.argtypes = [ctypes.c_int]
+        lib.bsa_tile_grid.restype = ctypes.c_int
+        lib.bsa_tile_grid.argtypes = [G] + [ctypes.POINTER(ctypes.c_int)] * 4
+        lib.bsa_workspace_bytes.restype = sz
+        lib.bsa_workspace_bytes.argtypes = [G, P]
+        lib.bsa_clear_error.restype = ctypes.c_int
+        lib.bsa_clear_error.argtypes = [vp, vp]
+        lib.bsa_reorder.restype = ctypes.c_int
+        lib.bsa_reorder.argtypes = [G, vp, vp, vp]
+        lib.bsa_unreorder.restype = ctypes.c_int
+        lib.bsa_unreorder.argtypes = [G, vp, vp, vp]
+        lib.bsa_build_mask.restype = ctypes.c_int
+        lib.bsa_build_mask.argtypes = [G, P, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.bsa_sparse_attn_fwd.restype = ctypes.c_int
+        lib.bsa_sparse_attn_fwd.argtypes = [G, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, sz, vp]
+        lib.bsa_launch_count.restype = ctypes.c_uint64
+        lib.bsa_launch_count.argtypes = []
+        if path is None:
+            _lib = lib
+        return lib
+
+
+@dataclass(frozen=True)
+class Geometry:
+    B: int
+    H: int
+    d: int
+    T: int
+    Hs: int
+    Ws: int
+
+    @property
+    def N(self) -> int:
+        return self.T * self.Hs * self.Ws
+
+    @property
+    def tiles(self) -> tuple[int, int, int]:
+        return (-(-self.T // 4), -(-self.Hs // 4), -(-self.Ws // 4))
+
+    @property
+    def NT(self) -> int:
+        a, b, c = self.tiles
+        return a * b * c
+
+    @property
+    def NW(self) -> int:
+        return -(-self.NT // 32)
+
+    def c(self) -> bsa_geom:
+        return bsa_geom(self.B, self.H, self.d, self.T, self.Hs, self.Ws)
+
+
+@dataclass(frozen=True)
+class MaskParams:
+    window_kind: int = 0
+    radius: int = 1
+    topk: int = 0
+    dense_fraction: float = 0.0
+    budget_mode: int = 0
+    budget_target: float = 0.0
+
+    def c(self) -> bsa_mask_params:
+        return bsa_mask_params(self.window_kind, self.radius, self.topk, self.dense_fraction,
+                               self.budget_mode, self.budget_target)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _need(t: torch.Tensor, dtype, shape, name: str) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _check(status: int, what: str) -> None:
+    if status != BSA_OK:
+        raise BsaError(status, what)
+
+
+def workspace_bytes(g: Geometry, p: MaskParams | None = None) -> int:
+    pc = p.c() if p is not None else None
+    return int(load_library().bsa_workspace_bytes(ctypes.byref(g.c()),
+                                                  ctypes.byref(pc) if pc is not None else None))
+
+
+def alloc_workspace(g: Geometry, device=None) -> torch.Tensor:
+    """A zeroed device workspace (byte 0 = kernel error word)."""
+    n = workspace_bytes(g)
+    if n == 0:
+        raise ValueError("invalid geometry")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def read_error(ws: torch.Tensor) -> int:
+    """The kernel error word (synchronises the current stream)."""
+    return int(ws[:4].view(torch.int32).item()) & 0xFFFFFFFF
+
+
+def clear_error(ws: torch.Tensor, stream=None) -> None:
+    _check(load_library().bsa_clear_error(_ptr(ws), _stream(stream)), "bsa_clear_error")
+
+
+def launch_count() -> int:
+    return int(load_library().bsa_launch_count())
+
+
+def reorder(g: Geometry, x: torch.Tensor, xt: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    _need(x, torch.bfloat16, (g.B, g.N, g.H, g.d), "x")
+    if xt is None:
+        xt = torch.empty((g.B, g.H, g.NT, 64, g.d), dtype=torch.bfloat16, device=x.device)
+    _need(xt, torch.bfloat16, (g.B, g.H, g.NT, 64, g.d), "xt")
+    _check(load_library().bsa_reorder(ctypes.byref(g.c()), _ptr(x), _ptr(xt), _stream(stream)),
+           "bsa_reorder")
+    return xt
+
+
+def unreorder(g: Geometry, xt: torch.Tensor, x: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    _need(xt, torch.bfloat16, (g.B, g.H, g.NT, 64, g.d), "xt")
+    if x is None:
+        x = torch.empty((g.B, g.N, g.H, g.d), dtype=torch.bfloat16, device=xt.device)
+    _need(x, torch.bfloat16, (g.B, g.N, g.H, g.d), "x")
+    _check(load_library().bsa_unreorder(ctypes.byref(g.c()), _ptr(xt), _ptr(x), _stream(stream)),
+           "bsa_unreorder")
+    return x
+
+
+def build_mask(g: Geometry, p: MaskParams, qt: torch.Tensor, kt: torch.Tensor,
+               difficulty: torch.Tensor, mask: torch.Tensor | None = None,
+               kv_count: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+               stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    _need(qt, torch.bfloat16, (g.B, g.H, g.NT, 64, g.d), "qt")
+    _need(kt, torch.bfloat16, (g.B, g.H, g.NT, 64, g.d), "kt")
+    _need(difficulty, torch.float32, (g.B, g.NT), "difficulty")
+    dev = qt.device
+    if mask is None:
+        mask = torch.empty((g.B, g.H, g.NT, g.NW), dtype=torch.int32, device=dev)
+    if kv_count is None:
+        kv_count = torch.empty((g.B, g.H, g.NT), dtype=torch.int32, device=dev)
+    _need(mask, torch.int32, (g.B, g.H, g.NT, g.NW), "mask")
+    _need(kv_count, torch.int32, (g.B, g.H, g.NT), "kv_count")
+    if ws is None:
+        ws = alloc_workspace(g, dev)
+    pc = p.c()
+    _check(load_library().bsa_build_mask(ctypes.byref(g.c()), ctypes.byref(pc), _ptr(qt), _ptr(kt),
+                                         _ptr(difficulty), _ptr(mask), _ptr(kv_count), _ptr(ws),
+                                         ctypes.c_size_t(ws.numel()), _stream(stream)),
+           "bsa_build_mask")
+    return mask, kv_count
+
+
+def sparse_attn_fwd(g: Geometry, qt: torch.Tensor, kt: torch.Tensor, vt: torch.Tensor,
+                    mask: torch.Tensor, kv_count: torch.Tensor, scale: float | None = None,
+                    out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                    ws: torch.Tensor | None = None, want_lse: bool = True,
+                    stream=None) -> tuple[torch.Tensor, torch.Tensor | None]:
+    for name, t in (("qt", qt), ("kt", kt), ("vt", vt)):
+        _need(t, torch.bfloat16, (g.B, g.H, g.NT, 64, g.d), name)
+    _need(mask, torch.int32, (g.B, g.H, g.NT, g.NW), "mask")
+    _need(kv_count, torch.int32, (g.B, g.H, g.NT), "kv_count")
+    dev = qt.device
+    if out is None:
+        out = torch.empty((g.B, g.N, g.H, g.d), dtype=torch.bfloat16, device=dev)
+    _need(out, torch.bfloat16, (g.B, g.N, g.H, g.d), "out")
+    if want_lse and lse is None:
+        lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _need(lse, torch.float32, (g.B, g.H, g.N), "lse")
+    if ws is None:
+        ws = alloc_workspace(g, dev)
+    sc = 1.0 / math.sqrt(g.d) if scale is None else float(scale)
+    _check(load_library().bsa_sparse_attn_fwd(ctypes.byref(g.c()), _ptr(qt), _ptr(kt), _ptr(vt),
+                                              _ptr(mask), _ptr(kv_count), ctypes.c_float(sc),
+                                              _ptr(out), _ptr(lse), _ptr(ws),
+                                              ctypes.c_size_t(ws.numel()), _stream(stream)),
+           "bsa_sparse_attn_fwd")
+    return out, lse
+
+
+class Buffers:
+    """Device buffers of one attention call, allocated once and reused across calls."""
+
+    def __init__(self, g: Geometry, device=None):
+        dev = device or "cuda"
+        tiled = (g.B, g.H, g.NT, 64, g.d)
+        self.qt = torch.empty(tiled, dtype=torch.bfloat16, device=dev)
+        self.kt = torch.empty(tiled, dtype=torch.bfloat16, device=dev)
+        self.vt = torch.empty(tiled, dtype=torch.bfloat16, device=dev)
+        self.mask = torch.empty((g.B, g.H, g.NT, g.NW), dtype=torch.int32, device=dev)
+        self.kv_count = torch.empty((g.B, g.H, g.NT), dtype=torch.int32, device=dev)
+        self.out = torch.empty((g.B, g.N, g.H, g.d), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device=dev)
+        self.ws = alloc_workspace(g, dev)
+
+
+def forward(g: Geometry, p: MaskParams, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+            difficulty: torch.Tensor, bufs: Buffers | None = None, scale: float | None = None,
+            stream=None) -> Buffers:
+    """The whole path: reorder Q, K, V; build the mask; block-sparse attention.
+
+    Returns the buffers; out / lse hold the attention output and LSE in raster order.
+    """
+    b = bufs or Buffers(g, q.device)
+    reorder(g, q, b.qt, stream)
+    reorder(g, k, b.kt, stream)
+    reorder(g, v, b.vt, stream)
+    build_mask(g, p, b.qt, b.kt, difficulty, b.mask, b.kv_count, b.ws, stream)
+    sparse_attn_fwd(g, b.qt, b.kt, b.vt, b.mask, b.kv_count, scale, b.out, b.lse, b.ws,
+                    stream=stream)
+    return b
+
+
+# kernels launched by forward(): 3 reorders, pool + route + 1 select (2 in budget mode),
+# 3 scheduler kernels + the attention kernel
+def launches_per_forward(p: MaskParams) -> int:
+    return 3 + 2 + (2 if p.budget_mode == 1 else 1) + 4

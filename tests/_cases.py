@@ -1,0 +1,109 @@
+"""Shared helpers of the parity tests: seeded inputs, oracle runs and comparisons."""
+from __future__ import annotations
+
+import functools
+import math
+
+import numpy as np
+import torch
+
+from bsa_synth import WORKLOADS, Workload, generate_difficulty, generate_qkv
+from oracle import bsa_oracle as O
+
+# Tolerances of the GPU path against the fp64 oracle (attention output relative L2 and max
+# abs error on bf16-rounded inputs; natural-log LSE absolute error).
+O_REL_L2 = 5e-3
+O_MAX_ABS = 2e-2
+LSE_ABS = 1e-3
+
+SMALL_D128 = {
+    "small128": Workload("small128", B=1, H=2, d=128, T=8, Hs=16, Ws=16, seed=1010,
+                         window_kind=1, radius=1, topk=2, dense_fraction=0.25),
+    "ragged128": Workload("ragged128", B=2, H=3, d=128, T=7, Hs=13, Ws=10, seed=1011,
+                          window_kind=0, radius=1, topk=3, dense_fraction=0.2),
+    "budget128": Workload("budget128", B=1, H=2, d=128, T=12, Hs=16, Ws=20, seed=1012,
+                          window_kind=1, radius=0, topk=0, dense_fraction=0.0,
+                          budget_mode=1, budget_target=0.19),
+}
+
+
+def workload(name: str) -> Workload:
+    return WORKLOADS[name] if name in WORKLOADS else SMALL_D128[name]
+
+
+@functools.lru_cache(maxsize=8)
+def inputs(name: str, overrides: tuple = ()):
+    """bf16 q, k, v [B,N,H,d] (CPU), difficulty [B,NQT] fp32 (CPU) and float64 copies."""
+    w = workload(name).with_(**dict(overrides))
+    q, k, v = generate_qkv(w)
+    diff = generate_difficulty(w)
+    return w, q, k, v, diff
+
+
+def geometry(w: Workload):
+    from block_sparse_attention_major_b200 import Geometry
+    return Geometry(w.B, w.H, w.d, w.T, w.Hs, w.Ws)
+
+
+def params(w: Workload):
+    from block_sparse_attention_major_b200 import MaskParams
+    return MaskParams(w.window_kind, w.radius, w.topk, w.dense_fraction, w.budget_mode,
+                      w.budget_target)
+
+
+def oracle_mask(w: Workload, qt64: np.ndarray, kt64: np.ndarray, diff: np.ndarray) -> dict:
+    return O.build_mask(qt64, kt64, diff, T=w.T, Hs=w.Hs, Ws=w.Ws, window_kind=w.window_kind,
+                        radius=w.radius, topk=w.topk, dense_fraction=w.dense_fraction,
+                        budget_mode=w.budget_mode, budget_target=w.budget_target)
+
+
+def gpu_mask_bool(mask_i32: torch.Tensor, NKT: int) -> np.ndarray:
+    bits = mask_i32.cpu().numpy().view(np.uint32)
+    return O.unpack_bitmask(bits, NKT)
+
+
+def compare_masks(gpu: np.ndarray, ref: dict) -> dict:
+    """Row-wise comparison; disagreements are allowed only in rows the oracle flags."""
+    diff_rows = np.any(gpu != ref["mask"], axis=-1)
+    unflagged = diff_rows & ~ref["near_tie"]
+    return dict(n_rows=int(diff_rows.size), n_diff=int(diff_rows.sum()),
+                n_unflagged=int(unflagged.sum()), n_flagged=int(ref["near_tie"].sum()),
+                diff_rows=diff_rows)
+
+
+def compare_attention(w: Workload, out: torch.Tensor, lse: torch.Tensor | None, ref: dict,
+                      skip_rows: np.ndarray | None = None) -> dict:
+    """GPU out [B,N,H,d] / lse [B,H,N] against oracle per-tile results {(b,h,i): entry}."""
+    src = O.slot_tokens(w.T, w.Hs, w.Ws)
+    out64 = out.float().cpu().numpy().astype(np.float64)
+    lse64 = lse.cpu().numpy().astype(np.float64) if lse is not None else None
+    num = den = 0.0
+    max_abs = 0.0
+    max_lse = 0.0
+    worst_tile = 0.0
+    compared = 0
+    for (b, h, i), e in ref.items():
+        if skip_rows is not None and skip_rows[b, h, i]:
+            continue
+        toks = src[i][e["valid"]]
+        got = out64[b, toks, h, :]
+        want = e["o"][e["valid"]]
+        dn = float(((got - want) ** 2).sum())
+        dd = float((want ** 2).sum())
+        num += dn
+        den += dd
+        worst_tile = max(worst_tile, math.sqrt(dn / max(dd, 1e-300)))
+        max_abs = max(max_abs, float(np.abs(got - want).max()))
+        if lse64 is not None:
+            max_lse = max(max_lse, float(np.abs(lse64[b, h, toks] - e["lse"][e["valid"]]).max()))
+        compared += 1
+    return dict(rel_l2=math.sqrt(num / max(den, 1e-300)), worst_tile_rel_l2=worst_tile,
+                max_abs=max_abs, max_lse=max_lse, tiles=compared)
+
+
+def assert_attention_close(stats: dict) -> None:
+    assert stats["tiles"] > 0
+    assert stats["rel_l2"] <= O_REL_L2, stats
+    assert stats["worst_tile_rel_l2"] <= O_REL_L2, stats
+    assert stats["max_abs"] <= O_MAX_ABS, stats
+    assert stats["max_lse"] <= LSE_ABS, stats

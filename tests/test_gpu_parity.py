@@ -1,0 +1,279 @@
+"""GPU parity: every CUDA kernel against the fp64 CPU oracle, through the C ABI.
+
+Reorder / unreorder must be bit-exact. Masks must be bit-exact except in rows the oracle
+flags as near-ties (score gaps below 1e-4 of the row's score scale), which are counted.
+Attention output must be within relative L2 5e-3 and max abs 2e-2 of the oracle, LSE
+within 1e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import _cases as C
+from oracle import bsa_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+SMALL = ["tiny", "tiny_s", "tiny_ragged", "small128", "ragged128", "budget128"]
+
+
+def _bsa():
+    import block_sparse_attention_major_b200 as bsa
+    return bsa
+
+
+def _i16(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy()
+
+
+# ----------------------------------------------------------------------------- reorder
+@pytest.mark.parametrize("name", SMALL + ["wan13b"])
+def test_reorder_bit_exact(name):
+    bsa = _bsa()
+    w, q, k, v, _ = C.inputs(name)
+    g = C.geometry(w)
+    for x in (q, k, v):
+        xt = bsa.reorder(g, x.cuda())
+        ref = O.reorder(_i16(x), w.T, w.Hs, w.Ws)
+        assert np.array_equal(_i16(xt), ref)
+
+
+@pytest.mark.parametrize("name", SMALL + ["wan13b"])
+def test_unreorder_round_trip_bit_exact(name):
+    bsa = _bsa()
+    w, q, _, _, _ = C.inputs(name)
+    g = C.geometry(w)
+    x = q.cuda()
+    back = bsa.unreorder(g, bsa.reorder(g, x))
+    assert torch.equal(back.view(torch.int16), x.view(torch.int16))
+    # unreorder of arbitrary tile-major data equals the oracle's (padding ignored)
+    xt = torch.randn((g.B, g.H, g.NT, 64, g.d), device="cuda").to(torch.bfloat16)
+    ref = O.unreorder(_i16(xt), w.T, w.Hs, w.Ws)
+    assert np.array_equal(_i16(bsa.unreorder(g, xt)), ref)
+
+
+# ----------------------------------------------------------------------------- mask
+def _mask_case(name, heads=None, overrides=()):
+    bsa = _bsa()
+    w, q, k, _, diff = C.inputs(name, overrides)
+    g = C.geometry(w)
+    qt = bsa.reorder(g, q.cuda())
+    kt = bsa.reorder(g, k.cuda())
+    ws = bsa.alloc_workspace(g)
+    mask, cnt = bsa.build_mask(g, C.params(w), qt, kt, diff.cuda(), ws=ws)
+    torch.cuda.synchronize()
+    assert bsa.read_error(ws) == 0
+    gm = C.gpu_mask_bool(mask, g.NT)
+    gc = cnt.cpu().numpy()
+    hsel = list(range(w.H)) if heads is None else heads
+    qt64 = O.reorder(O.to_f64(q), w.T, w.Hs, w.Ws)[:, hsel]
+    kt64 = O.reorder(O.to_f64(k), w.T, w.Hs, w.Ws)[:, hsel]
+    ref = C.oracle_mask(w, qt64, kt64, diff.numpy())
+    gm = gm[:, hsel]
+    cmp = C.compare_masks(gm, ref)
+    assert np.array_equal(gc[:, hsel], gm.sum(-1)), "kv_count is not the popcount of the row"
+    return w, g, gm, ref, cmp, mask, cnt
+
+
+@pytest.mark.parametrize("name", SMALL + ["wan13b"])
+def test_mask_bit_exact(name):
+    w, g, gm, ref, cmp, _, _ = _mask_case(name)
+    assert cmp["n_unflagged"] == 0, cmp
+    assert cmp["n_diff"] <= max(1, cmp["n_rows"] // 200), cmp
+    print(f"{name}: rows={cmp['n_rows']} differing={cmp['n_diff']} flagged={cmp['n_flagged']} "
+          f"retained={gm.mean():.4f}")
+
+
+@pytest.mark.parametrize("rho", [0.0, 0.1, 0.2, 0.4, 1.0])
+def test_mask_wan5b_rho_sweep(rho):
+    w, g, gm, ref, cmp, _, _ = _mask_case("wan5b", heads=[0, 11, 23],
+                                          overrides=(("dense_fraction", rho),))
+    assert cmp["n_unflagged"] == 0, cmp
+    assert ref["dense"].sum() == O.n_dense(rho, g.NT)
+
+
+def test_mask_wan14b_heads():
+    w, g, gm, ref, cmp, _, _ = _mask_case("wan14b", heads=[0, 39])
+    assert cmp["n_unflagged"] == 0, cmp
+
+
+@pytest.mark.parametrize("tau", [0.09, 0.19])
+def test_mask_hunyuan_budget_heads(tau):
+    w, g, gm, ref, cmp, _, _ = _mask_case("hunyuan", heads=[0, 23],
+                                          overrides=(("budget_target", tau),))
+    assert cmp["n_unflagged"] == 0, cmp
+    retained = gm.mean()
+    assert abs(retained - tau) < 0.05, retained
+
+
+def test_mask_deterministic():
+    bsa = _bsa()
+    w, q, k, _, diff = C.inputs("wan13b")
+    g = C.geometry(w)
+    qt, kt = bsa.reorder(g, q.cuda()), bsa.reorder(g, k.cuda())
+    m1, c1 = bsa.build_mask(g, C.params(w), qt, kt, diff.cuda())
+    m2, c2 = bsa.build_mask(g, C.params(w), qt, kt, diff.cuda())
+    assert torch.equal(m1, m2) and torch.equal(c1, c2)
+
+
+# ----------------------------------------------------------------------------- attention
+def _attn_with_mask(w, q, k, v, mask_bool, rows=None):
+    """GPU attention given a mask computed here (never from the GPU), plus oracle rows."""
+    bsa = _bsa()
+    g = C.geometry(w)
+    qt, kt, vt = (bsa.reorder(g, x.cuda()) for x in (q, k, v))
+    bits = O.pack_bitmask(mask_bool).view(np.int32)
+    mask = torch.from_numpy(bits.copy()).cuda()
+    cnt = torch.from_numpy(mask_bool.sum(-1).astype(np.int32)).cuda()
+    ws = bsa.alloc_workspace(g)
+    out, lse = bsa.sparse_attn_fwd(g, qt, kt, vt, mask, cnt, ws=ws)
+    torch.cuda.synchronize()
+    assert bsa.read_error(ws) == 0
+    if rows is None:
+        rows = [(b, h, i) for b in range(w.B) for h in range(w.H) for i in range(g.NT)]
+    qt64, kt64, vt64 = (O.reorder(O.to_f64(x), w.T, w.Hs, w.Ws) for x in (q, k, v))
+    ref = O.attention_tiles(qt64, kt64, vt64, mask_bool, rows, T=w.T, Hs=w.Hs, Ws=w.Ws)
+    return out, lse, ref
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_attention_oracle_mask(name):
+    w, q, k, v, diff = C.inputs(name)
+    qt64, kt64 = (O.reorder(O.to_f64(x), w.T, w.Hs, w.Ws) for x in (q, k))
+    mref = C.oracle_mask(w, qt64, kt64, diff.numpy())
+    out, lse, ref = _attn_with_mask(w, q, k, v, mref["mask"])
+    st = C.compare_attention(w, out, lse, ref)
+    print(name, st)
+    C.assert_attention_close(st)
+
+
+@pytest.mark.parametrize("pattern", ["random", "single", "all", "alternate", "last_only"])
+@pytest.mark.parametrize("name", ["ragged128", "tiny_ragged"])
+def test_attention_mask_patterns(name, pattern):
+    w, q, k, v, _ = C.inputs(name)
+    NT = w.NT
+    rng = np.random.default_rng(17)
+    if pattern == "random":
+        m = rng.random((w.B, w.H, NT, NT)) < 0.35
+        m[..., np.arange(NT), np.arange(NT)] = True
+    elif pattern == "single":
+        m = np.zeros((w.B, w.H, NT, NT), dtype=bool)
+        m[..., np.arange(NT), rng.integers(0, NT, NT)] = True
+    elif pattern == "all":
+        m = np.ones((w.B, w.H, NT, NT), dtype=bool)
+    elif pattern == "alternate":
+        m = np.zeros((w.B, w.H, NT, NT), dtype=bool)
+        m[..., 0::2, 0::2] = True      # even query tiles see even key tiles, odd see odd
+        m[..., 1::2, 1::2] = True
+    else:
+        m = np.zeros((w.B, w.H, NT, NT), dtype=bool)
+        m[..., :, NT - 1] = True       # every row keeps only the last (partial) tile
+    out, lse, ref = _attn_with_mask(w, q, k, v, m)
+    st = C.compare_attention(w, out, lse, ref)
+    C.assert_attention_close(st)
+
+
+def test_attention_all_retained_equals_dense():
+    """All tiles retained: equals dense softmax attention over the raster sequence."""
+    bsa = _bsa()
+    w, q, k, v, _ = C.inputs("ragged128")
+    NT = w.NT
+    m = np.ones((w.B, w.H, NT, NT), dtype=bool)
+    out, lse, _ = _attn_with_mask(w, q, k, v, m, rows=[])
+    tq, tk, tv = (x.double().permute(0, 2, 1, 3) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv).permute(0, 2, 1, 3)
+    got = out.double().cpu()
+    rel = ((got - ref).norm() / ref.norm()).item()
+    assert rel <= C.O_REL_L2 and (got - ref).abs().max().item() <= C.O_MAX_ABS
+    s = torch.einsum("bhnd,bhmd->bhnm", tq, tk) / np.sqrt(w.d)
+    assert (lse.double().cpu() - torch.logsumexp(s, -1)).abs().max().item() <= C.LSE_ABS
+
+
+def test_attention_invariants():
+    """V = 1 gives O = 1; V changes in unretained tiles leave O bit-identical."""
+    bsa = _bsa()
+    w, q, k, v, _ = C.inputs("ragged128")
+    g = C.geometry(w)
+    NT = w.NT
+    rng = np.random.default_rng(5)
+    m = rng.random((w.B, w.H, NT, NT)) < 0.3
+    m[..., np.arange(NT), np.arange(NT)] = True
+    mask = torch.from_numpy(O.pack_bitmask(m).view(np.int32).copy()).cuda()
+    cnt = torch.from_numpy(m.sum(-1).astype(np.int32)).cuda()
+    qt, kt = bsa.reorder(g, q.cuda()), bsa.reorder(g, k.cuda())
+    ones = torch.ones((g.B, g.H, NT, 64, g.d), dtype=torch.bfloat16, device="cuda")
+    out, _ = bsa.sparse_attn_fwd(g, qt, kt, ones, mask, cnt)
+    assert (out.float() - 1).abs().max().item() < 1e-2
+    vt = bsa.reorder(g, v.cuda())
+    o1, l1 = bsa.sparse_attn_fwd(g, qt, kt, vt, mask, cnt)
+    # perturb V in tiles that no query tile of head 0 retains
+    unret = ~m[0, 0].any(axis=0)
+    vt2 = vt.clone()
+    idx = torch.from_numpy(np.nonzero(unret)[0]).cuda()
+    if idx.numel() == 0:
+        pytest.skip("every tile retained somewhere")
+    vt2[0, 0, idx] = vt2[0, 0, idx] * 3 + 1
+    o2, l2 = bsa.sparse_attn_fwd(g, qt, kt, vt2, mask, cnt)
+    assert torch.equal(o1[0, :, 0].view(torch.int16), o2[0, :, 0].view(torch.int16))
+    assert torch.equal(l1, l2)
+
+
+def test_attention_zero_query_mean_of_values():
+    bsa = _bsa()
+    w, q, k, v, _ = C.inputs("tiny_ragged")
+    NT = w.NT
+    rng = np.random.default_rng(6)
+    m = rng.random((w.B, w.H, NT, NT)) < 0.4
+    m[..., np.arange(NT), np.arange(NT)] = True
+    qz = torch.zeros_like(q)
+    out, lse, ref = _attn_with_mask(w, qz, k, v, m)
+    st = C.compare_attention(w, out, lse, ref)
+    C.assert_attention_close(st)
+    valid = O.slot_valid(w.T, w.Hs, w.Ws)
+    src = O.slot_tokens(w.T, w.Hs, w.Ws)
+    for i in range(NT):
+        nk = int(sum(valid[j].sum() for j in np.nonzero(m[0, 0, i])[0]))
+        toks = src[i][valid[i]]
+        assert np.allclose(lse[0, 0, toks].cpu().numpy(), np.log(nk), atol=1e-5)
+
+
+def test_attention_wan13b_sampled_rows():
+    """Full 1.3B-shaped call; oracle on sampled dense and local query tiles."""
+    w, q, k, v, diff = C.inputs("wan13b")
+    qt64, kt64 = (O.reorder(O.to_f64(x), w.T, w.Hs, w.Ws) for x in (q, k))
+    mref = C.oracle_mask(w, qt64, kt64, diff.numpy())
+    rng = np.random.default_rng(3)
+    dense_i = np.nonzero(mref["dense"][0])[0]
+    local_i = np.nonzero(~mref["dense"][0])[0]
+    rows = [(0, int(rng.integers(w.H)), int(i)) for i in rng.choice(dense_i, 6, replace=False)]
+    rows += [(0, int(rng.integers(w.H)), int(i)) for i in rng.choice(local_i, 18, replace=False)]
+    rows += [(0, w.H - 1, w.NT - 1), (0, 0, 0)]
+    out, lse, ref = _attn_with_mask(w, q, k, v, mref["mask"], rows=rows)
+    st = C.compare_attention(w, out, lse, ref)
+    print(st)
+    C.assert_attention_close(st)
+
+
+# ----------------------------------------------------------------------------- whole path
+@pytest.mark.parametrize("name", ["tiny_ragged", "small128", "budget128", "wan13b"])
+def test_forward_path(name):
+    """reorder -> build_mask -> sparse attention on the GPU vs the oracle's whole path."""
+    bsa = _bsa()
+    w, q, k, v, diff = C.inputs(name)
+    g = C.geometry(w)
+    b = bsa.forward(g, C.params(w), q.cuda(), k.cuda(), v.cuda(), diff.cuda())
+    torch.cuda.synchronize()
+    assert bsa.read_error(b.ws) == 0
+    qt64, kt64, vt64 = (O.reorder(O.to_f64(x), w.T, w.Hs, w.Ws) for x in (q, k, v))
+    mref = C.oracle_mask(w, qt64, kt64, diff.numpy())
+    cmp = C.compare_masks(C.gpu_mask_bool(b.mask, g.NT), mref)
+    assert cmp["n_unflagged"] == 0, cmp
+    if name == "wan13b":
+        rng = np.random.default_rng(11)
+        rows = [(0, int(rng.integers(w.H)), int(rng.integers(g.NT))) for _ in range(20)]
+    else:
+        rows = [(bb, h, i) for bb in range(w.B) for h in range(w.H) for i in range(g.NT)]
+    ref = O.attention_tiles(qt64, kt64, vt64, mref["mask"], rows, T=w.T, Hs=w.Hs, Ws=w.Ws)
+    st = C.compare_attention(w, b.out, b.lse, ref, skip_rows=cmp["diff_rows"])
+    print(name, st, cmp["n_diff"])
+    C.assert_attention_close(st)
