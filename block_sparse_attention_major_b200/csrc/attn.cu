@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int half = row >> 6;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const uint32_t o_tmem = tmem + 256 + lane_base;
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_run = -INFINITY, l_run = 0.f, lr_run = 0.f;
     bool ok = nblk > 0;
     for (int blk = 0; blk < nblk && ok; ++blk) {
       if (!warp_wait(sfull(blk & 1), (blk >> 1) & 1, abort, a.err)) { ok = false; break; }
@@ -314,7 +314,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float m_ref = grow ? m_new : m_run;
       const float alpha = grow ? exp2f(m_run - m_new) : 1.0f;
       const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-      float sum = 0.f;
+      // l_run sums the fp32 probabilities (for the LSE); lr_run sums the bf16-rounded
+      // ones that enter P.V, so that O is normalised by exactly the weights it used.
+      float sum = 0.f, sum_r = 0.f;
       uint32_t pk[64];
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
@@ -322,8 +324,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float p1 = exp2f(x[2 * c + 1] - m_use);
         sum += p0 + p1;
         pk[c] = pack_bf16x2(p0, p1);
+        sum_r += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
       }
       l_run = l_run * alpha + sum;
+      lr_run = lr_run * alpha + sum_r;
       if (has1) {
         tmem_st_x64(s_tmem, pk);
       } else {
@@ -362,7 +366,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int t = tt * 4 + (r >> 4), y = ty * 4 + ((r >> 2) & 3), xx = tx * 4 + (r & 3);
           if (t < g.T && y < g.Hs && xx < g.Ws) n = (t * g.Hs + y) * g.Ws + xx;
         }
-        const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
+        const float inv_l = lr_run > 0.f ? 1.0f / lr_run : 0.f;
         const int b = bh / g.H, h = bh - (bh / g.H) * g.H;
         uint4* dst = n >= 0 ? reinterpret_cast<uint4*>(a.out + (((long long)b * g.N + n) * g.H + h) * D) : nullptr;
 #pragma unroll 1

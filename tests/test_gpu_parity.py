@@ -184,7 +184,8 @@ def test_attention_all_retained_equals_dense():
     ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv).permute(0, 2, 1, 3)
     got = out.double().cpu()
     rel = ((got - ref).norm() / ref.norm()).item()
-    assert rel <= C.O_REL_L2 and (got - ref).abs().max().item() <= C.O_MAX_ABS
+    excess = (got - ref).abs().numpy() - C.bf16_half_ulp(ref.numpy())
+    assert rel <= C.O_REL_L2 and excess.max() <= C.O_MAX_ABS
     s = torch.einsum("bhnd,bhmd->bhnm", tq, tk) / np.sqrt(w.d)
     assert (lse.double().cpu() - torch.logsumexp(s, -1)).abs().max().item() <= C.LSE_ABS
 
@@ -198,6 +199,9 @@ def test_attention_invariants():
     rng = np.random.default_rng(5)
     m = rng.random((w.B, w.H, NT, NT)) < 0.3
     m[..., np.arange(NT), np.arange(NT)] = True
+    unret_set = [3, 7, 11, 17]                 # key tiles no query tile of head 0 retains
+    m[0, 0, :, unret_set] = False
+    m[0, 0, unret_set, 0] = True
     mask = torch.from_numpy(O.pack_bitmask(m).view(np.int32).copy()).cuda()
     cnt = torch.from_numpy(m.sum(-1).astype(np.int32)).cuda()
     qt, kt = bsa.reorder(g, q.cuda()), bsa.reorder(g, k.cuda())
