@@ -1,0 +1,456 @@
+"""Benchmark of the block-sparse video attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole path over one attention call of the Wan-1.3B-480p-shaped
+workload (B=1, 12 heads, d=128, 21x30x52 latent grid = 32,760 tokens, 20% of query tiles
+dense, the rest a decayed window of radius 2 plus the top-8 key tiles): reorder Q, K, V
+to tile-major, build the block mask, block-sparse attention with the output and LSE
+written back in raster order. Inputs are synthetic (seeded generator) and resident in HBM
+(302 MB of raster Q/K/V, larger than the 126 MB L2) when the timed region starts.
+
+The metric is effective TFLOP/s: 4*64*64*d FLOPs per retained (query tile, key tile) pair,
+divided by the device time of the step; `ms_per_step` gives the time per call.
+Under torchrun each rank runs its own copy of the call (independent problems, weak
+scaling, no collective on the data path); the time is the max over ranks.
+
+--impl reference times the CPU oracle (test infrastructure) on a bounded sample of the
+same workload on the host cores, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "wan13b"
+METRIC = "sparse-attn ms/call & effective TFLOP/s at ~20% tiles; % of B200 BF16 peak"
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def _dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(bf16=d["bf16_tflops"], bf16_sustained=d["bf16_tflops_sustained"],
+                    hbm=d["hbm_gbs"], source="measured")
+    return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+def _workload_desc(w, retention):
+    return {
+        "workload": (f"Wan-1.3B-480p-shaped attention call: B={w.B} heads={w.H} d={w.d} "
+                     f"grid {w.T}x{w.Hs}x{w.Ws} ({w.N} tokens, {w.NT} tiles of 4x4x4), "
+                     f"rho={w.dense_fraction} dense query tiles, decayed window r={w.radius} "
+                     f"+ top-{w.topk}"),
+        "global_batch": w.B,
+        "seq_len": w.N,
+        "retained_tile_fraction": round(retention, 4),
+        "l2": "inputs larger than L2 (raster Q/K/V 302 MB > 126 MB)",
+        "parallelism": "independent call per rank (weak scaling)",
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region (rank 0)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpus):
+        self.gpus = gpus
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", ",".join(str(g) for g in self.gpus)],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        with open(self.tmp.name) as f:
+            lines = [ln.strip() for ln in f if ln.strip()]
+        os.unlink(self.tmp.name)
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = max(smax, float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _attn_source_hash():
+    h = hashlib.sha256()
+    for f in ("attn.cu", "sm100_ptx.cuh", "tmem_ops.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_attention_major_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if it is current."""
+    p = os.path.join(ROOT, "profiles", "attn_kernel_wan13b_traffic.json")
+    if not os.path.exists(p):
+        return None, None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("attn_source_sha256_16") != _attn_source_hash():
+        return None, "kernel changed since the ncu capture"
+    return d.get("dram_bytes_per_launch"), d.get("source")
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+def _oracle_sample(w, q, k, v, diff, head, rows):
+    """Oracle path for one head: reorder, mask, attention of the listed query tiles.
+
+    Returns (seconds, retained tile pairs attended)."""
+    import numpy as np
+    from oracle import bsa_oracle as O
+    t0 = time.perf_counter()
+    qh, kh, vh = (O.to_f64(x[:, :, head:head + 1]) for x in (q, k, v))
+    qt, kt, vt = (O.reorder(x, w.T, w.Hs, w.Ws) for x in (qh, kh, vh))
+    m = O.build_mask(qt, kt, diff.numpy(), T=w.T, Hs=w.Hs, Ws=w.Ws, window_kind=w.window_kind,
+                     radius=w.radius, topk=w.topk, dense_fraction=w.dense_fraction,
+                     budget_mode=w.budget_mode, budget_target=w.budget_target)
+    O.attention_tiles(qt, kt, vt, m["mask"], [(0, 0, i) for i in rows], T=w.T, Hs=w.Hs, Ws=w.Ws)
+    dt = time.perf_counter() - t0
+    pairs = int(sum(int(m["mask"][0, 0, i].sum()) for i in rows))
+    return dt, pairs
+
+
+def _blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max((x.get("num_threads", 1) for x in info if x.get("user_api") == "blas"), default=1)
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def run_reference(args):
+    """Oracle timed on the host cores, rank 0 only.
+
+    Setup (timed once): reorder of Q, K, V and the mask of the whole call. Each step then
+    attends a chunk of query tiles (a seeded shuffle of every (head, tile) row), taking rows
+    until the step's time budget of about 120 s / (steps + warmup) is used. A step is
+    charged its attention time plus the setup time in proportion to the retained tile
+    pairs it attended, so that the sum over all rows of the call would be the full call.
+    """
+    rank, world, _ = _dist_env()
+    if rank != 0:
+        return 0
+    import numpy as np
+    from bsa_synth import WORKLOADS, generate_difficulty, generate_qkv
+    from oracle import bsa_oracle as O
+    w = WORKLOADS[WORKLOAD]
+    q, k, v = generate_qkv(w)
+    diff = generate_difficulty(w)
+    t0 = time.perf_counter()
+    qt, kt, vt = (O.reorder(O.to_f64(x), w.T, w.Hs, w.Ws) for x in (q, k, v))
+    m = O.build_mask(qt, kt, diff.numpy(), T=w.T, Hs=w.Hs, Ws=w.Ws, window_kind=w.window_kind,
+                     radius=w.radius, topk=w.topk, dense_fraction=w.dense_fraction,
+                     budget_mode=w.budget_mode, budget_target=w.budget_target)
+    t_setup = time.perf_counter() - t0
+    counts = m["mask"].sum(-1)
+    pairs_call = int(counts.sum())
+    flop_pair = 4 * 64 * 64 * w.d
+    rows = [(0, h, i) for h in range(w.H) for i in range(w.NT)]
+    order = np.random.default_rng(7).permutation(len(rows))
+    budget = min(5.0, max(0.05, 120.0 / (args.steps + args.warmup)))
+    cursor = 0
+    times, flops = [], []
+    for s in range(args.warmup + args.steps):
+        t_attn, pairs = 0.0, 0
+        while t_attn < budget:
+            b, h, i = rows[order[cursor % len(rows)]]
+            cursor += 1
+            t1 = time.perf_counter()
+            O.attention_tiles(qt, kt, vt, m["mask"], [(b, h, i)], T=w.T, Hs=w.Hs, Ws=w.Ws)
+            t_attn += time.perf_counter() - t1
+            pairs += int(counts[b, h, i])
+        if s >= args.warmup:
+            times.append(t_attn + t_setup * pairs / pairs_call)
+            flops.append(pairs * flop_pair)
+    total_t = sum(times)
+    value = sum(flops) / total_t / 1e12
+    ms = 1e3 * total_t / len(times)
+    sample = (f"oracle on the whole call's reorder + mask ({t_setup:.1f} s, charged to the steps "
+              f"by retained pairs) and, per step, attention of seeded-shuffled (head, query "
+              f"tile) rows for about {budget:.2f} s; value = FLOPs of the attended retained "
+              "tile pairs / charged time")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _workload_desc(w, pairs_call / counts.size / w.NT),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------ GPU path
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_attention_major_b200 as bsa
+    from bsa_synth import WORKLOADS, generate_difficulty, generate_qkv
+
+    rank, world, local = _dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+
+    w = WORKLOADS[WORKLOAD]
+    q_h, k_h, v_h = generate_qkv(w)
+    diff_h = generate_difficulty(w)
+    g = bsa.Geometry(w.B, w.H, w.d, w.T, w.Hs, w.Ws)
+    p = bsa.MaskParams(w.window_kind, w.radius, w.topk, w.dense_fraction, w.budget_mode,
+                       w.budget_target)
+    q, k, v, diff = (x.to(dev) for x in (q_h, k_h, v_h, diff_h))
+    bufs = bsa.Buffers(g, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # one untimed call to learn the retained tile count (the mask is deterministic)
+    bsa.forward(g, p, q, k, v, diff, bufs)
+    torch.cuda.synchronize(dev)
+    if bsa.read_error(bufs.ws) != 0:
+        raise SystemExit("kernel error word set")
+    retained = int(bufs.kv_count.sum().item())
+    dense_pairs = g.B * g.H * g.NT * g.NT
+    flops_call = 4.0 * 64 * 64 * g.d * retained
+    retention = retained / dense_pairs
+
+    # ---------------------------------------------------------------- device-timed steps
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    attn_ev = [(ev(), ev()) for _ in range(args.steps)]
+    for _ in range(args.warmup):
+        bsa.forward(g, p, q, k, v, diff, bufs)
+    sampler = ClockSampler(list(range(world))) if rank == 0 else None
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    n0 = bsa.launch_count()
+    t_start, t_end = ev(), ev()
+    t_start.record(stream)
+    for s in range(args.steps):
+        bsa.reorder(g, q, bufs.qt)
+        bsa.reorder(g, k, bufs.kt)
+        bsa.reorder(g, v, bufs.vt)
+        bsa.build_mask(g, p, bufs.qt, bufs.kt, diff, bufs.mask, bufs.kv_count, bufs.ws)
+        attn_ev[s][0].record(stream)
+        bsa.sparse_attn_fwd(g, bufs.qt, bufs.kt, bufs.vt, bufs.mask, bufs.kv_count, None,
+                            bufs.out, bufs.lse, bufs.ws)
+        attn_ev[s][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = bsa.launch_count() - n0
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop() if sampler else None
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in attn_ev]))
+    attn_ms = max_over_ranks(attn_ms)
+    ms_step = elapsed_ms / args.steps
+    total_flops = sum_over_ranks(flops_call) * args.steps
+    value = total_flops / (elapsed_ms * 1e-3) / 1e12
+    if bsa.read_error(bufs.ws) != 0:
+        raise SystemExit("kernel error word set")
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        q_p, k_p, v_p, d_p = (x.pin_memory() for x in (q_h, k_h, v_h, diff_h))
+        out_p = torch.empty(bufs.out.shape, dtype=bufs.out.dtype).pin_memory()
+        lse_p = torch.empty(bufs.lse.shape, dtype=bufs.lse.dtype).pin_memory()
+        qd, kd, vd, dd = (torch.empty_like(x, device=dev) for x in (q_h, k_h, v_h, diff_h))
+        e2e_steps = max(3, min(args.steps, 60))
+
+        def e2e_step():
+            qd.copy_(q_p, non_blocking=True)
+            kd.copy_(k_p, non_blocking=True)
+            vd.copy_(v_p, non_blocking=True)
+            dd.copy_(d_p, non_blocking=True)
+            bsa.forward(g, p, qd, kd, vd, dd, bufs)
+            out_p.copy_(bufs.out, non_blocking=True)
+            lse_p.copy_(bufs.lse, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        torch.cuda.synchronize(dev)
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_ms = max_over_ranks(a.elapsed_time(b))
+        h2d = sum(x.numel() * x.element_size() for x in (q_h, k_h, v_h, diff_h))
+        d2h = out_p.numel() * out_p.element_size() + lse_p.numel() * lse_p.element_size()
+        e2e = {"value": sum_over_ranks(flops_call) * e2e_steps / (e2e_ms * 1e-3) / 1e12,
+               "unit": "TFLOP/s", "ms_per_step": e2e_ms / e2e_steps,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    # ---------------------------------------------------------------- own dense path (rho = 1)
+    pd = bsa.MaskParams(w.window_kind, w.radius, w.topk, 1.0, 0, 0.0)
+    bsa.build_mask(g, pd, bufs.qt, bufs.kt, diff, bufs.mask, bufs.kv_count, bufs.ws)
+    for _ in range(3):
+        bsa.sparse_attn_fwd(g, bufs.qt, bufs.kt, bufs.vt, bufs.mask, bufs.kv_count, None,
+                            bufs.out, bufs.lse, bufs.ws)
+    torch.cuda.synchronize(dev)
+    a, b = ev(), ev()
+    nd = 10
+    a.record(stream)
+    for _ in range(nd):
+        bsa.sparse_attn_fwd(g, bufs.qt, bufs.kt, bufs.vt, bufs.mask, bufs.kv_count, None,
+                            bufs.out, bufs.lse, bufs.ws)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    dense_ms = max_over_ranks(a.elapsed_time(b) / nd)
+    dense_tflops = 4.0 * 64 * 64 * g.d * dense_pairs / (dense_ms * 1e-3) / 1e12
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks = _peaks()
+    timed_s = elapsed_ms * 1e-3
+    peak_kind = "sustained" if timed_s > 1.0 else "burst"
+    peak = peaks["bf16_sustained"] if peak_kind == "sustained" else peaks["bf16"]
+    attn_tflops = flops_call / (attn_ms * 1e-3) / 1e12
+    traffic, traffic_src = _traffic()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": _workload_desc(w, retention),
+        "attn_ms_per_call": attn_ms,
+        "attn_effective_tflops": attn_tflops,
+        "attn_frac_of_nominal_bf16_peak": attn_tflops / NOMINAL_BF16_TFLOPS,
+        "dense_path": {"ms_per_call": dense_ms, "effective_tflops": dense_tflops,
+                       "sparse_speedup": dense_ms / attn_ms},
+        "roofline": {"kernel": "attn_kernel (+3 scheduler kernels in the same call)",
+                     "bound": "tensor", "achieved": attn_tflops, "peak": peak,
+                     "peak_kind": f"{peak_kind} bf16 GEMM, {peaks['source']}",
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak, "traffic": traffic,
+                     "traffic_source": traffic_src},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        heads = [0]
+        t_cpu, pairs = 0.0, 0
+        for hh in heads:
+            dt, pr = _oracle_sample(w, q_h, k_h, v_h, diff_h, hh, list(range(w.NT)))
+            t_cpu += dt
+            pairs += pr
+        line["cpu_baseline"] = {
+            "value": pairs * 4.0 * 64 * 64 * w.d / t_cpu / 1e12, "unit": "TFLOP/s",
+            "cores": _blas_threads(), "kind": "oracle",
+            "sample": (f"oracle path (reorder, mask, attention of all {w.NT} query tiles) for "
+                       f"head 0 of {w.H}: {pairs} retained tile pairs in {t_cpu:.1f} s")}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -128,7 +128,7 @@ def generate_qkv(w: Workload) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor]
     out = []
     for p in proj:
         eps = rng.standard_normal((w.B, w.N, w.H, w.d), dtype=np.float32)
-        base = np.einsum("nf,hfd->nhd", feats, p, optimize=True).astype(np.float32)
+        base = (feats @ p.transpose(1, 0, 2).reshape(19, w.H * w.d)).reshape(w.N, w.H, w.d)
         x = eps
         x *= np.float32(w.noise_std)
         x += base[None]
