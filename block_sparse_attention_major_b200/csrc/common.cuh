@@ -58,9 +58,10 @@ struct FastDiv {
 // [0, 256)        header: error word (u32 @0), attention unit count (i32 @4)
 // then 256-aligned regions: qbar, kbar (fp32 [B,H,NT,d]), dense flags (u8 [B,NT]),
 // row entropy (fp32 [B,H,NT]), per-(b,h) unit counts/offsets (int4 [B*H]),
-// attention units (int4 [B*H*(ceil(NT/2)+1)]).
-// Upper bound on attention work units: per (b, h), ceil(nd/2) + ceil(nl/2) <= NT/2 + 1.
-inline __host__ __device__ int units_per_bh(int NT) { return NT / 2 + 1; }
+// attention units (8 ints each, [B*H*(NT/4+2)]).
+// Upper bound on attention work units (four query tiles each): per (b, h),
+// ceil(nd/4) + ceil(nl/4) <= NT/4 + 2.
+inline __host__ __device__ int units_per_bh(int NT) { return NT / 4 + 2; }
 
 struct WsLayout {
   size_t qbar, kbar, dense, entropy, bhcnt, units, total;
@@ -77,7 +78,7 @@ inline WsLayout ws_layout(const Geom& g) {
   L.dense = off; off = align256(off + (size_t)g.B * g.NT);
   L.entropy = off; off = align256(off + (size_t)g.B * g.H * g.NT * sizeof(float));
   L.bhcnt = off; off = align256(off + (size_t)g.B * g.H * 4 * sizeof(int));
-  L.units = off; off = align256(off + (size_t)g.B * g.H * units_per_bh(g.NT) * 4 * sizeof(int));
+  L.units = off; off = align256(off + (size_t)g.B * g.H * units_per_bh(g.NT) * 8 * sizeof(int));
   L.total = off;
   return L;
 }
