@@ -55,6 +55,7 @@ constexpr int kUnitInts = 8;                       // {bh, q0, q1, q2, q3, 0, 0,
 
 template <int D>
 struct Cfg {
+  static constexpr int kD = D;
   static constexpr int kTileBytes = 64 * D * 2;         // one 64-token tile
   static constexpr int kBufBytes = 2 * kTileBytes;      // two tiles (128 rows)
   static constexpr int kDBlockStride = 128 * 128;       // bytes between 64-column blocks
@@ -67,7 +68,8 @@ struct Cfg {
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;         // tmem base, counts, abort
   static constexpr int kListOff = kMiscOff + 64;
   static constexpr int kBlkOff = kListOff + kMaxTiles * 4;        // uint16 block lists A, B
-  static constexpr int kSmemBytes = 1024 + kBlkOff + 2 * kMaxBlocks * 2;
+  static constexpr int kNeedOff = kBlkOff + 2 * kMaxBlocks * 2;   // uint8 per block
+  static constexpr int kSmemBytes = 1024 + kNeedOff + kMaxBlocks;
 };
 
 struct AttnArgs {
@@ -103,25 +105,29 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, ok);
 }
 
-// Mask 64 score columns of key tile `e` (a list entry) for this thread's query row: all
-// -inf when the row's query tile does not retain the tile, the tile's padding slots -inf
-// otherwise. Both conditions are warp-uniform, so full retained tiles cost one test.
-__device__ __forceinline__ void mask_tile(uint32_t (&r)[64], uint32_t e, int mshift, const Geom& g) {
-  constexpr uint32_t kNegInf = 0xff800000u;
-  if (!((e >> mshift) & 1u)) {
-#pragma unroll
-    for (int c = 0; c < 64; ++c) r[c] = kNegInf;
-  } else if (!((e >> 20) & 1u)) {
-    int tt, ty, tx;
-    tile_xyz(g, (int)(e & 0xffffu), tt, ty, tx);
-    const uint64_t valid = tile_valid_mask(g, tt, ty, tx);
-    const uint32_t lo = (uint32_t)valid, hi = (uint32_t)(valid >> 32);
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      r[c] = ((lo >> c) & 1u) ? r[c] : kNegInf;
-      r[32 + c] = ((hi >> c) & 1u) ? r[32 + c] : kNegInf;
-    }
-  }
+// How one key tile's 64 score columns enter this thread's row (warp-uniform): all of them
+// (the row's query tile retains the tile and the tile has no padding), only the valid
+// slots (a retained edge tile), or none (the tile is not retained by this row's query
+// tile: its probabilities are zero). The scores themselves are never rewritten, so the
+// three paths share the registers the TMEM load filled.
+enum TileUse { kUseFull = 0, kUsePartial = 1, kUseSkip = 2 };
+
+// 64 score columns as two 32-column TMEM loads (32-register destination ranges are easier
+// for the register allocator to place than one 64-register range).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  tmem_ld_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  tmem_ld_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+}
+
+__device__ __forceinline__ int tile_use(uint32_t e, int mshift) {
+  if (!((e >> mshift) & 1u)) return kUseSkip;
+  return ((e >> 20) & 1u) ? kUseFull : kUsePartial;
+}
+
+__device__ __forceinline__ uint64_t entry_valid_mask(uint32_t e, const Geom& g) {
+  int tt, ty, tx;
+  tile_xyz(g, (int)(e & 0xffffu), tt, ty, tx);
+  return tile_valid_mask(g, tt, ty, tx);
 }
 
 // Row maximum with four independent chains (short dependency chains for the scheduler).
@@ -137,25 +143,153 @@ __device__ __forceinline__ float row_max64(const uint32_t (&r)[64], float m) {
   return fmaxf(max3(a0, a1, a2), a3);
 }
 
-// p = 2^(s*c - m) for 64 columns; accumulates the fp32 sum and packs the bf16 pairs into
-// pk (column 2i in the low half of pk[i]).
-__device__ __forceinline__ void exp_pack64(const uint32_t (&r)[64], float c, float m, float& sum,
-                                           uint32_t (&pk)[32]) {
+// Same over the valid slots only (bit c of `valid` set).
+__device__ __forceinline__ float row_max64_valid(const uint32_t (&r)[64], uint64_t valid, float m) {
+  const uint32_t lo = (uint32_t)valid, hi = (uint32_t)(valid >> 32);
+  float a0 = m, a1 = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    a0 = fmaxf(a0, ((lo >> c) & 1u) ? __uint_as_float(r[c]) : -INFINITY);
+    a1 = fmaxf(a1, ((hi >> c) & 1u) ? __uint_as_float(r[32 + c]) : -INFINITY);
+  }
+  return fmaxf(a0, a1);
+}
+
+// p = 2^(s*c - m) for 64 columns (zero on slots whose bit in `valid` is clear), added to
+// the fp32 row sum and stored to TMEM as bf16 pairs (column 2i in the low half of 32-bit
+// column i), 16 columns per store.
+template <bool kMasked>
+__device__ __forceinline__ void exp_store64(const uint32_t (&r)[64], uint64_t valid, float c, float m,
+                                            float& sum, uint32_t taddr) {
+  const uint32_t lo = (uint32_t)valid, hi = (uint32_t)(valid >> 32);
   float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;       // four short chains
 #pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    const float p0 = ex2(fmaf(__uint_as_float(r[2 * i]), c, -m));
-    const float p1 = ex2(fmaf(__uint_as_float(r[2 * i + 1]), c, -m));
-    const float p2 = ex2(fmaf(__uint_as_float(r[2 * i + 2]), c, -m));
-    const float p3 = ex2(fmaf(__uint_as_float(r[2 * i + 3]), c, -m));
-    pk[i] = pack_bf16x2(p0, p1);
-    pk[i + 1] = pack_bf16x2(p2, p3);
-    s0 += p0;
-    s1 += p1;
-    s2 += p2;
-    s3 += p3;
+  for (int k = 0; k < 4; ++k) {
+    uint32_t pk[8];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      const int b = 16 * k + 2 * i;
+      float p0 = ex2(fmaf(__uint_as_float(r[b + 0]), c, -m));
+      float p1 = ex2(fmaf(__uint_as_float(r[b + 1]), c, -m));
+      float p2 = ex2(fmaf(__uint_as_float(r[b + 2]), c, -m));
+      float p3 = ex2(fmaf(__uint_as_float(r[b + 3]), c, -m));
+      if (kMasked) {
+        const uint32_t w = b < 32 ? lo : hi;
+        const int sh = b & 31;
+        p0 = ((w >> sh) & 1u) ? p0 : 0.f;
+        p1 = ((w >> (sh + 1)) & 1u) ? p1 : 0.f;
+        p2 = ((w >> (sh + 2)) & 1u) ? p2 : 0.f;
+        p3 = ((w >> (sh + 3)) & 1u) ? p3 : 0.f;
+      }
+      pk[i] = pack_bf16x2(p0, p1);
+      pk[i + 1] = pack_bf16x2(p2, p3);
+      s0 += p0;
+      s1 += p1;
+      s2 += p2;
+      s3 += p3;
+    }
+    tmem_st_x8(taddr + 8 * k, pk);
   }
   sum += (s0 + s1) + (s2 + s3);
+}
+
+// Zero probabilities for a tile the row does not retain (32 TMEM columns of bf16 pairs).
+__device__ __forceinline__ void store_zero_p(uint32_t taddr) {
+  uint32_t z[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) z[i] = 0u;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) tmem_st_x8(taddr + 8 * k, z);
+}
+
+// Max over one key tile's columns for this row, by its use.
+__device__ __forceinline__ float tile_max(const uint32_t (&r)[64], int use, uint64_t valid, float m) {
+  if (use == kUseFull) return row_max64(r, m);
+  if (use == kUsePartial) return row_max64_valid(r, valid, m);
+  return m;
+}
+
+// Probabilities of one key tile into TMEM, by its use.
+__device__ __forceinline__ void tile_exp(const uint32_t (&r)[64], int use, uint64_t valid, float c, float m,
+                                         float& sum, uint32_t taddr) {
+  if (use == kUseFull) exp_store64<false>(r, 0ull, c, m, sum, taddr);
+  else if (use == kUsePartial) exp_store64<true>(r, valid, c, m, sum, taddr);
+  else store_zero_p(taddr);
+}
+
+// O *= alpha for this thread's row of the D accumulator columns, 32 columns per TMEM
+// round trip.
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t o_tmem, float alpha) {
+#pragma unroll
+  for (int h = 0; h < D / 32; ++h) {
+    uint32_t o[32];
+    tmem_ld_x32(o_tmem + 32 * h, o);
+    ptx::tmem_wait_ld();
+#pragma unroll
+    for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+    tmem_st_x32(o_tmem + 32 * h, o);
+  }
+}
+
+// MMA-issue state of one sub-unit: block whose P.V is pending (-1: none), the tile slots
+// it uses, and the number of P.V products issued so far.
+struct SubUnitIssue {
+  int pend;
+  uint32_t pneed;
+  int npv;
+};
+
+// What the MMA-issuing thread needs: TMEM base, descriptors of the Q / K / V stage bases
+// (an offset of x bytes adds x >> 4 to a descriptor), barrier addresses.
+struct MmaCtx {
+  uint32_t tmem;
+  uint64_t dQ0, dK0, dV0;
+  uint32_t pfull0, vfull0, vempty0, sfull0, odone0;
+  volatile int* abort;
+  uint32_t* err;
+};
+
+// O_u += P_u V for the pending block of sub-unit u, then release its V stage once no other
+// product still reads it.
+template <class C>
+__device__ __forceinline__ bool issue_pv(SubUnitIssue& st, int u, const MmaCtx& m, int& vref0, int& vref1) {
+  constexpr uint32_t kIdPV = ptx::idesc_bf16_f32(128, C::kD, 0, 1);
+  const int j = st.pend;
+  const int sv = j & 1;
+  if (!ptx::mbar_wait(m.pfull0 + 8 * u, st.npv & 1, m.abort, m.err, kWaitLimit)) return false;
+  if (!ptx::mbar_wait(m.vfull0 + 8 * sv, (j >> 1) & 1, m.abort, m.err, kWaitLimit)) return false;
+  ptx::tc_fence_after();
+  const uint32_t p_tmem = m.tmem + 128 * u;
+  const uint32_t o_tmem = m.tmem + 256 + 128 * u;
+  const uint64_t vd = m.dV0 + sv * (C::kBufBytes >> 4) + (st.pneed == 2u ? (8192u >> 4) : 0u);
+  const int nk = (st.pneed == 3u) ? 8 : 4;
+  for (int kk = 0; kk < nk; ++kk)
+    ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + kk * (2048 >> 4), kIdPV, (st.npv > 0 || kk > 0) ? 1u : 0u);
+  ptx::mma_commit(m.odone0 + 8 * u);
+  ++st.npv;
+  const int left = sv ? --vref1 : --vref0;
+  if (left == 0) ptx::mma_commit(m.vempty0 + 8 * sv);
+  st.pend = -1;
+  return true;
+}
+
+// S_u = Q_u K^T on the needed tile slots n of block j.
+template <class C, int D>
+__device__ __forceinline__ void issue_qk(SubUnitIssue& st, int u, int j, uint32_t n, const MmaCtx& m) {
+  constexpr uint32_t kIdQK128 = ptx::idesc_bf16_f32(128, 128, 0, 0);
+  constexpr uint32_t kIdQK64 = ptx::idesc_bf16_f32(128, 64, 0, 0);
+  const uint64_t qd = m.dQ0 + u * (C::kBufBytes >> 4);
+  const uint64_t kd = m.dK0 + (j & 1) * (C::kBufBytes >> 4) + (n == 2u ? (8192u >> 4) : 0u);
+  const uint32_t id = n == 3u ? kIdQK128 : kIdQK64;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = ((kk >> 2) * C::kDBlockStride + (kk & 3) * 32) >> 4;
+    ptx::mma_ss(m.tmem + 128 * u, qd + off, kd + off, id, kk > 0 ? 1u : 0u);
+  }
+  ptx::mma_commit(m.sfull0 + 8 * u);
+  st.pend = j;
+  st.pneed = n;
 }
 
 template <int D>
@@ -173,41 +307,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if ((int)blockIdx.x >= a.header[1]) return;
   const int* up = a.units + (size_t)blockIdx.x * kUnitInts;
   const int bh = up[0];
-  int q[4];
-#pragma unroll
-  for (int t = 0; t < 4; ++t) q[t] = up[1 + t];
-  bool bad = bh < 0 || bh >= g.B * g.H || q[0] < 0;
-#pragma unroll
-  for (int t = 0; t < 4; ++t) bad = bad || q[t] >= g.NT || q[t] < -1;
+  const int q0 = up[1], q1 = up[2], q2 = up[3], q3 = up[4];
+  const bool bad = bh < 0 || bh >= g.B * g.H || q0 < 0 || q0 >= g.NT || q1 >= g.NT || q2 >= g.NT ||
+                   q3 >= g.NT || q1 < -1 || q2 < -1 || q3 < -1;
   if (bad) {
     if (threadIdx.x == 0) report_error(a.err, BSA_KERR_BAD_UNIT);
     return;
   }
-  const bool hasB = q[2] >= 0;
+  const bool hasB = q2 >= 0;
 
-  const uint32_t bar_q = sbase + C::kBarOff;
-  auto kfull = [&](int s) { return sbase + C::kBarOff + 8 * (1 + s); };
-  auto kempty = [&](int s) { return sbase + C::kBarOff + 8 * (1 + kNSK + s); };
-  auto vfull = [&](int s) { return sbase + C::kBarOff + 8 * (1 + 2 * kNSK + s); };
-  auto vempty = [&](int s) { return sbase + C::kBarOff + 8 * (1 + 2 * kNSK + kNSV + s); };
-  auto sfull = [&](int u) { return sbase + C::kBarOff + 8 * (1 + 2 * kNSK + 2 * kNSV + u); };
-  auto pfull = [&](int u) { return sbase + C::kBarOff + 8 * (3 + 2 * kNSK + 2 * kNSV + u); };
-  auto odone = [&](int u) { return sbase + C::kBarOff + 8 * (5 + 2 * kNSK + 2 * kNSV + u); };
-  const uint32_t bar_drain = sbase + C::kBarOff + 8 * (7 + 2 * kNSK + 2 * kNSV);
+  const uint32_t bar0 = sbase + C::kBarOff;
+  // barrier addresses: q, kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], pfull[2], odone[2], drain
+  const uint32_t bar_q = bar0;
+  const uint32_t kfull0 = bar0 + 8, kempty0 = bar0 + 24, vfull0 = bar0 + 40, vempty0 = bar0 + 56;
+  const uint32_t sfull0 = bar0 + 72, pfull0 = bar0 + 88, odone0 = bar0 + 104, bar_drain = bar0 + 120;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   int* counts = reinterpret_cast<int*>(smem + C::kMiscOff + 4);        // L, cntA, cntB
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 16);
   uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::kListOff);
   uint16_t* blk = reinterpret_cast<uint16_t*>(smem + C::kBlkOff);      // [2][kMaxBlocks]
+  uint8_t* needs = smem + C::kNeedOff;                                  // per block: nA | nB << 2
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar_q, 1);
-    for (int s = 0; s < kNSK; ++s) { ptx::mbar_init(kfull(s), 1); ptx::mbar_init(kempty(s), 1); }
-    for (int s = 0; s < kNSV; ++s) { ptx::mbar_init(vfull(s), 1); ptx::mbar_init(vempty(s), 1); }
-    for (int u = 0; u < 2; ++u) {
-      ptx::mbar_init(sfull(u), 1);
-      ptx::mbar_init(pfull(u), 128);
-      ptx::mbar_init(odone(u), 1);
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(kfull0 + 8 * s, 1);
+      ptx::mbar_init(kempty0 + 8 * s, 1);
+      ptx::mbar_init(vfull0 + 8 * s, 1);
+      ptx::mbar_init(vempty0 + 8 * s, 1);
+      ptx::mbar_init(sfull0 + 8 * s, 1);
+      ptx::mbar_init(pfull0 + 8 * s, 128);
+      ptx::mbar_init(odone0 + 8 * s, 1);
     }
     ptx::mbar_init(bar_drain, 1);
     *abort = 0;
@@ -218,27 +348,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     ptx::tmem_relinquish();
   }
   if (warp == 8) {
-    // Union of the four rows' key tiles, ascending; bit 16+t: retained by query tile q[t];
+    // Union of the four rows' key tiles, ascending; bit 16+t: retained by query tile q_t;
     // bit 20: the tile has no padding slot.
     if (lane == 0) {
       ptx::prefetch_tensormap(&tmQ);
       ptx::prefetch_tensormap(&tmK);
       ptx::prefetch_tensormap(&tmV);
     }
-    const uint32_t* mrow[4];
-#pragma unroll
-    for (int t = 0; t < 4; ++t) mrow[t] = a.mask + ((long long)bh * g.NT + (q[t] >= 0 ? q[t] : q[0])) * g.NW;
+    const long long rbase = (long long)bh * g.NT;
+    const uint32_t* m0 = a.mask + (rbase + q0) * g.NW;
+    const uint32_t* m1 = a.mask + (rbase + (q1 >= 0 ? q1 : q0)) * g.NW;
+    const uint32_t* m2 = a.mask + (rbase + (q2 >= 0 ? q2 : q0)) * g.NW;
+    const uint32_t* m3 = a.mask + (rbase + (q3 >= 0 ? q3 : q0)) * g.NW;
     int running = 0;
     for (int w0 = 0; w0 < g.NW; w0 += 32) {
       const int w = w0 + lane;
-      uint32_t b[4] = {0u, 0u, 0u, 0u};
+      uint32_t b0 = 0u, b1 = 0u, b2 = 0u, b3 = 0u;
       if (w < g.NW) {
         const int rem = g.NT - 32 * w;
         const uint32_t keep = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
-#pragma unroll
-        for (int t = 0; t < 4; ++t) b[t] = q[t] >= 0 ? (__ldg(&mrow[t][w]) & keep) : 0u;
+        b0 = __ldg(&m0[w]) & keep;
+        b1 = q1 >= 0 ? (__ldg(&m1[w]) & keep) : 0u;
+        b2 = q2 >= 0 ? (__ldg(&m2[w]) & keep) : 0u;
+        b3 = q3 >= 0 ? (__ldg(&m3[w]) & keep) : 0u;
       }
-      uint32_t u = b[0] | b[1] | b[2] | b[3];
+      uint32_t u = b0 | b1 | b2 | b3;
       const int cnt = __popc(u);
       int incl = cnt;
 #pragma unroll
@@ -254,13 +388,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         int tt, ty, tx;
         tile_xyz(g, j, tt, ty, tx);
         const uint32_t full = tile_valid_count(g, tt, ty, tx) == 64 ? 1u : 0u;
-        list[pos++] = (uint32_t)j | (((b[0] >> bit) & 1u) << 16) | (((b[1] >> bit) & 1u) << 17) |
-                      (((b[2] >> bit) & 1u) << 18) | (((b[3] >> bit) & 1u) << 19) | (full << 20);
+        list[pos++] = (uint32_t)j | (((b0 >> bit) & 1u) << 16) | (((b1 >> bit) & 1u) << 17) |
+                      (((b2 >> bit) & 1u) << 18) | (((b3 >> bit) & 1u) << 19) | (full << 20);
       }
       running += __shfl_sync(0xffffffffu, incl, 31);
     }
     __syncwarp();
-    // Per-sub-unit block lists: entry = block | need << 12, need bit t = tile slot t used.
+    // Per-sub-unit block lists (entry = block | need << 12) and per-block needs, where
+    // need bit t = tile slot t of the block is retained by one of the sub-unit's tiles.
     const int L = running, nblk = (L + 1) >> 1;
     int ca = 0, cb = 0;
     for (int j0 = 0; j0 < nblk; j0 += 32) {
@@ -271,6 +406,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t e1 = (2 * j + 1 < L) ? list[2 * j + 1] : 0u;
         na = (((e0 >> 16) & 3u) ? 1u : 0u) | (((e1 >> 16) & 3u) ? 2u : 0u);
         nb = (((e0 >> 18) & 3u) ? 1u : 0u) | (((e1 >> 18) & 3u) ? 2u : 0u);
+        needs[j] = (uint8_t)(na | (nb << 2));
       }
       const uint32_t ba = __ballot_sync(0xffffffffu, na != 0), bb = __ballot_sync(0xffffffffu, nb != 0);
       const uint32_t lt = (1u << lane) - 1u;
@@ -297,120 +433,89 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && nblk > 0) {
-      int last_k[kNSK], last_v[kNSV];
-      for (int s = 0; s < kNSK; ++s) last_k[s] = -1;
-      for (int s = 0; s < kNSV; ++s) last_v[s] = -1;
+      int last_k0 = -1, last_k1 = -1, last_v0 = -1, last_v1 = -1;
       const int nsub = hasB ? 2 : 1;
       ptx::mbar_arrive_expect_tx(bar_q, nsub * C::kBufBytes);
-      for (int u = 0; u < nsub; ++u)
-        for (int half = 0; half < 2; ++half) {
-          const int tile = q[2 * u + half] >= 0 ? q[2 * u + half] : q[2 * u];
-          const int row = (int)((tile_row0 + tile) * 64);
-          for (int db = 0; db < D / 64; ++db)
-            ptx::tma_load_2d(sbase + C::kQOff + u * C::kBufBytes + db * C::kDBlockStride + half * 8192, &tmQ,
-                             bar_q, db * 64, row);
-        }
+      for (int t = 0; t < 2 * nsub; ++t) {
+        const int qt = t == 0 ? q0 : t == 1 ? q1 : t == 2 ? q2 : q3;
+        const int tile = qt >= 0 ? qt : (t < 2 ? q0 : q2);
+        const int row = (int)((tile_row0 + tile) * 64);
+        const uint32_t dst = sbase + C::kQOff + (t >> 1) * C::kBufBytes + (t & 1) * 8192;
+#pragma unroll
+        for (int db = 0; db < D / 64; ++db) ptx::tma_load_2d(dst + db * C::kDBlockStride, &tmQ, bar_q, db * 64, row);
+      }
       for (int j = 0; j < nblk; ++j) {
         const int nt = (2 * j + 1 < L) ? 2 : 1;
-        const int sk = j % kNSK;
-        if (!ptx::mbar_wait(kempty(sk), ((j / kNSK) & 1) ^ 1, abort, a.err, kWaitLimit)) break;
-        ptx::mbar_arrive_expect_tx(kfull(sk), nt * C::kTileBytes);
+        const int s = j & 1;
+        const uint32_t ph = ((j >> 1) & 1) ^ 1;
+        if (!ptx::mbar_wait(kempty0 + 8 * s, ph, abort, a.err, kWaitLimit)) break;
+        ptx::mbar_arrive_expect_tx(kfull0 + 8 * s, nt * C::kTileBytes);
         for (int t = 0; t < nt; ++t) {
           const int row = (int)((tile_row0 + (int)(list[2 * j + t] & 0xffffu)) * 64);
+          const uint32_t dst = sbase + C::kKOff + s * C::kBufBytes + t * 8192;
+#pragma unroll
           for (int db = 0; db < D / 64; ++db)
-            ptx::tma_load_2d(sbase + C::kKOff + sk * C::kBufBytes + db * C::kDBlockStride + t * 8192, &tmK,
-                             kfull(sk), db * 64, row);
+            ptx::tma_load_2d(dst + db * C::kDBlockStride, &tmK, kfull0 + 8 * s, db * 64, row);
         }
-        last_k[sk] = j;
-        const int sv = j % kNSV;
-        if (!ptx::mbar_wait(vempty(sv), ((j / kNSV) & 1) ^ 1, abort, a.err, kWaitLimit)) break;
-        ptx::mbar_arrive_expect_tx(vfull(sv), nt * C::kTileBytes);
+        if (s) last_k1 = j; else last_k0 = j;
+        if (!ptx::mbar_wait(vempty0 + 8 * s, ph, abort, a.err, kWaitLimit)) break;
+        ptx::mbar_arrive_expect_tx(vfull0 + 8 * s, nt * C::kTileBytes);
         for (int t = 0; t < nt; ++t) {
           const int row = (int)((tile_row0 + (int)(list[2 * j + t] & 0xffffu)) * 64);
+          const uint32_t dst = sbase + C::kVOff + s * C::kBufBytes + t * 8192;
+#pragma unroll
           for (int db = 0; db < D / 64; ++db)
-            ptx::tma_load_2d(sbase + C::kVOff + sv * C::kBufBytes + db * C::kDBlockStride + t * 8192, &tmV,
-                             vfull(sv), db * 64, row);
+            ptx::tma_load_2d(dst + db * C::kDBlockStride, &tmV, vfull0 + 8 * s, db * 64, row);
         }
-        last_v[sv] = j;
+        if (s) last_v1 = j; else last_v0 = j;
       }
       // Never leave with copies in flight: wait for the last load issued into each stage.
       int zero = 0;
-      for (int s = 0; s < kNSK; ++s)
-        if (last_k[s] >= 0) ptx::mbar_wait(kfull(s), (last_k[s] / kNSK) & 1, &zero, a.err, kWaitLimit);
-      for (int s = 0; s < kNSV; ++s)
-        if (last_v[s] >= 0) ptx::mbar_wait(vfull(s), (last_v[s] / kNSV) & 1, &zero, a.err, kWaitLimit);
+      if (last_k0 >= 0) ptx::mbar_wait(kfull0, (last_k0 >> 1) & 1, &zero, a.err, kWaitLimit);
+      if (last_k1 >= 0) ptx::mbar_wait(kfull0 + 8, (last_k1 >> 1) & 1, &zero, a.err, kWaitLimit);
+      if (last_v0 >= 0) ptx::mbar_wait(vfull0, (last_v0 >> 1) & 1, &zero, a.err, kWaitLimit);
+      if (last_v1 >= 0) ptx::mbar_wait(vfull0 + 8, (last_v1 >> 1) & 1, &zero, a.err, kWaitLimit);
       ptx::mbar_wait(bar_q, 0, &zero, a.err, kWaitLimit);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && nblk > 0) {
-      constexpr uint32_t kIdQK128 = ptx::idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t kIdQK64 = ptx::idesc_bf16_f32(128, 64, 0, 0);
-      constexpr uint32_t kIdPV = ptx::idesc_bf16_f32(128, D, 0, 1);
-      int pend[2] = {-1, -1};       // block whose P.V is still to be issued, per sub-unit
-      uint32_t pneed[2] = {0u, 0u};
-      int npv[2] = {0, 0};          // P.V products issued, per sub-unit
-      int vref[kNSV] = {0, 0};      // P.V products still to read each V stage
+      MmaCtx m;
+      m.tmem = tmem;
+      m.dQ0 = ptx::smem_desc_sw128(sbase + C::kQOff, 16, 1024);
+      m.dK0 = ptx::smem_desc_sw128(sbase + C::kKOff, 16, 1024);
+      m.dV0 = ptx::smem_desc_sw128(sbase + C::kVOff, C::kDBlockStride, 1024);
+      m.pfull0 = pfull0;
+      m.vfull0 = vfull0;
+      m.vempty0 = vempty0;
+      m.sfull0 = sfull0;
+      m.odone0 = odone0;
+      m.abort = abort;
+      m.err = a.err;
+      SubUnitIssue sA{-1, 0u, 0}, sB{-1, 0u, 0};
+      int vref0 = 0, vref1 = 0;     // P.V products still to read V stage 0 / 1
       bool ok = ptx::mbar_wait(bar_q, 0, abort, a.err, kWaitLimit);
 
-      auto need_of = [&](int j, int u) -> uint32_t {
-        const uint32_t e0 = list[2 * j];
-        const uint32_t e1 = (2 * j + 1 < L) ? list[2 * j + 1] : 0u;
-        const int sh = 16 + 2 * u;
-        return (((e0 >> sh) & 3u) ? 1u : 0u) | (((e1 >> sh) & 3u) ? 2u : 0u);
-      };
-      auto issue_pv = [&](int u) -> bool {
-        const int j = pend[u];
-        const uint32_t n = pneed[u];
-        const int sv = j % kNSV;
-        if (!ptx::mbar_wait(pfull(u), npv[u] & 1, abort, a.err, kWaitLimit)) return false;
-        if (!ptx::mbar_wait(vfull(sv), (j / kNSV) & 1, abort, a.err, kWaitLimit)) return false;
-        ptx::tc_fence_after();
-        const uint32_t p_tmem = tmem + 128 * u;
-        const uint32_t o_tmem = tmem + 256 + 128 * u;
-        const uint32_t vaddr = sbase + C::kVOff + sv * C::kBufBytes + (n == 2u ? 8192u : 0u);
-        const int nk = (n == 3u) ? 8 : 4;
-        for (int kk = 0; kk < nk; ++kk) {
-          const uint64_t bd = ptx::smem_desc_sw128(vaddr + kk * 2048, C::kDBlockStride, 1024);
-          ptx::mma_ts(o_tmem, p_tmem + kk * 8, bd, kIdPV, (npv[u] > 0 || kk > 0) ? 1u : 0u);
-        }
-        ptx::mma_commit(odone(u));
-        ++npv[u];
-        if (--vref[sv] == 0) ptx::mma_commit(vempty(sv));
-        pend[u] = -1;
-        return true;
-      };
-
       for (int j = 0; j < nblk && ok; ++j) {
-        const int sk = j % kNSK;
-        const uint32_t nA = need_of(j, 0), nB = need_of(j, 1);
-        if (!ptx::mbar_wait(kfull(sk), (j / kNSK) & 1, abort, a.err, kWaitLimit)) break;
+        const uint32_t nn = needs[j];
+        const uint32_t nA = nn & 3u, nB = nn >> 2;
+        if (!ptx::mbar_wait(kfull0 + 8 * (j & 1), (j >> 1) & 1, abort, a.err, kWaitLimit)) break;
         ptx::tc_fence_after();
-        vref[j % kNSV] = (nA != 0u) + (nB != 0u);
-        for (int u = 0; u < 2 && ok; ++u) {
-          const uint32_t n = u ? nB : nA;
-          if (n == 0u) continue;
-          if (pend[u] >= 0 && !issue_pv(u)) { ok = false; break; }
-          const uint32_t s_tmem = tmem + 128 * u;
-          const uint32_t qaddr = sbase + C::kQOff + u * C::kBufBytes;
-          const uint32_t kaddr = sbase + C::kKOff + sk * C::kBufBytes + (n == 2u ? 8192u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kDBlockStride + (kk & 3) * 32;
-            const uint64_t ad = ptx::smem_desc_sw128(qaddr + off, 16, 1024);
-            const uint64_t bd = ptx::smem_desc_sw128(kaddr + off, 16, 1024);
-            ptx::mma_ss(s_tmem, ad, bd, n == 3u ? kIdQK128 : kIdQK64, kk > 0 ? 1u : 0u);
-          }
-          ptx::mma_commit(sfull(u));
-          pend[u] = j;
-          pneed[u] = n;
+        if (j & 1) vref1 = (nA != 0u) + (nB != 0u); else vref0 = (nA != 0u) + (nB != 0u);
+        if (nA) {
+          if (sA.pend >= 0 && !issue_pv<C>(sA, 0, m, vref0, vref1)) break;
+          issue_qk<C, D>(sA, 0, j, nA, m);
         }
-        if (!ok) break;
-        ptx::mma_commit(kempty(sk));
+        if (nB) {
+          if (sB.pend >= 0 && !issue_pv<C>(sB, 1, m, vref0, vref1)) break;
+          issue_qk<C, D>(sB, 1, j, nB, m);
+        }
+        ptx::mma_commit(kempty0 + 8 * (j & 1));
         // P.V of a sub-unit that has no work in the next block goes out now, so that every
         // V stage is released within one block of its use.
-        for (int u = 0; u < 2; ++u)
-          if (pend[u] >= 0 && (j + 1 >= nblk || need_of(j + 1, u) == 0u) && !issue_pv(u)) { ok = false; break; }
+        const uint32_t nn1 = (j + 1 < nblk) ? needs[j + 1] : 0u;
+        if (sA.pend >= 0 && (nn1 & 3u) == 0u && !issue_pv<C>(sA, 0, m, vref0, vref1)) break;
+        if (sB.pend >= 0 && (nn1 >> 2) == 0u && !issue_pv<C>(sB, 1, m, vref0, vref1)) break;
       }
       // Never free TMEM under a running MMA: wait until everything issued has completed.
       int zero = 0;
@@ -422,10 +527,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int u = warp >> 2;                 // sub-unit of this warpgroup
     const int row = threadIdx.x & 127;       // TMEM lane
     const int half = row >> 6;
-    const int qt = q[2 * u + half];          // this row's query tile (-1: none)
+    const int qt = u ? (half ? q3 : q2) : (half ? q1 : q0);   // this row's query tile (-1: none)
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t s_tmem = tmem + 128 * u + lane_base;
     const uint32_t o_tmem = tmem + 256 + 128 * u + lane_base;
+    const uint32_t sfull_u = sfull0 + 8 * u, pfull_u = pfull0 + 8 * u, odone_u = odone0 + 8 * u;
     const int cnt = counts[1 + u];
     const uint16_t* my_blk = blk + u * kMaxBlocks;
     const int mshift = 16 + 2 * u + half;
@@ -433,77 +539,64 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = cnt > 0;
     for (int it = 0; it < cnt; ++it) {
-      if (!warp_wait(sfull(u), it & 1, abort, a.err)) { ok = false; break; }
+      if (!warp_wait(sfull_u, it & 1, abort, a.err)) { ok = false; break; }
       ptx::tc_fence_after();
       const uint32_t bj = my_blk[it];
       const int j = bj & 4095;
       const uint32_t n = bj >> 12;
+      const bool two = n == 3u;                    // tile slots 0 and 1 both used
       const uint32_t e0 = list[2 * j];
       const uint32_t e1 = (2 * j + 1 < L) ? list[2 * j + 1] : 0u;
       const uint32_t ea = (n & 1u) ? e0 : e1;      // tile in S columns 0-63
-      const bool two = n == 3u;                    // e1 in columns 64-127
+      const int use_a = tile_use(ea, mshift);
+      const int use_b = two ? tile_use(e1, mshift) : kUseSkip;
+      const uint64_t val_a = use_a == kUsePartial ? entry_valid_mask(ea, g) : ~0ull;
+      const uint64_t val_b = use_b == kUsePartial ? entry_valid_mask(e1, g) : ~0ull;
       // Tile b's scores are read twice (max, then exponentials) instead of being kept
       // live next to tile a's, which keeps the warpgroup within its register budget.
-      float mx;
-      {
+      float mx = -INFINITY;
+      if (use_b != kUseSkip) {
         uint32_t rb[64];
-        if (two) {
-          tmem_ld_x64(s_tmem + 64, rb);
-          ptx::tmem_wait_ld();
-          mask_tile(rb, e1, mshift, g);
-          mx = row_max64(rb, -INFINITY);
-        } else {
-          mx = -INFINITY;
-        }
+        tmem_ld64(s_tmem + 64, rb);
+        ptx::tmem_wait_ld();
+        mx = tile_max(rb, use_b, val_b, mx);
       }
       uint32_t ra[64];
-      tmem_ld_x64(s_tmem, ra);
-      ptx::tmem_wait_ld();
-      mask_tile(ra, ea, mshift, g);
-      mx = row_max64(ra, mx);
+      if (use_a != kUseSkip) {
+        tmem_ld64(s_tmem, ra);
+        ptx::tmem_wait_ld();
+        mx = tile_max(ra, use_a, val_a, mx);
+      }
       // The reference follows the running max exactly, so the row's largest probability
       // is 2^0 = 1, which bf16 holds exactly: rows dominated by one key lose nothing to
       // the bf16 rounding of P. O is rescaled in TMEM whenever the max grows.
       const float m_new = fmaxf(m_run, mx * c);
       const bool grow = m_new > m_run;
-      const float m_ref = m_new;
       const float alpha = grow ? ex2(m_run - m_new) : 1.0f;
-      const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+      const float m_use = (m_new == -INFINITY) ? 0.0f : m_new;
       float sum = 0.f;
-      uint32_t pk[32];
-      exp_pack64(ra, c, m_use, sum, pk);
-      tmem_st_x32(s_tmem, pk);
+      tile_exp(ra, use_a, val_a, c, m_use, sum, s_tmem);
       if (two) {
         uint32_t rb[64];
-        tmem_ld_x64(s_tmem + 64, rb);
-        ptx::tmem_wait_ld();
-        mask_tile(rb, e1, mshift, g);
-        exp_pack64(rb, c, m_use, sum, pk);
-        tmem_st_x32(s_tmem + 32, pk);
+        if (use_b != kUseSkip) {
+          tmem_ld64(s_tmem + 64, rb);
+          ptx::tmem_wait_ld();
+        }
+        tile_exp(rb, use_b, val_b, c, m_use, sum, s_tmem + 32);
       }
       l_run = l_run * alpha + sum;
       if (it > 0) {
         // O must hold exactly the previous blocks before it is rescaled.
-        if (!warp_wait(odone(u), (it - 1) & 1, abort, a.err)) { ok = false; break; }
+        if (!warp_wait(odone_u, (it - 1) & 1, abort, a.err)) { ok = false; break; }
         ptx::tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll 1
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t ov[32];
-            tmem_ld_x32(o_tmem + ch * 32, ov);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
-            tmem_st_x32(o_tmem + ch * 32, ov);
-          }
-        }
+        if (__any_sync(0xffffffffu, grow)) rescale_o<D>(o_tmem, alpha);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(pfull(u));
-      m_run = m_ref;
+      ptx::mbar_arrive(pfull_u);
+      m_run = m_new;
     }
-    if (ok && warp_wait(odone(u), (cnt - 1) & 1, abort, a.err)) {
+    if (ok && warp_wait(odone_u, (cnt - 1) & 1, abort, a.err)) {
       ptx::tc_fence_after();
       const int r = row & 63;
       int n_tok = -1;

@@ -7,7 +7,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/bsa.h"
+#include "bsa.h"
 
 namespace bsa {
 

@@ -31,15 +31,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
       "r"(bytes)
       : "memory");
 }
-// One try_wait; the thread may be suspended in hardware for up to about 20 us while the
-// phase is incomplete, so that waiting warps do not take issue slots from working ones.
+// One try_wait (the hardware may suspend the thread for a short, system-defined time while
+// the phase is incomplete).
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "n"(20000)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
