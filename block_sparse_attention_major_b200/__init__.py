@@ -80,6 +80,9 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.bsa_build_mask.argtypes = [G, P, vp, vp, vp, vp, vp, vp, sz, vp]
         lib.bsa_sparse_attn_fwd.restype = ctypes.c_int
         lib.bsa_sparse_attn_fwd.argtypes = [G, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, sz, vp]
+        lib.bsa_sparse_attn_fwd_fixed_scratch.restype = ctypes.c_int
+        lib.bsa_sparse_attn_fwd_fixed_scratch.argtypes = [G, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp,
+                                                          vp, vp]
         lib.bsa_launch_count.restype = ctypes.c_uint64
         lib.bsa_launch_count.argtypes = []
         if path is None:
@@ -252,6 +255,46 @@ def sparse_attn_fwd(g: Geometry, qt: torch.Tensor, kt: torch.Tensor, vt: torch.T
                                               _ptr(out), _ptr(lse), _ptr(ws),
                                               ctypes.c_size_t(ws.numel()), _stream(stream)),
            "bsa_sparse_attn_fwd")
+    return out, lse
+
+
+def sparse_attn_fwd_fixed_scratch(g: Geometry, qt: torch.Tensor, kt: torch.Tensor, vt: torch.Tensor,
+                                  mask: torch.Tensor, kv_count: torch.Tensor,
+                                  scale: float | None = None, out: torch.Tensor | None = None,
+                                  lse: torch.Tensor | None = None,
+                                  kernel_errors: torch.Tensor | None = None,
+                                  want_lse: bool = True,
+                                  stream=None) -> tuple[torch.Tensor, torch.Tensor | None]:
+    """Block-sparse attention whose scratch is the library's own fixed device array.
+
+    For callers that cannot allocate device memory (a plug-in that receives tensors from a
+    host application which owns all device memory, or a serving loop that forbids
+    allocation after start-up): pass preallocated `out` / `lse` and nothing is allocated
+    here or in the library. Limits and sharing rules are those of
+    bsa_sparse_attn_fwd_fixed_scratch in include/bsa.h: one call at a time per device, and
+    the first call on a device should come before any stream capture.
+    `kernel_errors`, if given, is a 1-element int32 device tensor that receives the call's
+    kernel error word.
+    """
+    for name, t in (("qt", qt), ("kt", kt), ("vt", vt)):
+        _need(t, torch.bfloat16, (g.B, g.H, g.NT, 64, g.d), name)
+    _need(mask, torch.int32, (g.B, g.H, g.NT, g.NW), "mask")
+    _need(kv_count, torch.int32, (g.B, g.H, g.NT), "kv_count")
+    dev = qt.device
+    if out is None:
+        out = torch.empty((g.B, g.N, g.H, g.d), dtype=torch.bfloat16, device=dev)
+    _need(out, torch.bfloat16, (g.B, g.N, g.H, g.d), "out")
+    if want_lse and lse is None:
+        lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _need(lse, torch.float32, (g.B, g.H, g.N), "lse")
+    if kernel_errors is not None:
+        _need(kernel_errors, torch.int32, (1,), "kernel_errors")
+    sc = 1.0 / math.sqrt(g.d) if scale is None else float(scale)
+    _check(load_library().bsa_sparse_attn_fwd_fixed_scratch(
+        ctypes.byref(g.c()), _ptr(qt), _ptr(kt), _ptr(vt), _ptr(mask), _ptr(kv_count),
+        ctypes.c_float(sc), _ptr(out), _ptr(lse), _ptr(kernel_errors), _stream(stream)),
+        "bsa_sparse_attn_fwd_fixed_scratch")
     return out, lse
 
 

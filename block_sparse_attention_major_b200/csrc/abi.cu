@@ -147,6 +147,27 @@ int bsa_sparse_attn_fwd(const bsa_geom* g, const void* qt, const void* kt, const
                                       static_cast<uint8_t*>(ws), static_cast<cudaStream_t>(stream)));
 }
 
+int bsa_sparse_attn_fwd_fixed_scratch(const bsa_geom* g, const void* qt, const void* kt, const void* vt,
+                                      const uint32_t* mask, const int32_t* kv_count, float softmax_scale,
+                                      void* out, float* lse, uint32_t* kernel_errors, void* stream) {
+  if (!valid_geom(g)) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(qt) || !aligned16(kt) || !aligned16(vt) || !aligned16(mask) || !aligned16(kv_count) ||
+      !aligned16(out))
+    return BSA_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return BSA_ERR_INVALID_ARG;
+  if (kernel_errors && (reinterpret_cast<uintptr_t>(kernel_errors) & 3u) != 0) return BSA_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.0f) || isinf(softmax_scale)) return BSA_ERR_INVALID_ARG;
+  const Geom G = make_geom(*g);
+  if (fixed_scratch_need(G) > fixed_scratch_capacity()) return BSA_ERR_WORKSPACE;
+  const int dev = device_ok();
+  if (dev != BSA_OK) return dev;
+  return status_of(launch_sparse_attn_fixed_scratch(G, static_cast<const __nv_bfloat16*>(qt),
+                                                    static_cast<const __nv_bfloat16*>(kt),
+                                                    static_cast<const __nv_bfloat16*>(vt), mask, kv_count,
+                                                    softmax_scale, static_cast<__nv_bfloat16*>(out), lse,
+                                                    kernel_errors, static_cast<cudaStream_t>(stream)));
+}
+
 uint64_t bsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"

@@ -793,3 +793,100 @@ cudaError_t launch_sparse_attn(const Geom& g, const __nv_bfloat16* qt, const __n
 }
 
 }  // namespace bsa
+
+// ---------------------------------------------------------------------------------------
+// Fixed-scratch variant of the attention call.
+//
+// Some callers cannot allocate device memory at all: a plug-in loaded into a host
+// application whose device memory belongs to the host's own allocator (the plug-in gets
+// tensors, never an allocator), or a serving loop that forbids cudaMalloc after start-up
+// because it can block and synchronise the whole device. For them the attention call's
+// scratch (work-list header, per-(b, h) counts, work units) lives in the library's own
+// file-scope device array below, fixed in size and held by every GPU that loads the
+// library until the process exits. The caller passes only inputs and outputs.
+// ---------------------------------------------------------------------------------------
+#include <mutex>
+
+namespace bsa {
+namespace {
+
+constexpr size_t kFixedScratchBytes = size_t(1) << 20;   // 1 MiB
+static __device__ __align__(256) uint8_t g_fixed_scratch[kFixedScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_fixed_mu;
+uint8_t* g_fixed_addr[kMaxDevices] = {};   // device address of g_fixed_scratch, per device
+
+// The array's device address on the current device. In host code the array's name is a
+// host-side stand-in, not a device address, so the first call on each device looks the
+// address up (with that device current) and keeps it.
+cudaError_t fixed_scratch_addr(uint8_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_fixed_mu);
+  if (!g_fixed_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_fixed_scratch);
+    if (e != cudaSuccess) return e;
+    g_fixed_addr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = g_fixed_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+size_t fixed_scratch_capacity() { return kFixedScratchBytes; }
+
+// Scratch of one call: 256-byte header (error word, unit count), per-(b, h) counts, units.
+size_t fixed_scratch_need(const Geom& g) {
+  const size_t bh = (size_t)g.B * g.H;
+  return 256 + align256(bh * sizeof(int4)) + bh * units_per_bh(g.NT) * kUnitInts * sizeof(int);
+}
+
+cudaError_t launch_sparse_attn_fixed_scratch(const Geom& g, const __nv_bfloat16* qt, const __nv_bfloat16* kt,
+                                             const __nv_bfloat16* vt, const uint32_t* mask,
+                                             const int32_t* kv_count, float scale, __nv_bfloat16* out,
+                                             float* lse, uint32_t* errors, cudaStream_t s) {
+  if (fixed_scratch_need(g) > kFixedScratchBytes) return cudaErrorInvalidValue;
+  uint8_t* base = nullptr;
+  cudaError_t e = fixed_scratch_addr(&base);
+  if (e != cudaSuccess) return e;
+  const int BH = g.B * g.H;
+  int* header = reinterpret_cast<int*>(base);
+  int4* bhcnt = reinterpret_cast<int4*>(base + 256);
+  int* units = reinterpret_cast<int*>(base + 256 + align256((size_t)BH * sizeof(int4)));
+
+  // The array keeps the previous call's contents: the error word and the unit count must
+  // start at zero; counts and units are fully rewritten by the scheduler before use.
+  e = cudaMemsetAsync(base, 0, 256, s);
+  if (e != cudaSuccess) return e;
+  sched_count_kernel<<<BH, 256, 0, s>>>(g, kv_count, bhcnt);
+  sched_scan_kernel<<<1, 32, 0, s>>>(BH, bhcnt, header);
+  sched_write_kernel<<<BH, 32, 0, s>>>(g, kv_count, bhcnt, units);
+  count_launches(3);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  const long long rows = (long long)g.B * g.H * g.NT * 64;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, qt, rows, g.d) || !make_map(&mk, kt, rows, g.d) || !make_map(&mv, vt, rows, g.d))
+    return cudaErrorInvalidValue;
+  AttnArgs a;
+  a.g = g;
+  a.mask = mask;
+  a.units = units;
+  a.header = header;
+  a.out = out;
+  a.lse = lse;
+  a.err = reinterpret_cast<uint32_t*>(base);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  e = (g.d == 128) ? run_attn<128>(g, mq, mk, mv, a, s) : run_attn<64>(g, mq, mk, mv, a, s);
+  if (e != cudaSuccess) return e;
+  if (errors) e = cudaMemcpyAsync(errors, base, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s);
+  return e;
+}
+
+}  // namespace bsa

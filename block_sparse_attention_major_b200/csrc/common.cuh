@@ -129,5 +129,12 @@ cudaError_t launch_build_mask(const Geom& g, const bsa_mask_params& p, const __n
 cudaError_t launch_sparse_attn(const Geom& g, const __nv_bfloat16* qt, const __nv_bfloat16* kt,
                                const __nv_bfloat16* vt, const uint32_t* mask, const int32_t* kv_count,
                                float scale, __nv_bfloat16* out, float* lse, uint8_t* ws, cudaStream_t s);
+// Attention with its scratch in the library's fixed device array (no workspace argument).
+size_t fixed_scratch_capacity();
+size_t fixed_scratch_need(const Geom& g);
+cudaError_t launch_sparse_attn_fixed_scratch(const Geom& g, const __nv_bfloat16* qt, const __nv_bfloat16* kt,
+                                             const __nv_bfloat16* vt, const uint32_t* mask,
+                                             const int32_t* kv_count, float scale, __nv_bfloat16* out,
+                                             float* lse, uint32_t* errors, cudaStream_t s);
 void count_launches(int n);
 }  // namespace bsa

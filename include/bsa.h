@@ -154,6 +154,28 @@ int bsa_sparse_attn_fwd(const bsa_geom* g, const void* qt, const void* kt, const
                         const uint32_t* mask, const int32_t* kv_count, float softmax_scale,
                         void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
 
+/* Block-sparse attention forward without a workspace argument. The papers have no
+ * counterpart: this entry point exists for callers that cannot allocate device memory,
+ * such as a plug-in inside a host application that owns all device memory through its own
+ * allocator and hands the plug-in tensors but no allocator, or a serving loop that bans
+ * cudaMalloc after start-up because it can block and synchronise the device.
+ *   Arguments as bsa_sparse_attn_fwd, minus ws / ws_bytes, plus
+ *   kernel_errors : optional device pointer to one uint32; if not NULL it receives the
+ *                   call's kernel error word (BSA_KERR_* bits) at the end of the call
+ * Scratch: a fixed 1 MiB array inside the library (a file-scope device array that every
+ * GPU which loads the library holds until the process exits). A call needs
+ * 256 + align256(16*B*H) + 32*B*H*(floor(NT/4) + 2) bytes of it (about 61 KB for 12 heads
+ * of 624 tiles, 464 KB for 40 heads of 1440 tiles); a larger call is rejected with
+ * BSA_ERR_WORKSPACE before anything is launched. The call allocates and frees nothing.
+ * Every call uses the same array and leaves its contents there: each call zeroes the
+ * array's header on its stream before use, and calls that overlap on the GPU (other
+ * streams, other host threads, same device) race on the array and must not be issued.
+ * The first call on each device looks up the array's device address (with that device
+ * current); make that first call before any stream capture. */
+int bsa_sparse_attn_fwd_fixed_scratch(const bsa_geom* g, const void* qt, const void* kt, const void* vt,
+                                      const uint32_t* mask, const int32_t* kv_count, float softmax_scale,
+                                      void* out, float* lse, uint32_t* kernel_errors, void* stream);
+
 /* Number of kernels the library launched since it was loaded (all entry points, all
  * threads). Host-side counter, for accounting only. */
 uint64_t bsa_launch_count(void);
