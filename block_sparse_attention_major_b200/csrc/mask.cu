@@ -13,10 +13,11 @@
 //
 // The pooled-score contraction is an fp32 SIMT GEMM of [ROWS x d] query means against
 // 64-key chunks staged in shared memory (float4 operands, padded rows, no bank
-// conflicts). Selection is a per-row, per-warp radix select on order-preserving integer
-// keys of the fp32 scores (4 passes of 8 bits) followed by an index-ordered pass that
-// takes tied threshold keys from the lowest tile index up, which reproduces the
-// "highest score, ties to the lower index" rule exactly.
+// conflicts). Selection works per row and per warp on order-preserving integer keys of
+// the fp32 scores: a few extra tiles by repeated warp argmax (largest key, then lowest
+// tile index), many by a bitwise binary search for the threshold key followed by an
+// index-ordered pass over tied keys. Both reproduce "highest score, ties to the lower
+// index" exactly and use no atomics.
 #include "common.cuh"
 
 #include <math.h>
@@ -162,8 +163,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
   float* ks = qs + ROWS * DP;                                     // kKeyChunk * DP
   float* sc = ks + kKeyChunk * DP;                                // ROWS * NKTP
   uint32_t* coord = reinterpret_cast<uint32_t*>(sc + ROWS * NKTP); // NKTP
-  uint32_t* hist = coord + NKTP;                                  // kSelWarps * 256
-  double* dsum = reinterpret_cast<double*>(hist + kSelWarps * 256);
+  double* dsum = reinterpret_cast<double*>(coord + NKTP);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -289,101 +289,90 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
       extra = budget - wsize;
     }
 
-    // threshold key: the extra-th largest key among candidates (tiles outside the window)
-    uint32_t thr;
-    int need_eq;
-    if (extra <= 0) {
-      thr = 0xffffffffu;
-      need_eq = 0;
-    } else {
-      uint32_t* hw = hist + warp * 256;
-      uint32_t prefix = 0, pmask = 0;
-      int rem = extra;
-      int total_cand = 0;
-      for (int w = 0; w < g.NW; ++w) {
-        const int j = 32 * w + lane;
-        total_cand += __popc(__ballot_sync(0xffffffffu, j < NKT && !in_window(ci, coord[j], kind, rad)));
-      }
-      if (rem >= total_cand) {
-        thr = 0u;
-        need_eq = 0x7fffffff;
-      } else {
-        for (int pass = 0; pass < 4; ++pass) {
-          const int shift = 24 - 8 * pass;
-          for (int k = lane; k < 256; k += 32) hw[k] = 0u;
-          __syncwarp();
-          for (int w = 0; w < g.NW; ++w) {
-            const int j = 32 * w + lane;
-            if (j < NKT && !in_window(ci, coord[j], kind, rad)) {
-              const uint32_t u = order_key(srow[j]);
-              if ((u & pmask) == prefix) atomicAdd(&hw[(u >> shift) & 255u], 1u);
-            }
-          }
-          __syncwarp();
-          // lane L owns bins 255-8L .. 248-8L (descending key order)
-          uint32_t c[8];
-          uint32_t lsum = 0;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            c[k] = hw[255 - 8 * lane - k];
-            lsum += c[k];
-          }
-          uint32_t incl = lsum;
-#pragma unroll
-          for (int off = 1; off < 32; off <<= 1) {
-            const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += v;
-          }
-          const uint32_t excl = incl - lsum;
-          const bool found = excl < (uint32_t)rem && (uint32_t)rem <= incl;
-          const uint32_t bal = __ballot_sync(0xffffffffu, found);
-          const int src = __ffs(bal) - 1;
-          uint32_t bin = 0, above = 0;
-          if (found) {
-            uint32_t acc = excl;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              if (acc + c[k] >= (uint32_t)rem) {
-                bin = 255 - 8 * lane - k;
-                above = acc;
-                break;
-              }
-              acc += c[k];
-            }
-          }
-          bin = __shfl_sync(0xffffffffu, bin, src);
-          above = __shfl_sync(0xffffffffu, above, src);
-          rem -= (int)above;
-          prefix |= bin << shift;
-          pmask |= 0xffu << shift;
-          __syncwarp();
-        }
-        thr = prefix;
-        need_eq = rem;
-      }
-    }
-
-    // write the row: window | key > thr | (key == thr and among the first need_eq ties)
-    int count = 0, eq_before = 0;
+    // Order-preserving integer keys of the candidates (tiles outside the window), written
+    // over the row's scores; 0 marks a window tile or a slot beyond NKT (no real score maps
+    // to 0 or 1).
+    uint32_t* krow = reinterpret_cast<uint32_t*>(sc + rr * NKTP);
+    int ncand = 0;
     for (int w = 0; w < g.NW; ++w) {
       const int j = 32 * w + lane;
-      bool sel = false, eq = false;
-      if (j < NKT) {
-        if (in_window(ci, coord[j], kind, rad)) {
-          sel = true;
-        } else if (extra > 0) {
-          const uint32_t u = order_key(srow[j]);
-          sel = u > thr;
-          eq = u == thr;
+      const bool cand = j < NKT && !in_window(ci, coord[j], kind, rad);
+      if (j < NKTP) krow[j] = cand ? order_key(srow[j]) : 0u;
+      ncand += __popc(__ballot_sync(0xffffffffu, cand));
+    }
+    __syncwarp();
+    extra = max(0, min(extra, ncand));
+
+    int count = 0;
+    if (extra == ncand || extra <= 32) {
+      // Few extra tiles (or all of them): repeated warp argmax, the largest key first and
+      // the lowest tile index among equal keys; a chosen tile's key becomes 1.
+      for (int round = 0; round < extra && extra < ncand; ++round) {
+        uint64_t best = 0;
+        for (int w = 0; w < g.NW; ++w) {
+          const int j = 32 * w + lane;
+          const uint32_t k = j < NKTP ? krow[j] : 0u;
+          const uint64_t v = ((uint64_t)k << 32) | (uint32_t)(0xffffffffu - (uint32_t)j);
+          best = (k > 1u && v > best) ? v : best;
         }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
+          best = o > best ? o : best;
+        }
+        const int jbest = (int)(0xffffffffu - (uint32_t)best);
+        if (lane == 0) krow[jbest] = 1u;
+        __syncwarp();
       }
-      const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
-      const int rank = eq_before + __popc(eqb & ((1u << lane) - 1u));
-      sel = sel || (eq && rank < need_eq);
-      eq_before += __popc(eqb);
-      const uint32_t bits = __ballot_sync(0xffffffffu, sel);
-      if (lane == 0) mrow[w] = bits;
-      count += __popc(bits);
+      for (int w = 0; w < g.NW; ++w) {
+        const int j = 32 * w + lane;
+        bool sel = false;
+        if (j < NKT) {
+          const uint32_t k = krow[j];
+          sel = k <= 1u || extra == ncand;        // window (0), chosen (1), or every candidate
+        }
+        const uint32_t bits = __ballot_sync(0xffffffffu, sel);
+        if (lane == 0) mrow[w] = bits;
+        count += __popc(bits);
+      }
+    } else {
+      // Many extra tiles: bitwise binary search for the extra-th largest key T, counting
+      // with warp reductions (no atomics); then every key above T and, among keys equal to
+      // T, the lowest tile indices.
+      uint32_t thr = 0u;
+      for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand_t = thr | (1u << bit);
+        int c = 0;
+        for (int w = 0; w < g.NW; ++w) {
+          const int j = 32 * w + lane;
+          c += (j < NKTP && krow[j] >= cand_t) ? 1 : 0;
+        }
+        c = __reduce_add_sync(0xffffffffu, c);
+        if (c >= extra) thr = cand_t;
+      }
+      int gt = 0;
+      for (int w = 0; w < g.NW; ++w) {
+        const int j = 32 * w + lane;
+        gt += (j < NKTP && krow[j] > thr) ? 1 : 0;
+      }
+      const int need_eq = extra - __reduce_add_sync(0xffffffffu, gt);
+      int eq_before = 0;
+      for (int w = 0; w < g.NW; ++w) {
+        const int j = 32 * w + lane;
+        bool sel = false, eq = false;
+        if (j < NKT) {
+          const uint32_t k = krow[j];
+          sel = k == 0u || k > thr;
+          eq = k == thr;
+        }
+        const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+        const int rank = eq_before + __popc(eqb & ((1u << lane) - 1u));
+        sel = sel || (eq && rank < need_eq);
+        eq_before += __popc(eqb);
+        const uint32_t bits = __ballot_sync(0xffffffffu, sel);
+        if (lane == 0) mrow[w] = bits;
+        count += __popc(bits);
+      }
     }
     if (lane == 0) a.kv_count[rowid] = count;
   }
@@ -394,7 +383,7 @@ cudaError_t run_select(const SelArgs& a, cudaStream_t s) {
   const Geom& g = a.g;
   const int NKTP = (g.NT + 3) & ~3;
   const size_t smem = sizeof(float) * ((size_t)(ROWS + kKeyChunk) * (D + 4) + (size_t)ROWS * NKTP) +
-                      sizeof(uint32_t) * ((size_t)NKTP + kSelWarps * 256) + sizeof(double);
+                      sizeof(uint32_t) * (size_t)NKTP + sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(select_kernel<D, ROWS, MODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -408,7 +397,7 @@ template <int D, int MODE>
 cudaError_t run_select_rows(const SelArgs& a, cudaStream_t s) {
   // 16 query rows per block while the score rows fit in shared memory, else 8.
   const size_t rows16 = sizeof(float) * ((size_t)(16 + kKeyChunk) * (D + 4) + 16ull * ((a.g.NT + 3) & ~3)) +
-                        sizeof(uint32_t) * ((size_t)((a.g.NT + 3) & ~3) + kSelWarps * 256) + 8;
+                        sizeof(uint32_t) * (size_t)((a.g.NT + 3) & ~3) + 8;
   if (rows16 <= 200 * 1024) return run_select<D, 16, MODE>(a, s);
   return run_select<D, 8, MODE>(a, s);
 }
