@@ -45,6 +45,9 @@ def _args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--report", action="store_true",
+                    help="per-stage timings of every benchmark workload (one JSON line each); "
+                         "not the headline measurement")
     return ap.parse_args()
 
 
@@ -448,10 +451,95 @@ def run_ours(args):
     return 0
 
 
+def _report_workloads():
+    from bsa_synth import HUNYUAN_TAU_SWEEP, WAN5B_RHO_SWEEP, WORKLOADS
+    out = [("tiny", WORKLOADS["tiny"]), ("wan13b", WORKLOADS["wan13b"])]
+    out += [(f"wan5b_rho{r}", WORKLOADS["wan5b"].with_(dense_fraction=r)) for r in WAN5B_RHO_SWEEP]
+    out.append(("wan14b", WORKLOADS["wan14b"]))
+    out += [(f"hunyuan_tau{t}", WORKLOADS["hunyuan"].with_(budget_target=t)) for t in HUNYUAN_TAU_SWEEP]
+    return out
+
+
+def run_report(args):
+    """Per-stage device times of every benchmark workload on one GPU."""
+    import torch
+
+    import block_sparse_attention_major_b200 as bsa
+    from bsa_synth import generate_difficulty, generate_qkv
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cache = {}
+    for name, w in _report_workloads():
+        key = (w.H, w.d, w.T, w.Hs, w.Ws, w.seed, w.sink_frac)
+        if key not in cache:
+            cache.clear()
+            cache[key] = tuple(x.to(dev) for x in (*generate_qkv(w), generate_difficulty(w)))
+        q, k, v, diff = cache[key]
+        g = bsa.Geometry(w.B, w.H, w.d, w.T, w.Hs, w.Ws)
+        p = bsa.MaskParams(w.window_kind, w.radius, w.topk, w.dense_fraction, w.budget_mode,
+                           w.budget_target)
+        b = bsa.Buffers(g, dev)
+        bsa.forward(g, p, q, k, v, diff, b)
+        torch.cuda.synchronize()
+        retained = int(b.kv_count.sum().item())
+        stages = {"reorder_qkv": lambda: [bsa.reorder(g, x, y) for x, y in ((q, b.qt), (k, b.kt), (v, b.vt))],
+                  "build_mask": lambda: bsa.build_mask(g, p, b.qt, b.kt, diff, b.mask, b.kv_count, b.ws),
+                  "sparse_attn": lambda: bsa.sparse_attn_fwd(g, b.qt, b.kt, b.vt, b.mask, b.kv_count, None,
+                                                             b.out, b.lse, b.ws)}
+        res = {}
+        for st, fn in stages.items():
+            for _ in range(max(3, args.warmup)):
+                fn()
+            n = max(5, min(args.steps, 30))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(n):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            res[st] = e0.elapsed_time(e1) / n
+        err = bsa.read_error(b.ws)
+        flops = 4.0 * 64 * 64 * g.d * retained
+        dense_pairs = g.B * g.H * g.NT * g.NT
+        # own dense path: the same attention kernel with every tile retained
+        pd = bsa.MaskParams(w.window_kind, max(w.radius, 0), w.topk, 1.0, 0, 0.0)
+        bsa.build_mask(g, pd, b.qt, b.kt, diff, b.mask, b.kv_count, b.ws)
+        for _ in range(2):
+            bsa.sparse_attn_fwd(g, b.qt, b.kt, b.vt, b.mask, b.kv_count, None, b.out, b.lse, b.ws)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nd = 3
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(nd):
+            bsa.sparse_attn_fwd(g, b.qt, b.kt, b.vt, b.mask, b.kv_count, None, b.out, b.lse, b.ws)
+        e1.record()
+        torch.cuda.synchronize()
+        dense_ms = e0.elapsed_time(e1) / nd
+        qkv_bytes = 3 * (g.B * g.N * g.H * g.d * 2 + g.B * g.H * g.NT * 64 * g.d * 2)
+        print(json.dumps({
+            "workload": name, "B": g.B, "H": g.H, "d": g.d, "grid": [g.T, g.Hs, g.Ws], "tiles": g.NT,
+            "retained_tile_fraction": retained / dense_pairs, "ms": res,
+            "ms_step": sum(res.values()),
+            "attn_effective_tflops": flops / (res["sparse_attn"] * 1e-3) / 1e12,
+            "step_effective_tflops": flops / (sum(res.values()) * 1e-3) / 1e12,
+            "reorder_gbs": qkv_bytes / (res["reorder_qkv"] * 1e-3) / 1e9,
+            "dense_ms": dense_ms,
+            "dense_effective_tflops": 4.0 * 64 * 64 * g.d * dense_pairs / (dense_ms * 1e-3) / 1e12,
+            "sparse_speedup_vs_own_dense": dense_ms / res["sparse_attn"],
+            "kernel_error_word": err}), flush=True)
+        del b
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     args = _args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.report:
+        return run_report(args)
     return run_ours(args)
 
 

@@ -281,3 +281,30 @@ def test_forward_path(name):
     st = C.compare_attention(w, b.out, b.lse, ref, skip_rows=cmp["diff_rows"])
     print(name, st, cmp["n_diff"])
     C.assert_attention_close(st)
+
+
+@pytest.mark.parametrize("name,overrides", [("wan14b", ()), ("hunyuan", (("budget_target", 0.14),))])
+def test_forward_path_full_size(name, overrides):
+    """Whole path on the 14B- and Hunyuan-shaped calls; the oracle checks two heads."""
+    bsa = _bsa()
+    w, q, k, v, diff = C.inputs(name, overrides)
+    g = C.geometry(w)
+    b = bsa.forward(g, C.params(w), q.cuda(), k.cuda(), v.cuda(), diff.cuda())
+    torch.cuda.synchronize()
+    assert bsa.read_error(b.ws) == 0
+    heads = [0, w.H - 1]
+    qt64, kt64, vt64 = (O.reorder(O.to_f64(x[:, :, heads]), w.T, w.Hs, w.Ws) for x in (q, k, v))
+    mref = C.oracle_mask(w, qt64, kt64, diff.numpy())
+    gm = C.gpu_mask_bool(b.mask, g.NT)[:, heads]
+    cmp = C.compare_masks(gm, mref)
+    assert cmp["n_unflagged"] == 0, cmp
+    rng = np.random.default_rng(23)
+    rows = [(0, int(rng.integers(2)), int(rng.integers(g.NT))) for _ in range(10)]
+    ref = O.attention_tiles(qt64, kt64, vt64, mref["mask"], rows, T=w.T, Hs=w.Hs, Ws=w.Ws)
+    # map the oracle's head slots back to the call's heads
+    ref = {(bb, heads[h], i): e for (bb, h, i), e in ref.items()}
+    skip = np.zeros((w.B, w.H, g.NT), dtype=bool)
+    skip[:, heads] = cmp["diff_rows"]
+    st = C.compare_attention(w, b.out, b.lse, ref, skip_rows=skip)
+    print(name, st, cmp["n_diff"], "retained", float(gm.mean()))
+    C.assert_attention_close(st)
