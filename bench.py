@@ -48,6 +48,7 @@ def _args():
     ap.add_argument("--report", action="store_true",
                     help="per-stage timings of every benchmark workload (one JSON line each); "
                          "not the headline measurement")
+    ap.add_argument("--only", default=None, help="with --report: workloads whose name starts with this")
     return ap.parse_args()
 
 
@@ -471,6 +472,8 @@ def run_report(args):
     torch.cuda.set_device(dev)
     cache = {}
     for name, w in _report_workloads():
+        if args.only and not name.startswith(args.only):
+            continue
         key = (w.H, w.d, w.T, w.Hs, w.Ws, w.seed, w.sink_frac)
         if key not in cache:
             cache.clear()

@@ -331,7 +331,7 @@ def forward(g: Geometry, p: MaskParams, q: torch.Tensor, k: torch.Tensor, v: tor
     return b
 
 
-# kernels launched by forward(): 3 reorders, pool + route + 1 select (2 in budget mode),
-# 3 scheduler kernels + the attention kernel
+# kernels launched by forward(): 3 reorders; pool, route, score and select (plus entropy
+# and budget in budget mode); 3 scheduler kernels and the attention kernel
 def launches_per_forward(p: MaskParams) -> int:
-    return 3 + 2 + (2 if p.budget_mode == 1 else 1) + 4
+    return 3 + 4 + (2 if p.budget_mode == 1 else 0) + 4

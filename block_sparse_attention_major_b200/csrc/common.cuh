@@ -58,13 +58,14 @@ struct FastDiv {
 // [0, 256)        header: error word (u32 @0), attention unit count (i32 @4)
 // then 256-aligned regions: qbar, kbar (fp32 [B,H,NT,d]), dense flags (u8 [B,NT]),
 // row entropy (fp32 [B,H,NT]), per-(b,h) unit counts/offsets (int4 [B*H]),
-// attention units (8 ints each, [B*H*(NT/4+2)]).
+// attention units (8 ints each, [B*H*(NT/4+2)]), pooled scores (fp32 [B,H,NT,NTP],
+// NTP = NT rounded up to a multiple of 4).
 // Upper bound on attention work units (four query tiles each): per (b, h),
 // ceil(nd/4) + ceil(nl/4) <= NT/4 + 2.
 inline __host__ __device__ int units_per_bh(int NT) { return NT / 4 + 2; }
 
 struct WsLayout {
-  size_t qbar, kbar, dense, entropy, bhcnt, units, total;
+  size_t qbar, kbar, dense, entropy, plan, bhcnt, units, scores, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -77,8 +78,10 @@ inline WsLayout ws_layout(const Geom& g) {
   L.kbar = off; off = align256(off + pooled);
   L.dense = off; off = align256(off + (size_t)g.B * g.NT);
   L.entropy = off; off = align256(off + (size_t)g.B * g.H * g.NT * sizeof(float));
+  L.plan = off; off = align256(off + (size_t)g.B * g.H * g.NT * 2 * sizeof(int));
   L.bhcnt = off; off = align256(off + (size_t)g.B * g.H * 4 * sizeof(int));
   L.units = off; off = align256(off + (size_t)g.B * g.H * units_per_bh(g.NT) * 8 * sizeof(int));
+  L.scores = off; off = align256(off + (size_t)g.B * g.H * g.NT * (size_t)((g.NT + 3) & ~3) * sizeof(float));
   L.total = off;
   return L;
 }

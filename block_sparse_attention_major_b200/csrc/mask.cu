@@ -4,16 +4,18 @@
 //            pooling" of tiles) -> qbar, kbar fp32 [B, H, NT, d]
 //  route     HetA-DiT routing (Abstract): the floor(rho*NQT + 1/2) query tiles of highest
 //            difficulty of each batch item take dense attention, ties to the lower index
-//  select    per (b, h, query tile): pooled scores against every key tile, then the local
-//            support - a cube window or a window whose spatial radius decays with the
-//            frame-tile distance (Token Radius Attention summary, "Radius construction") -
-//            plus the best tiles outside it by pooled score: a fixed top-k, or the
-//            remainder of a budget derived from the entropy of the pooled-score softmax
+//  score     pooled scores qbar_i . kbar_j of every (b, h, query tile, key tile), fp32,
+//            into the workspace (a register-blocked SIMT SGEMM per head)
+//  entropy   (budget mode) entropy of each row's softmax of the scaled scores
+//  budget    (budget mode) per row: the tile budget, the window radius it affords and the
+//            number of extra tiles
+//  select    per (b, h, query tile): the local support - a cube window or a window whose
+//            spatial radius decays with the frame-tile distance (Token Radius Attention
+//            summary, "Radius construction") - plus the best tiles outside it by pooled
+//            score: a fixed top-k, or the remainder of a budget derived from the entropy
 //            (Token Radius Attention summary, "Entropy-guided budgeting").
 //
-// The pooled-score contraction is an fp32 SIMT GEMM of [ROWS x d] query means against
-// 64-key chunks staged in shared memory (float4 operands, padded rows, no bank
-// conflicts). Selection works per row and per warp on order-preserving integer keys of
+// Selection works per row and per warp on order-preserving integer keys of
 // the fp32 scores: a few extra tiles by repeated warp argmax (largest key, then lowest
 // tile index), many by a bitwise binary search for the threshold key followed by an
 // index-ordered pass over tied keys. Both reproduce "highest score, ties to the lower
@@ -27,7 +29,6 @@ namespace {
 
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kKeyChunk = 64;
 
 // ------------------------------------------------------------------------ pooling
 template <int D>
@@ -99,17 +100,17 @@ __global__ void __launch_bounds__(256) route_kernel(Geom g, const float* __restr
 }
 
 // ------------------------------------------------------------------------ selection
-enum SelMode { kSelectFixed = 0, kEntropy = 1, kSelectBudget = 2 };
+enum SelMode { kSelectFixed = 0, kSelectBudget = 2 };
 
 struct SelArgs {
   Geom g;
   int window_kind, radius, topk;
   float scale;                 // 1/sqrt(d), used by the entropy only
-  double tau;
   const float* qbar;
   const float* kbar;
   const uint8_t* dense;
   float* entropy;              // [B, H, NQT]
+  const int2* plan;            // budget mode: [B, H, NQT] (window radius, extra tiles)
   uint32_t* mask;              // [B, H, NQT, NW]
   int32_t* kv_count;           // [B, H, NQT]
 };
@@ -147,259 +148,301 @@ __device__ int decayed_window_size(const Geom& g, int tt, int ty, int tx, int r)
   return s;
 }
 
-template <int D, int ROWS, int MODE>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
+// ---- pooled scores: one 64 x 64 tile of S = qbar kbar^T (unscaled) per block, for one
+// (b, h). Register-blocked SIMT SGEMM: each thread owns a 4 x 4 sub-tile and reads one
+// float4 of each transposed operand per step of the d-loop (2 shared loads per 16 FMAs).
+// Each output is summed over d in increasing order, so the scores are deterministic.
+constexpr int kScoreTile = 64;
+constexpr int kScorePad = kScoreTile + 4;
+
+template <int D>
+__global__ void __launch_bounds__(256) score_kernel(Geom g, const float* __restrict__ qbar,
+                                                    const float* __restrict__ kbar, float* __restrict__ S,
+                                                    int NKTP) {
   extern __shared__ __align__(16) float smem[];
-  constexpr int DP = D + 4;                         // padded row stride (floats)
-  constexpr int TPR = kSelThreads / ROWS;           // threads per query row in the GEMM
-  constexpr int KPT = kKeyChunk / TPR;              // keys per thread per chunk
+  float* sA = smem;                          // [D][kScorePad]: sA[c][r] = qbar[i0 + r][c]
+  float* sB = smem + D * kScorePad;          // [D][kScorePad]: sB[c][r] = kbar[j0 + r][c]
+  const int i0 = blockIdx.x * kScoreTile, j0 = blockIdx.y * kScoreTile;
+  const long long bh = blockIdx.z;
+  const int tid = threadIdx.x;
+  const float4* q4 = reinterpret_cast<const float4*>(qbar + (bh * g.NT) * D);
+  const float4* k4 = reinterpret_cast<const float4*>(kbar + (bh * g.NT) * D);
+  for (int e = tid; e < kScoreTile * (D / 4); e += 256) {
+    const int r = e / (D / 4), c4 = e % (D / 4);
+    float4 va = make_float4(0.f, 0.f, 0.f, 0.f), vb = va;
+    if (i0 + r < g.NT) va = q4[(long long)(i0 + r) * (D / 4) + c4];
+    if (j0 + r < g.NT) vb = k4[(long long)(j0 + r) * (D / 4) + c4];
+    sA[(4 * c4 + 0) * kScorePad + r] = va.x;
+    sA[(4 * c4 + 1) * kScorePad + r] = va.y;
+    sA[(4 * c4 + 2) * kScorePad + r] = va.z;
+    sA[(4 * c4 + 3) * kScorePad + r] = va.w;
+    sB[(4 * c4 + 0) * kScorePad + r] = vb.x;
+    sB[(4 * c4 + 1) * kScorePad + r] = vb.y;
+    sB[(4 * c4 + 2) * kScorePad + r] = vb.z;
+    sB[(4 * c4 + 3) * kScorePad + r] = vb.w;
+  }
+  __syncthreads();
+  const int tx = tid & 15, ty = tid >> 4;
+  float acc[4][4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+#pragma unroll 8
+  for (int c = 0; c < D; ++c) {
+    const float4 qa = *reinterpret_cast<const float4*>(sA + c * kScorePad + 4 * ty);
+    const float4 kb = *reinterpret_cast<const float4*>(sB + c * kScorePad + 4 * tx);
+    const float qv[4] = {qa.x, qa.y, qa.z, qa.w};
+    const float kv[4] = {kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) acc[r][cc] = fmaf(qv[r], kv[cc], acc[r][cc]);
+  }
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int i = i0 + 4 * ty + r;
+    const int j = j0 + 4 * tx;
+    if (i < g.NT && j < NKTP)
+      *reinterpret_cast<float4*>(S + (bh * g.NT + i) * (long long)NKTP + j) =
+          make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+  }
+}
+
+// ---- row entropy (budget mode): H = log Z - sum(e (s - m)) / Z with s = scale * score,
+// e = exp(s - m); one warp per row.
+__global__ void __launch_bounds__(256) entropy_kernel(Geom g, const float* __restrict__ S, int NKTP,
+                                                      float scale, float* __restrict__ entropy) {
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);   // (b*H + h)*NT + i
+  const int lane = threadIdx.x & 31;
+  if (row >= (long long)g.B * g.H * g.NT) return;
+  const float* srow = S + row * NKTP;
+  float m = -INFINITY;
+  for (int j = lane; j < g.NT; j += 32) m = fmaxf(m, srow[j] * scale);
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  float z = 0.f, t = 0.f;
+  for (int j = lane; j < g.NT; j += 32) {
+    const float x = srow[j] * scale - m;
+    const float e = expf(x);
+    z += e;
+    t = fmaf(e, x, t);
+  }
+  for (int off = 16; off > 0; off >>= 1) {
+    z += __shfl_xor_sync(0xffffffffu, z, off);
+    t += __shfl_xor_sync(0xffffffffu, t, off);
+  }
+  if (lane == 0) entropy[row] = logf(z) - t / z;
+}
+
+// ---- budgets (budget mode): one block per (b, h). Z = sum_i exp(H_i) over the query tiles
+// of the head in a fixed order (thread-strided partial sums, then a fixed tree), so every
+// row sees the same value; then, per row, budget = round(tau * NKT * NQT * exp(H_i) / Z)
+// clipped to [1, NKT], the largest decayed-window radius whose window fits in it, and the
+// number of tiles left for the score ranking.
+constexpr int kBudgetThreads = 256;
+
+__global__ void __launch_bounds__(kBudgetThreads) budget_kernel(Geom g, const float* __restrict__ entropy,
+                                                                const uint8_t* __restrict__ dense,
+                                                                double tau, int2* __restrict__ plan) {
+  __shared__ double part[kBudgetThreads];
+  const int NKT = g.NT, NQT = g.NT;
+  const long long bh = blockIdx.x;
+  const int b = (int)(bh / g.H);
+  const int tid = threadIdx.x;
+  double z = 0.0;
+  for (int i = tid; i < NQT; i += kBudgetThreads) z += exp((double)entropy[bh * NQT + i]);
+  part[tid] = z;
+  __syncthreads();
+  for (int n = kBudgetThreads / 2; n > 0; n >>= 1) {
+    if (tid < n) part[tid] += part[tid + n];
+    __syncthreads();
+  }
+  const double zsum = part[0];
+  const int rmax = g.nT + g.nY + g.nX;
+  for (int i = tid; i < NQT; i += kBudgetThreads) {
+    const long long rowid = bh * NQT + i;
+    if (dense[(long long)b * NQT + i]) {
+      plan[rowid] = make_int2(0, 0);
+      continue;
+    }
+    const double x = tau * (double)NKT * (double)NQT * exp((double)entropy[rowid]) / zsum;
+    const int budget = (int)fmin(fmax(floor(x + 0.5), 1.0), (double)NKT);
+    int tt, ty, tx;
+    tile_xyz(g, i, tt, ty, tx);
+    int rad = 0, wsize = 1;
+    while (rad < rmax && wsize < NKT) {
+      const int next = decayed_window_size(g, tt, ty, tx, rad + 1);
+      if (next > budget) break;
+      ++rad;
+      wsize = next;
+    }
+    plan[rowid] = make_int2(rad, budget - wsize);
+  }
+}
+
+// ---- selection: one warp per (b, h, query tile) row, eight rows per block.
+template <int MODE, int KW>
+__global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const float* __restrict__ S, int NKTP) {
+  extern __shared__ __align__(16) uint32_t sm_u32[];
   const Geom& g = a.g;
   const int NKT = g.NT, NQT = g.NT;
-  const int NKTP = (NKT + 3) & ~3;
-  const int b = blockIdx.z, h = blockIdx.y, i0 = blockIdx.x * ROWS;
+  const int b = blockIdx.z, h = blockIdx.y, i0 = blockIdx.x * kSelWarps;
   const long long bh = (long long)b * g.H + h;
-
-  float* qs = smem;                                               // ROWS * DP
-  float* ks = qs + ROWS * DP;                                     // kKeyChunk * DP
-  float* sc = ks + kKeyChunk * DP;                                // ROWS * NKTP
-  uint32_t* coord = reinterpret_cast<uint32_t*>(sc + ROWS * NKTP); // NKTP
-  double* dsum = reinterpret_cast<double*>(coord + NKTP);
-
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint32_t* coord = sm_u32;                                   // NKTP tile coordinates
 
-  // query means of this row block, tile coordinate table
-  const float4* qbar4 = reinterpret_cast<const float4*>(a.qbar);
-  for (int e = tid; e < ROWS * (D / 4); e += kSelThreads) {
-    const int r = e / (D / 4), c4 = e % (D / 4);
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i0 + r < NQT) v = qbar4[(bh * g.NT + i0 + r) * (D / 4) + c4];
-    reinterpret_cast<float4*>(qs + r * DP)[c4] = v;
-  }
   for (int j = tid; j < NKT; j += kSelThreads) {
     int tt, ty, tx;
     tile_xyz(g, j, tt, ty, tx);
     coord[j] = pack_coord(tt, ty, tx);
   }
-  if (MODE == kSelectBudget && warp == 0) {
-    // sum_i exp(H_i) over every query tile of this (b, h), fixed order: lane-strided
-    // partial sums, then a fixed butterfly; every block computes the same value.
-    double s = 0.0;
-    for (int i = lane; i < NQT; i += 32) s += exp((double)a.entropy[bh * NQT + i]);
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (lane == 0) *dsum = s;
-  }
-
-  // pooled scores qbar . kbar (unscaled) for ROWS x NKT
-  const float4* kbar4 = reinterpret_cast<const float4*>(a.kbar);
-  const int grow = tid / TPR, gk = tid % TPR;
-  for (int c0 = 0; c0 < NKT; c0 += kKeyChunk) {
-    __syncthreads();
-    for (int e = tid; e < kKeyChunk * (D / 4); e += kSelThreads) {
-      const int kr = e / (D / 4), c4 = e % (D / 4);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c0 + kr < NKT) v = kbar4[(bh * g.NT + c0 + kr) * (D / 4) + c4];
-      reinterpret_cast<float4*>(ks + kr * DP)[c4] = v;
-    }
-    __syncthreads();
-    float acc[KPT];
-#pragma unroll
-    for (int u = 0; u < KPT; ++u) acc[u] = 0.f;
-    const float4* qrow = reinterpret_cast<const float4*>(qs + grow * DP);
-#pragma unroll 4
-    for (int c4 = 0; c4 < D / 4; ++c4) {
-      const float4 q = qrow[c4];
-#pragma unroll
-      for (int u = 0; u < KPT; ++u) {
-        const float4 k = reinterpret_cast<const float4*>(ks + (gk + u * TPR) * DP)[c4];
-        acc[u] = fmaf(q.x, k.x, acc[u]);
-        acc[u] = fmaf(q.y, k.y, acc[u]);
-        acc[u] = fmaf(q.z, k.z, acc[u]);
-        acc[u] = fmaf(q.w, k.w, acc[u]);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < KPT; ++u) {
-      const int j = c0 + gk + u * TPR;
-      if (j < NKT) sc[grow * NKTP + j] = acc[u];
-    }
-  }
   __syncthreads();
 
-  // one warp per query row
-  for (int rr = warp; rr < ROWS; rr += kSelWarps) {
-    const int i = i0 + rr;
-    if (i >= NQT) break;
-    const float* srow = sc + rr * NKTP;
-    const long long rowid = bh * NQT + i;
-
-    if (MODE == kEntropy) {
-      // H = log Z - sum(e (s - m)) / Z with s = scale * qbar.kbar, e = exp(s - m)
-      float m = -INFINITY;
-      for (int j = lane; j < NKT; j += 32) m = fmaxf(m, srow[j] * a.scale);
-      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      float z = 0.f, t = 0.f;
-      for (int j = lane; j < NKT; j += 32) {
-        const float x = srow[j] * a.scale - m;
-        const float e = expf(x);
-        z += e;
-        t = fmaf(e, x, t);
-      }
-      for (int off = 16; off > 0; off >>= 1) {
-        z += __shfl_xor_sync(0xffffffffu, z, off);
-        t += __shfl_xor_sync(0xffffffffu, t, off);
-      }
-      if (lane == 0) a.entropy[rowid] = logf(z) - t / z;
-      continue;
+  const int i = i0 + warp;
+  if (i >= NQT) return;
+  const long long rowid = bh * NQT + i;
+  const float* srow = S + rowid * NKTP;
+  uint32_t* mrow = a.mask + rowid * g.NW;
+  if (a.dense[(long long)b * NQT + i]) {
+    for (int w = lane; w < g.NW; w += 32) {
+      const int rem = NKT - 32 * w;
+      mrow[w] = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
     }
-
-    uint32_t* mrow = a.mask + rowid * g.NW;
-    if (a.dense[(long long)b * NQT + i]) {
-      for (int w = lane; w < g.NW; w += 32) {
-        const int rem = NKT - 32 * w;
-        mrow[w] = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
-      }
-      if (lane == 0) a.kv_count[rowid] = NKT;
-      continue;
-    }
-
-    const uint32_t ci = coord[i];
-    int kind = a.window_kind, rad = a.radius, extra;
-    if (MODE == kSelectFixed) {
-      int wsize = 0;
-      for (int w = 0; w < g.NW; ++w) {
-        const int j = 32 * w + lane;
-        wsize += __popc(__ballot_sync(0xffffffffu, j < NKT && in_window(ci, coord[j], kind, rad)));
-      }
-      extra = min(a.topk, NKT - wsize);
-    } else {
-      const double x = a.tau * (double)NKT * (double)NQT * exp((double)a.entropy[rowid]) / *dsum;
-      int budget = (int)floor(x + 0.5);
-      budget = max(1, min(budget, NKT));
-      const int tt = (int)(ci >> 20), ty = (int)((ci >> 10) & 1023u), tx = (int)(ci & 1023u);
-      kind = 1;
-      rad = 0;
-      int wsize = 1;
-      const int rmax = g.nT + g.nY + g.nX;
-      while (rad < rmax && wsize < NKT) {
-        const int next = decayed_window_size(g, tt, ty, tx, rad + 1);
-        if (next > budget) break;
-        ++rad;
-        wsize = next;
-      }
-      extra = budget - wsize;
-    }
-
-    // Order-preserving integer keys of the candidates (tiles outside the window), written
-    // over the row's scores; 0 marks a window tile or a slot beyond NKT (no real score maps
-    // to 0 or 1).
-    uint32_t* krow = reinterpret_cast<uint32_t*>(sc + rr * NKTP);
-    int ncand = 0;
-    for (int w = 0; w < g.NW; ++w) {
-      const int j = 32 * w + lane;
-      const bool cand = j < NKT && !in_window(ci, coord[j], kind, rad);
-      if (j < NKTP) krow[j] = cand ? order_key(srow[j]) : 0u;
-      ncand += __popc(__ballot_sync(0xffffffffu, cand));
-    }
-    __syncwarp();
-    extra = max(0, min(extra, ncand));
-
-    int count = 0;
-    if (extra == ncand || extra <= 32) {
-      // Few extra tiles (or all of them): repeated warp argmax, the largest key first and
-      // the lowest tile index among equal keys; a chosen tile's key becomes 1.
-      for (int round = 0; round < extra && extra < ncand; ++round) {
-        uint64_t best = 0;
-        for (int w = 0; w < g.NW; ++w) {
-          const int j = 32 * w + lane;
-          const uint32_t k = j < NKTP ? krow[j] : 0u;
-          const uint64_t v = ((uint64_t)k << 32) | (uint32_t)(0xffffffffu - (uint32_t)j);
-          best = (k > 1u && v > best) ? v : best;
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
-          best = o > best ? o : best;
-        }
-        const int jbest = (int)(0xffffffffu - (uint32_t)best);
-        if (lane == 0) krow[jbest] = 1u;
-        __syncwarp();
-      }
-      for (int w = 0; w < g.NW; ++w) {
-        const int j = 32 * w + lane;
-        bool sel = false;
-        if (j < NKT) {
-          const uint32_t k = krow[j];
-          sel = k <= 1u || extra == ncand;        // window (0), chosen (1), or every candidate
-        }
-        const uint32_t bits = __ballot_sync(0xffffffffu, sel);
-        if (lane == 0) mrow[w] = bits;
-        count += __popc(bits);
-      }
-    } else {
-      // Many extra tiles: bitwise binary search for the extra-th largest key T, counting
-      // with warp reductions (no atomics); then every key above T and, among keys equal to
-      // T, the lowest tile indices.
-      uint32_t thr = 0u;
-      for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t cand_t = thr | (1u << bit);
-        int c = 0;
-        for (int w = 0; w < g.NW; ++w) {
-          const int j = 32 * w + lane;
-          c += (j < NKTP && krow[j] >= cand_t) ? 1 : 0;
-        }
-        c = __reduce_add_sync(0xffffffffu, c);
-        if (c >= extra) thr = cand_t;
-      }
-      int gt = 0;
-      for (int w = 0; w < g.NW; ++w) {
-        const int j = 32 * w + lane;
-        gt += (j < NKTP && krow[j] > thr) ? 1 : 0;
-      }
-      const int need_eq = extra - __reduce_add_sync(0xffffffffu, gt);
-      int eq_before = 0;
-      for (int w = 0; w < g.NW; ++w) {
-        const int j = 32 * w + lane;
-        bool sel = false, eq = false;
-        if (j < NKT) {
-          const uint32_t k = krow[j];
-          sel = k == 0u || k > thr;
-          eq = k == thr;
-        }
-        const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
-        const int rank = eq_before + __popc(eqb & ((1u << lane) - 1u));
-        sel = sel || (eq && rank < need_eq);
-        eq_before += __popc(eqb);
-        const uint32_t bits = __ballot_sync(0xffffffffu, sel);
-        if (lane == 0) mrow[w] = bits;
-        count += __popc(bits);
-      }
-    }
-    if (lane == 0) a.kv_count[rowid] = count;
+    if (lane == 0) a.kv_count[rowid] = NKT;
+    return;
   }
+
+  const uint32_t ci = coord[i];
+  int kind = a.window_kind, rad = a.radius, extra;
+  if (MODE == kSelectFixed) {
+    extra = a.topk;
+  } else {
+    const int2 pl = a.plan[rowid];
+    kind = 1;
+    rad = pl.x;
+    extra = pl.y;
+  }
+
+  // Order-preserving integer keys of the candidates (tiles outside the window), held in
+  // registers: element j = 32*w + lane is kr[w]. 0 marks a window tile or a slot beyond NKT
+  // (no real score maps to 0 or 1).
+  uint32_t kr[KW];
+  int ncand = 0;
+#pragma unroll
+  for (int w = 0; w < KW; ++w) {
+    const int j = 32 * w + lane;
+    const bool cand = j < NKT && !in_window(ci, coord[j], kind, rad);
+    kr[w] = cand ? order_key(srow[j]) : 0u;
+    if (w < g.NW) ncand += __popc(__ballot_sync(0xffffffffu, cand));
+  }
+  extra = max(0, min(extra, ncand));
+
+  // Threshold key thr and how many keys equal to it to take (need_eq, lowest index first):
+  // every key > thr is selected. extra == ncand selects every candidate.
+  // extra and ncand are warp-uniform by construction; the explicit broadcast from lane 0 is
+  // kept because builds without it (nvcc 12.9, -O3) selected every candidate of budget-mode
+  // rows, a code-generation effect whose cause was not identified.
+  extra = __shfl_sync(0xffffffffu, extra, 0);
+  ncand = __shfl_sync(0xffffffffu, ncand, 0);
+  uint32_t thr;
+  int need_eq;
+  if (extra == 0) {
+    thr = 0xffffffffu;
+    need_eq = 0;
+  } else if (extra == ncand) {
+    thr = 1u;
+    need_eq = 0;
+  } else if (extra <= 32) {
+    // Few extra tiles: repeated warp argmax, the largest key first and the lowest tile
+    // index among equal keys; a chosen key becomes 0xffffffff (above any score's key) and
+    // thr = 0xfffffffe then selects exactly the chosen.
+    for (int round = 0; round < extra; ++round) {
+      uint64_t best = 0;
+#pragma unroll
+      for (int w = 0; w < KW; ++w) {
+        const uint32_t j = 32u * w + lane;
+        const uint64_t v = ((uint64_t)kr[w] << 32) | (0xffffffffu - j);
+        best = (kr[w] > 1u && kr[w] != 0xffffffffu && v > best) ? v : best;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
+        best = o > best ? o : best;
+      }
+      const uint32_t jbest = 0xffffffffu - (uint32_t)best;
+#pragma unroll
+      for (int w = 0; w < KW; ++w)
+        if (32u * w + lane == jbest) kr[w] = 0xffffffffu;      // chosen: above any score
+    }
+    thr = 0xfffffffeu;
+    need_eq = 0;
+  } else {
+    // Many extra tiles: bitwise binary search for the largest thr with at least `extra`
+    // keys >= thr, counting with warp reductions; it stops early once exactly `extra`
+    // keys are >= the candidate, which then needs no tie pass.
+    uint32_t t = 0u;
+    bool exact = false;
+    for (int bit = 31; bit >= 0 && !exact; --bit) {
+      const uint32_t cand_t = t | (1u << bit);
+      int c = 0;
+#pragma unroll
+      for (int w = 0; w < KW; ++w) c += kr[w] >= cand_t ? 1 : 0;
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (c >= extra) t = cand_t;
+      exact = c == extra;
+    }
+    if (exact) {
+      thr = t - 1u;           // every key >= t, i.e. > t - 1
+      need_eq = 0;
+    } else {
+      int gt = 0;
+#pragma unroll
+      for (int w = 0; w < KW; ++w) gt += kr[w] > t ? 1 : 0;
+      thr = t;
+      need_eq = extra - __reduce_add_sync(0xffffffffu, gt);
+    }
+  }
+
+  // The row: window | key > thr | (key == thr, among the first need_eq in index order).
+  int count = 0, eq_before = 0;
+#pragma unroll
+  for (int w = 0; w < KW; ++w) {
+    if (w < g.NW) {
+      const int j = 32 * w + lane;
+      const uint32_t k = kr[w];
+      const bool inrow = j < NKT;
+      bool sel = inrow && (k == 0u || k > thr);
+      const bool eq = inrow && k != 0u && k == thr;
+      const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+      const int rank = eq_before + __popc(eqb & ((1u << lane) - 1u));
+      sel = sel || (eq && rank < need_eq);
+      eq_before += __popc(eqb);
+      const uint32_t bits = __ballot_sync(0xffffffffu, sel);
+      if (lane == 0) mrow[w] = bits;
+      count += __popc(bits);
+    }
+  }
+  if (lane == 0) a.kv_count[rowid] = count;
 }
 
-template <int D, int ROWS, int MODE>
-cudaError_t run_select(const SelArgs& a, cudaStream_t s) {
-  const Geom& g = a.g;
-  const int NKTP = (g.NT + 3) & ~3;
-  const size_t smem = sizeof(float) * ((size_t)(ROWS + kKeyChunk) * (D + 4) + (size_t)ROWS * NKTP) +
-                      sizeof(uint32_t) * (size_t)NKTP + sizeof(double);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<D, ROWS, MODE>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+template <int MODE, int KW>
+cudaError_t launch_select_kw(dim3 grid, size_t smem, const SelArgs& a, const float* S, int NKTP, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<MODE, KW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(ceil_div(g.NT, ROWS), g.H, g.B);
-  select_kernel<D, ROWS, MODE><<<grid, kSelThreads, smem, s>>>(a);
-  count_launches(1);
+  select_kernel<MODE, KW><<<grid, kSelThreads, smem, s>>>(a, S, NKTP);
   return cudaGetLastError();
 }
 
-template <int D, int MODE>
-cudaError_t run_select_rows(const SelArgs& a, cudaStream_t s) {
-  // 16 query rows per block while the score rows fit in shared memory, else 8.
-  const size_t rows16 = sizeof(float) * ((size_t)(16 + kKeyChunk) * (D + 4) + 16ull * ((a.g.NT + 3) & ~3)) +
-                        sizeof(uint32_t) * (size_t)((a.g.NT + 3) & ~3) + 8;
-  if (rows16 <= 200 * 1024) return run_select<D, 16, MODE>(a, s);
-  return run_select<D, 8, MODE>(a, s);
+template <int MODE>
+cudaError_t launch_select(int kw, dim3 grid, size_t smem, const SelArgs& a, const float* S, int NKTP,
+                          cudaStream_t s) {
+  switch (kw) {
+    case 8: return launch_select_kw<MODE, 8>(grid, smem, a, S, NKTP, s);
+    case 16: return launch_select_kw<MODE, 16>(grid, smem, a, S, NKTP, s);
+    case 32: return launch_select_kw<MODE, 32>(grid, smem, a, S, NKTP, s);
+    case 64: return launch_select_kw<MODE, 64>(grid, smem, a, S, NKTP, s);
+    default: return launch_select_kw<MODE, 128>(grid, smem, a, S, NKTP, s);
+  }
 }
 
 template <int D>
@@ -411,6 +454,7 @@ cudaError_t build_mask_d(const Geom& g, const bsa_mask_params& p, const __nv_bfl
   float* kbar = reinterpret_cast<float*>(ws + L.kbar);
   uint8_t* dense = ws + L.dense;
   float* entropy = reinterpret_cast<float*>(ws + L.entropy);
+  int2* plan = reinterpret_cast<int2*>(ws + L.plan);
 
   const long long warps = 2LL * g.B * g.H * g.NT;
   pool_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(g, qt, kt, qbar, kbar);
@@ -430,17 +474,46 @@ cudaError_t build_mask_d(const Geom& g, const bsa_mask_params& p, const __nv_bfl
   a.radius = p.radius;
   a.topk = p.topk;
   a.scale = 1.0f / sqrtf((float)g.d);
-  a.tau = (double)p.budget_target;
   a.qbar = qbar;
   a.kbar = kbar;
   a.dense = dense;
   a.entropy = entropy;
+  a.plan = plan;
   a.mask = mask;
   a.kv_count = kv_count;
-  if (p.budget_mode == 0) return run_select_rows<D, kSelectFixed>(a, s);
-  e = run_select_rows<D, kEntropy>(a, s);
+
+  float* S = reinterpret_cast<float*>(ws + L.scores);
+  const int NKTP = (g.NT + 3) & ~3;
+  const size_t score_smem = 2 * D * kScorePad * sizeof(float);
+  e = cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)score_smem);
   if (e != cudaSuccess) return e;
-  return run_select_rows<D, kSelectBudget>(a, s);
+  score_kernel<D><<<dim3(ceil_div(g.NT, kScoreTile), ceil_div(g.NT, kScoreTile), g.B * g.H), 256, score_smem, s>>>(
+      g, qbar, kbar, S, NKTP);
+  count_launches(1);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  const long long rows = (long long)g.B * g.H * g.NT;
+  if (p.budget_mode == 1) {
+    entropy_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(g, S, NKTP, a.scale, entropy);
+    count_launches(1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    budget_kernel<<<(unsigned)(g.B * g.H), kBudgetThreads, 0, s>>>(g, entropy, dense,
+                                                                  (double)p.budget_target, plan);
+    count_launches(1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const size_t sel_smem = sizeof(uint32_t) * (size_t)NKTP;
+  dim3 grid(ceil_div(g.NT, kSelWarps), g.H, g.B);
+  // words of a mask row per lane, rounded up to the kernel's register array
+  const int kw = g.NW <= 8 ? 8 : g.NW <= 16 ? 16 : g.NW <= 32 ? 32 : g.NW <= 64 ? 64 : 128;
+  e = (p.budget_mode == 0) ? launch_select<kSelectFixed>(kw, grid, sel_smem, a, S, NKTP, s)
+                           : launch_select<kSelectBudget>(kw, grid, sel_smem, a, S, NKTP, s);
+  if (e != cudaSuccess) return e;
+  count_launches(1);
+  return cudaGetLastError();
 }
 
 }  // namespace

@@ -50,9 +50,10 @@ def test_tile_grid_and_workspace(lib):
     assert lib.bsa_tile_grid(ctypes.byref(g.c()), *[ctypes.byref(o) for o in out]) == 0
     assert [o.value for o in out] == [6, 8, 13, 624]
     n = bsa.workspace_bytes(g)
-    pooled = 12 * 624 * 128 * 4
-    assert n >= 2 * pooled + 256 and n % 256 == 0
-    assert n < 2 * pooled + 4 * 1024 * 1024
+    pooled = 12 * 624 * 128 * 4          # qbar and kbar, fp32
+    scores = 12 * 624 * 624 * 4          # pooled scores, fp32, rows padded to 4
+    assert n >= 2 * pooled + scores + 256 and n % 256 == 0
+    assert n < 2 * pooled + scores + 4 * 1024 * 1024
 
 
 @pytest.mark.parametrize("bad", [
