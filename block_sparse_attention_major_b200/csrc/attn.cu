@@ -8,14 +8,18 @@
 // Work unit: up to four query tiles of one (b, h) and of the same route class (all
 // dense, or all local), consecutive in tile order. They form two sub-units of two tiles,
 // A and B, each one M=128 tcgen05 tile. The CTA streams the union of the four rows'
-// retained key tiles through one shared K/V ring, two key tiles (128 keys) per block.
-// Each sub-unit issues its MMAs only for the blocks it needs, with N=128, or N=64 on the
-// one tile it needs (descriptor offset), so no tensor work is spent on tiles that neither
-// of its two query tiles retains; a tile retained by only one of its two query tiles is
-// masked to -inf for the other half of the rows.
+// retained key tiles, in ascending order, through a K ring and a V ring of one key tile
+// (64 keys) per stage. A sub-unit's blocks are the union tiles one of its two query tiles
+// retains; for each it computes S = Q K^T (N=64) and O += P V, so no tensor work is spent
+// on tiles that neither of its query tiles retains; a tile retained by only one of them
+// gets zero probabilities in the other half of the rows.
 //
-// The two sub-units ping-pong on the tensor core: while softmax warpgroup A turns S_A
-// into P_A, the MMA warp runs P_B V and the next S_B = Q_B K^T, and the other way round.
+// Each sub-unit has two S buffers in TMEM. S of block c+1 is computed while the softmax
+// warpgroup turns S of block c into P (written as bf16 over S), so the softmax warpgroups
+// run back to back while the tensor pipe runs the other products. Each sub-unit has its
+// own issuing thread, which sends each product out as soon as its inputs and buffers are
+// ready; the two issuers cover each other's barrier tests, during which a single issuer
+// would leave the tensor pipe idle.
 //
 // Schedule (one launch each, on the caller's stream):
 //   sched_count  per (b, h): number of dense rows (kv_count == NKT) and local rows
@@ -24,18 +28,19 @@
 //   attn         one CTA per unit, in list order: heavy (dense) units first, and units of
 //                the same head next to each other so that their K/V tiles stay in L2.
 //
-// CTA roles (320 threads):
+// CTA roles (352 threads):
 //   warps 0-3  softmax of sub-unit A: thread t owns query row t = TMEM lane t
 //   warps 4-7  softmax of sub-unit B
 //              (each reads S from TMEM, writes P as bf16 pairs over S, rescales its O in
 //              TMEM when the running max grows, and runs the epilogue)
 //   warp 8     builds the key-tile lists in shared memory, then lane 0 issues the TMA
-//              loads of Q and of the K/V ring
-//   warp 9     allocates TMEM; lane 0 issues S = Q K^T (SS) and O += P V (TS)
-// TMEM columns: S_A 0-127, S_B 128-255, O_A 256-383, O_B 384-511.
-// Shared memory (1024-byte aligned): Q_A, Q_B, 2 K stages, 2 V stages, each
-// [D/64][128 rows][128 B] with the 128-byte swizzle that TMA and tcgen05 share; the
-// key-tile list; the per-sub-unit block lists; barriers.
+//              loads of Q and of the K/V rings
+//   warp 9     allocates TMEM; lane 0 issues S_A = Q_A K^T (SS) and O_A += P_A V (TS)
+//   warp 10    lane 0 issues the products of sub-unit B
+// TMEM columns: S buffers A0, A1, B0, B1 at 0, 64, 128, 192 (64 each); O_A at 256, O_B at
+// 256 + D. Shared memory (1024-byte aligned): Q_A, Q_B as [D/64][128 rows][128 B], four
+// K and four V stages as [D/64][64 rows][128 B], each with the 128-byte swizzle that TMA
+// and tcgen05 share; barriers; the key-tile list; the per-sub-unit block lists.
 #include "common.cuh"
 #include "sm100_ptx.cuh"
 #include "tmem_ops.cuh"
@@ -45,31 +50,32 @@
 namespace bsa {
 namespace {
 
-constexpr int kAttnThreads = 320;
-constexpr int kNSK = 2;                            // K ring stages
-constexpr int kNSV = 2;                            // V ring stages
-constexpr int kMaxBlocks = kMaxTiles / 2 + 1;
+constexpr int kAttnThreads = 352;
+constexpr int kNS = 4;                             // K and V ring stages, one key tile each
 constexpr long long kWaitLimit = 4000000000LL;     // SM cycles, about 2 s
 constexpr int kTmemCols = 512;
 constexpr int kUnitInts = 8;                       // {bh, q0, q1, q2, q3, 0, 0, 0}
 
 template <int D>
 struct Cfg {
-  static constexpr int kD = D;
   static constexpr int kTileBytes = 64 * D * 2;         // one 64-token tile
-  static constexpr int kBufBytes = 2 * kTileBytes;      // two tiles (128 rows)
-  static constexpr int kDBlockStride = 128 * 128;       // bytes between 64-column blocks
+  static constexpr int kQBytes = 2 * kTileBytes;        // one sub-unit's Q (128 rows)
+  static constexpr int kQDB = 128 * 128;                // Q: bytes between 64-column blocks
+  static constexpr int kKDB = 64 * 128;                 // K/V stage: bytes between 64-column blocks
   static constexpr int kQOff = 0;                       // Q_A, then Q_B
-  static constexpr int kKOff = 2 * kBufBytes;
-  static constexpr int kVOff = kKOff + kNSK * kBufBytes;
-  static constexpr int kBarOff = kVOff + kNSV * kBufBytes;
-  // barriers: q, kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], pfull[2], odone[2], drain
-  static constexpr int kNumBars = 1 + 2 * kNSK + 2 * kNSV + 2 + 2 + 2 + 1;
-  static constexpr int kMiscOff = kBarOff + kNumBars * 8;         // tmem base, counts, abort
-  static constexpr int kListOff = kMiscOff + 64;
-  static constexpr int kBlkOff = kListOff + kMaxTiles * 4;        // uint16 block lists A, B
-  static constexpr int kNeedOff = kBlkOff + 2 * kMaxBlocks * 2;   // uint8 per block
-  static constexpr int kSmemBytes = 1024 + kNeedOff + kMaxBlocks;
+  static constexpr int kKOff = 2 * kQBytes;
+  static constexpr int kVOff = kKOff + kNS * kTileBytes;
+  static constexpr int kBarOff = kVOff + kNS * kTileBytes;
+  // barriers: q, kfull[NS], kempty[NS], vfull[NS], vempty[NS], sfull[4] (sub-unit u,
+  // S buffer b at 2u + b), pfull[2], odone[2], drain[2] (one per issuer)
+  static constexpr int kNumBars = 1 + 4 * kNS + 4 + 2 + 2 + 2;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base, counts, abort, stage counters
+  static constexpr int kListOff = kMiscOff + 128;
+  static constexpr int kBlkOff = kListOff + kMaxTiles * 4;  // uint16 block lists of A and B
+  static constexpr int kSmemBytes = 1024 + kBlkOff + 2 * kMaxTiles * 2;
+  // TMEM columns: S buffer b of sub-unit u at 64 (2u + b); O of sub-unit u at 256 + u D.
+  static constexpr uint32_t s_col(int u, int b) { return 64u * (2u * u + b); }
+  static constexpr uint32_t o_col(int u) { return 256u + (uint32_t)(u * D); }
 };
 
 struct AttnArgs {
@@ -232,66 +238,6 @@ __device__ __forceinline__ void rescale_o(uint32_t o_tmem, float alpha) {
   }
 }
 
-// MMA-issue state of one sub-unit: block whose P.V is pending (-1: none), the tile slots
-// it uses, and the number of P.V products issued so far.
-struct SubUnitIssue {
-  int pend;
-  uint32_t pneed;
-  int npv;
-};
-
-// What the MMA-issuing thread needs: TMEM base, descriptors of the Q / K / V stage bases
-// (an offset of x bytes adds x >> 4 to a descriptor), barrier addresses.
-struct MmaCtx {
-  uint32_t tmem;
-  uint64_t dQ0, dK0, dV0;
-  uint32_t pfull0, vfull0, vempty0, sfull0, odone0;
-  volatile int* abort;
-  uint32_t* err;
-};
-
-// O_u += P_u V for the pending block of sub-unit u, then release its V stage once no other
-// product still reads it.
-template <class C>
-__device__ __forceinline__ bool issue_pv(SubUnitIssue& st, int u, const MmaCtx& m, int& vref0, int& vref1) {
-  constexpr uint32_t kIdPV = ptx::idesc_bf16_f32(128, C::kD, 0, 1);
-  const int j = st.pend;
-  const int sv = j & 1;
-  if (!ptx::mbar_wait(m.pfull0 + 8 * u, st.npv & 1, m.abort, m.err, kWaitLimit)) return false;
-  if (!ptx::mbar_wait(m.vfull0 + 8 * sv, (j >> 1) & 1, m.abort, m.err, kWaitLimit)) return false;
-  ptx::tc_fence_after();
-  const uint32_t p_tmem = m.tmem + 128 * u;
-  const uint32_t o_tmem = m.tmem + 256 + 128 * u;
-  const uint64_t vd = m.dV0 + sv * (C::kBufBytes >> 4) + (st.pneed == 2u ? (8192u >> 4) : 0u);
-  const int nk = (st.pneed == 3u) ? 8 : 4;
-  for (int kk = 0; kk < nk; ++kk)
-    ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + kk * (2048 >> 4), kIdPV, (st.npv > 0 || kk > 0) ? 1u : 0u);
-  ptx::mma_commit(m.odone0 + 8 * u);
-  ++st.npv;
-  const int left = sv ? --vref1 : --vref0;
-  if (left == 0) ptx::mma_commit(m.vempty0 + 8 * sv);
-  st.pend = -1;
-  return true;
-}
-
-// S_u = Q_u K^T on the needed tile slots n of block j.
-template <class C, int D>
-__device__ __forceinline__ void issue_qk(SubUnitIssue& st, int u, int j, uint32_t n, const MmaCtx& m) {
-  constexpr uint32_t kIdQK128 = ptx::idesc_bf16_f32(128, 128, 0, 0);
-  constexpr uint32_t kIdQK64 = ptx::idesc_bf16_f32(128, 64, 0, 0);
-  const uint64_t qd = m.dQ0 + u * (C::kBufBytes >> 4);
-  const uint64_t kd = m.dK0 + (j & 1) * (C::kBufBytes >> 4) + (n == 2u ? (8192u >> 4) : 0u);
-  const uint32_t id = n == 3u ? kIdQK128 : kIdQK64;
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = ((kk >> 2) * C::kDBlockStride + (kk & 3) * 32) >> 4;
-    ptx::mma_ss(m.tmem + 128 * u, qd + off, kd + off, id, kk > 0 ? 1u : 0u);
-  }
-  ptx::mma_commit(m.sfull0 + 8 * u);
-  st.pend = j;
-  st.pneed = n;
-}
-
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -317,29 +263,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const bool hasB = q2 >= 0;
 
   const uint32_t bar0 = sbase + C::kBarOff;
-  // barrier addresses: q, kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], pfull[2], odone[2], drain
   const uint32_t bar_q = bar0;
-  const uint32_t kfull0 = bar0 + 8, kempty0 = bar0 + 24, vfull0 = bar0 + 40, vempty0 = bar0 + 56;
-  const uint32_t sfull0 = bar0 + 72, pfull0 = bar0 + 88, odone0 = bar0 + 104, bar_drain = bar0 + 120;
+  const uint32_t kfull0 = bar0 + 8, kempty0 = kfull0 + 8 * kNS, vfull0 = kempty0 + 8 * kNS,
+                 vempty0 = vfull0 + 8 * kNS;
+  const uint32_t sfull0 = vempty0 + 8 * kNS, pfull0 = sfull0 + 32, odone0 = pfull0 + 16,
+                 bar_drain = odone0 + 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
-  int* counts = reinterpret_cast<int*>(smem + C::kMiscOff + 4);        // L, cntA, cntB
+  int* counts = reinterpret_cast<int*>(smem + C::kMiscOff + 4);        // L, nA, nB
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 16);
   uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::kListOff);
-  uint16_t* blk = reinterpret_cast<uint16_t*>(smem + C::kBlkOff);      // [2][kMaxBlocks]
-  uint8_t* needs = smem + C::kNeedOff;                                  // per block: nA | nB << 2
+  uint16_t* blk = reinterpret_cast<uint16_t*>(smem + C::kBlkOff);      // [2][kMaxTiles]
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar_q, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kNS; ++s) {
       ptx::mbar_init(kfull0 + 8 * s, 1);
-      ptx::mbar_init(kempty0 + 8 * s, 1);
+      ptx::mbar_init(kempty0 + 8 * s, hasB ? 2 : 1);     // one arrival per issuer
       ptx::mbar_init(vfull0 + 8 * s, 1);
-      ptx::mbar_init(vempty0 + 8 * s, 1);
-      ptx::mbar_init(sfull0 + 8 * s, 1);
-      ptx::mbar_init(pfull0 + 8 * s, 128);
-      ptx::mbar_init(odone0 + 8 * s, 1);
+      ptx::mbar_init(vempty0 + 8 * s, hasB ? 2 : 1);
+    }
+    for (int s = 0; s < 4; ++s) ptx::mbar_init(sfull0 + 8 * s, 1);
+    for (int u = 0; u < 2; ++u) {
+      ptx::mbar_init(pfull0 + 8 * u, 128);
+      ptx::mbar_init(odone0 + 8 * u, 1);
     }
     ptx::mbar_init(bar_drain, 1);
+    ptx::mbar_init(bar_drain + 8, 1);
     *abort = 0;
     ptx::fence_mbar_init();
   }
@@ -394,24 +343,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       running += __shfl_sync(0xffffffffu, incl, 31);
     }
     __syncwarp();
-    // Per-sub-unit block lists (entry = block | need << 12) and per-block needs, where
-    // need bit t = tile slot t of the block is retained by one of the sub-unit's tiles.
-    const int L = running, nblk = (L + 1) >> 1;
+    // Per-sub-unit block lists: the union entries one of the sub-unit's two query tiles
+    // retains, in union order (one key tile per block), each with the number of sub-units
+    // that use it (bits 13-14).
+    const int L = running;
     int ca = 0, cb = 0;
-    for (int j0 = 0; j0 < nblk; j0 += 32) {
-      const int j = j0 + lane;
-      uint32_t na = 0, nb = 0;
-      if (j < nblk) {
-        const uint32_t e0 = list[2 * j];
-        const uint32_t e1 = (2 * j + 1 < L) ? list[2 * j + 1] : 0u;
-        na = (((e0 >> 16) & 3u) ? 1u : 0u) | (((e1 >> 16) & 3u) ? 2u : 0u);
-        nb = (((e0 >> 18) & 3u) ? 1u : 0u) | (((e1 >> 18) & 3u) ? 2u : 0u);
-        needs[j] = (uint8_t)(na | (nb << 2));
-      }
-      const uint32_t ba = __ballot_sync(0xffffffffu, na != 0), bb = __ballot_sync(0xffffffffu, nb != 0);
+    for (int i0 = 0; i0 < L; i0 += 32) {
+      const int i = i0 + lane;
+      const uint32_t e = i < L ? list[i] : 0u;
+      const bool na = ((e >> 16) & 3u) != 0u, nb = ((e >> 18) & 3u) != 0u;
+      const uint32_t ba = __ballot_sync(0xffffffffu, na), bb = __ballot_sync(0xffffffffu, nb);
       const uint32_t lt = (1u << lane) - 1u;
-      if (na) blk[ca + __popc(ba & lt)] = (uint16_t)(j | (na << 12));
-      if (nb) blk[kMaxBlocks + cb + __popc(bb & lt)] = (uint16_t)(j | (nb << 12));
+      const uint16_t ent = (uint16_t)(i | ((na && nb ? 2 : 1) << 13));   // entry | users << 13
+      if (na) blk[ca + __popc(ba & lt)] = ent;
+      if (nb) blk[kMaxTiles + cb + __popc(bb & lt)] = ent;
       ca += __popc(ba);
       cb += __popc(bb);
     }
@@ -426,101 +371,155 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int L = counts[0];
-  const int nblk = (L + 1) >> 1;
-  if (nblk == 0 && threadIdx.x == 0) report_error(a.err, BSA_KERR_BAD_MASK);
+  if (L == 0 && threadIdx.x == 0) report_error(a.err, BSA_KERR_BAD_MASK);
   const long long tile_row0 = (long long)bh * g.NT;   // tile index base of this (b, h)
 
   if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0 && nblk > 0) {
-      int last_k0 = -1, last_k1 = -1, last_v0 = -1, last_v1 = -1;
+    if (lane == 0 && L > 0) {
       const int nsub = hasB ? 2 : 1;
-      ptx::mbar_arrive_expect_tx(bar_q, nsub * C::kBufBytes);
+      ptx::mbar_arrive_expect_tx(bar_q, nsub * C::kQBytes);
       for (int t = 0; t < 2 * nsub; ++t) {
         const int qt = t == 0 ? q0 : t == 1 ? q1 : t == 2 ? q2 : q3;
         const int tile = qt >= 0 ? qt : (t < 2 ? q0 : q2);
         const int row = (int)((tile_row0 + tile) * 64);
-        const uint32_t dst = sbase + C::kQOff + (t >> 1) * C::kBufBytes + (t & 1) * 8192;
+        const uint32_t dst = sbase + C::kQOff + (t >> 1) * C::kQBytes + (t & 1) * 8192;
 #pragma unroll
-        for (int db = 0; db < D / 64; ++db) ptx::tma_load_2d(dst + db * C::kDBlockStride, &tmQ, bar_q, db * 64, row);
+        for (int db = 0; db < D / 64; ++db) ptx::tma_load_2d(dst + db * C::kQDB, &tmQ, bar_q, db * 64, row);
       }
-      for (int j = 0; j < nblk; ++j) {
-        const int nt = (2 * j + 1 < L) ? 2 : 1;
-        const int s = j & 1;
-        const uint32_t ph = ((j >> 1) & 1) ^ 1;
+      int nk = 0, nv = 0;       // tiles whose K / V load was issued
+      for (int i = 0; i < L; ++i) {
+        const int s = i % kNS;
+        const uint32_t ph = ((i / kNS) & 1) ^ 1;
+        const int row = (int)((tile_row0 + (int)(list[i] & 0xffffu)) * 64);
         if (!ptx::mbar_wait(kempty0 + 8 * s, ph, abort, a.err, kWaitLimit)) break;
-        ptx::mbar_arrive_expect_tx(kfull0 + 8 * s, nt * C::kTileBytes);
-        for (int t = 0; t < nt; ++t) {
-          const int row = (int)((tile_row0 + (int)(list[2 * j + t] & 0xffffu)) * 64);
-          const uint32_t dst = sbase + C::kKOff + s * C::kBufBytes + t * 8192;
+        ptx::mbar_arrive_expect_tx(kfull0 + 8 * s, C::kTileBytes);
 #pragma unroll
-          for (int db = 0; db < D / 64; ++db)
-            ptx::tma_load_2d(dst + db * C::kDBlockStride, &tmK, kfull0 + 8 * s, db * 64, row);
-        }
-        if (s) last_k1 = j; else last_k0 = j;
+        for (int db = 0; db < D / 64; ++db)
+          ptx::tma_load_2d(sbase + C::kKOff + s * C::kTileBytes + db * C::kKDB, &tmK, kfull0 + 8 * s, db * 64, row);
+        ++nk;
         if (!ptx::mbar_wait(vempty0 + 8 * s, ph, abort, a.err, kWaitLimit)) break;
-        ptx::mbar_arrive_expect_tx(vfull0 + 8 * s, nt * C::kTileBytes);
-        for (int t = 0; t < nt; ++t) {
-          const int row = (int)((tile_row0 + (int)(list[2 * j + t] & 0xffffu)) * 64);
-          const uint32_t dst = sbase + C::kVOff + s * C::kBufBytes + t * 8192;
+        ptx::mbar_arrive_expect_tx(vfull0 + 8 * s, C::kTileBytes);
 #pragma unroll
-          for (int db = 0; db < D / 64; ++db)
-            ptx::tma_load_2d(dst + db * C::kDBlockStride, &tmV, vfull0 + 8 * s, db * 64, row);
-        }
-        if (s) last_v1 = j; else last_v0 = j;
+        for (int db = 0; db < D / 64; ++db)
+          ptx::tma_load_2d(sbase + C::kVOff + s * C::kTileBytes + db * C::kKDB, &tmV, vfull0 + 8 * s, db * 64, row);
+        ++nv;
       }
       // Never leave with copies in flight: wait for the last load issued into each stage.
       int zero = 0;
-      if (last_k0 >= 0) ptx::mbar_wait(kfull0, (last_k0 >> 1) & 1, &zero, a.err, kWaitLimit);
-      if (last_k1 >= 0) ptx::mbar_wait(kfull0 + 8, (last_k1 >> 1) & 1, &zero, a.err, kWaitLimit);
-      if (last_v0 >= 0) ptx::mbar_wait(vfull0, (last_v0 >> 1) & 1, &zero, a.err, kWaitLimit);
-      if (last_v1 >= 0) ptx::mbar_wait(vfull0 + 8, (last_v1 >> 1) & 1, &zero, a.err, kWaitLimit);
+      for (int s = 0; s < kNS; ++s) {
+        if (nk > s) {
+          const int last = s + kNS * ((nk - 1 - s) / kNS);
+          ptx::mbar_wait(kfull0 + 8 * s, (last / kNS) & 1, &zero, a.err, kWaitLimit);
+        }
+        if (nv > s) {
+          const int last = s + kNS * ((nv - 1 - s) / kNS);
+          ptx::mbar_wait(vfull0 + 8 * s, (last / kNS) & 1, &zero, a.err, kWaitLimit);
+        }
+      }
       ptx::mbar_wait(bar_q, 0, &zero, a.err, kWaitLimit);
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nblk > 0) {
-      MmaCtx m;
-      m.tmem = tmem;
-      m.dQ0 = ptx::smem_desc_sw128(sbase + C::kQOff, 16, 1024);
-      m.dK0 = ptx::smem_desc_sw128(sbase + C::kKOff, 16, 1024);
-      m.dV0 = ptx::smem_desc_sw128(sbase + C::kVOff, C::kDBlockStride, 1024);
-      m.pfull0 = pfull0;
-      m.vfull0 = vfull0;
-      m.vempty0 = vempty0;
-      m.sfull0 = sfull0;
-      m.odone0 = odone0;
-      m.abort = abort;
-      m.err = a.err;
-      SubUnitIssue sA{-1, 0u, 0}, sB{-1, 0u, 0};
-      int vref0 = 0, vref1 = 0;     // P.V products still to read V stage 0 / 1
+  } else if (warp == 9 || warp == 10) {
+    // ------------------------------------------------------------------ MMA issuers
+    // One issuing thread per sub-unit (lane 0 of warp 9 for A, of warp 10 for B). Issue is
+    // throttled to the tensor pipe's pace, so a single thread leaves the pipe idle while it
+    // tests barriers between products; two threads cover each other's tests.
+    //
+    // Each issuer walks the whole union list in order with two cursors. K cursor: for an
+    // entry its sub-unit uses, S = Q K^T into the next S buffer once the K tile is in and
+    // the buffer is free (the P.V two blocks back has been issued: the tensor pipe runs a
+    // thread's products in issue order, so S of block c can overwrite the P of block c - 2
+    // issued before it), then a commit on the stage's empty barrier; for any other entry, a
+    // plain arrive there once the entry's K tile was seen loaded. V cursor: for an entry it
+    // uses, O += P V once its softmax has written P and the V tile is in, then a commit on
+    // the stage's empty barrier; for any other entry, a plain arrive once its V tile was
+    // seen loaded. The empty barriers count one arrival per issuer, so a stage is reloaded
+    // only after both issuers' products on it have completed (a commit tracks its own
+    // thread's products). Because each cursor sees every load of its ring in order, the
+    // full barrier is never more than one phase behind the entry tested and the parity
+    // tests are exact. Nothing blocks: a wait on one cursor could hold up the other.
+    static_assert(kNS == 4, "stage arithmetic below assumes four stages");
+    const int u = warp - 9;
+    if (lane == 0 && L > 0 && (u == 0 || hasB)) {
+      constexpr uint32_t kIdQK = ptx::idesc_bf16_f32(128, 64, 0, 0);
+      constexpr uint32_t kIdPV = ptx::idesc_bf16_f32(128, D, 0, 1);
+      constexpr int kNoEntry = 1 << 20;
+      const uint64_t qd = ptx::smem_desc_sw128(sbase + C::kQOff + u * C::kQBytes, 16, 1024);
+      const uint64_t dK0 = ptx::smem_desc_sw128(sbase + C::kKOff, 16, 1024);
+      const uint64_t dV0 = ptx::smem_desc_sw128(sbase + C::kVOff, C::kKDB, 1024);
+      const uint32_t o_tmem = tmem + C::o_col(u);
+      const uint32_t pfull_u = pfull0 + 8 * u, odone_u = odone0 + 8 * u;
+      const int n = counts[1 + u];
+      const uint16_t* my_blk = blk + u * kMaxTiles;
+      int qc = 0, pc = 0, ki = 0, vi = 0;
+      int qnext = n > 0 ? (int)(my_blk[0] & 0x1fffu) : kNoEntry;   // union index of the next QK block
+      int pnext = qnext;                                            // and of the next P.V block
       bool ok = ptx::mbar_wait(bar_q, 0, abort, a.err, kWaitLimit);
-
-      for (int j = 0; j < nblk && ok; ++j) {
-        const uint32_t nn = needs[j];
-        const uint32_t nA = nn & 3u, nB = nn >> 2;
-        if (!ptx::mbar_wait(kfull0 + 8 * (j & 1), (j >> 1) & 1, abort, a.err, kWaitLimit)) break;
-        ptx::tc_fence_after();
-        if (j & 1) vref1 = (nA != 0u) + (nB != 0u); else vref0 = (nA != 0u) + (nB != 0u);
-        if (nA) {
-          if (sA.pend >= 0 && !issue_pv<C>(sA, 0, m, vref0, vref1)) break;
-          issue_qk<C, D>(sA, 0, j, nA, m);
+      long long idle_since = clock64();
+      while (ok && vi < L) {
+        bool progress = false;
+        if (ki < L) {
+          const uint32_t s = ki & 3;
+          if (ki == qnext) {
+            if (qc - pc < 2 && ptx::mbar_test_wait(kfull0 + 8 * s, (ki >> 2) & 1)) {
+              // No tcgen05 fence: K arrived through the TMA barrier, and the S buffer is
+              // reused behind this thread's own P.V (ordered by the fence on that path).
+              const uint32_t s_tmem = tmem + C::s_col(u, qc & 1);
+              const uint64_t kd = dK0 + s * (C::kTileBytes >> 4);
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk)
+                ptx::mma_ss(s_tmem, qd + (((kk >> 2) * C::kQDB + (kk & 3) * 32) >> 4),
+                            kd + (((kk >> 2) * C::kKDB + (kk & 3) * 32) >> 4), kIdQK, kk > 0 ? 1u : 0u);
+              ptx::mma_commit(sfull0 + 8 * (2 * u + (qc & 1)));
+              ptx::mma_commit(kempty0 + 8 * s);
+              ++qc;
+              qnext = qc < n ? (int)(my_blk[qc] & 0x1fffu) : kNoEntry;
+              ++ki;
+              progress = true;
+            }
+          } else if (ptx::mbar_test_wait(kfull0 + 8 * s, (ki >> 2) & 1)) {
+            ptx::mbar_arrive(kempty0 + 8 * s);
+            ++ki;
+            progress = true;
+          }
         }
-        if (nB) {
-          if (sB.pend >= 0 && !issue_pv<C>(sB, 1, m, vref0, vref1)) break;
-          issue_qk<C, D>(sB, 1, j, nB, m);
+        if (vi < ki) {
+          const uint32_t s = vi & 3;
+          if (vi == pnext) {
+            if (ptx::mbar_test_wait(pfull_u, pc & 1) && ptx::mbar_test_wait(vfull0 + 8 * s, (vi >> 2) & 1)) {
+              ptx::tc_fence_after();
+              const uint32_t p_tmem = tmem + C::s_col(u, pc & 1);
+              const uint64_t vd = dV0 + s * (C::kTileBytes >> 4);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + kk * (2048 >> 4), kIdPV, (pc > 0 || kk > 0) ? 1u : 0u);
+              ptx::mma_commit(odone_u);
+              ptx::mma_commit(vempty0 + 8 * s);
+              ++pc;
+              pnext = pc < n ? (int)(my_blk[pc] & 0x1fffu) : kNoEntry;
+              ++vi;
+              progress = true;
+            }
+          } else if (ptx::mbar_test_wait(vfull0 + 8 * s, (vi >> 2) & 1)) {
+            ptx::mbar_arrive(vempty0 + 8 * s);
+            ++vi;
+            progress = true;
+          }
         }
-        ptx::mma_commit(kempty0 + 8 * (j & 1));
-        // P.V of a sub-unit that has no work in the next block goes out now, so that every
-        // V stage is released within one block of its use.
-        const uint32_t nn1 = (j + 1 < nblk) ? needs[j + 1] : 0u;
-        if (sA.pend >= 0 && (nn1 & 3u) == 0u && !issue_pv<C>(sA, 0, m, vref0, vref1)) break;
-        if (sB.pend >= 0 && (nn1 >> 2) == 0u && !issue_pv<C>(sB, 1, m, vref0, vref1)) break;
+        if (progress) {
+          idle_since = clock64();
+        } else if (*abort) {
+          ok = false;
+        } else if (clock64() - idle_since > kWaitLimit) {
+          *abort = 1;
+          report_error(a.err, BSA_KERR_WAIT_TIMEOUT);
+          ok = false;
+        }
       }
       // Never free TMEM under a running MMA: wait until everything issued has completed.
       int zero = 0;
-      ptx::mma_commit(bar_drain);
-      ptx::mbar_wait(bar_drain, 0, &zero, a.err, kWaitLimit);
+      ptx::mma_commit(bar_drain + 8 * u);
+      ptx::mbar_wait(bar_drain + 8 * u, 0, &zero, a.err, kWaitLimit);
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
@@ -529,43 +528,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int half = row >> 6;
     const int qt = u ? (half ? q3 : q2) : (half ? q1 : q0);   // this row's query tile (-1: none)
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t s_tmem = tmem + 128 * u + lane_base;
-    const uint32_t o_tmem = tmem + 256 + 128 * u + lane_base;
-    const uint32_t sfull_u = sfull0 + 8 * u, pfull_u = pfull0 + 8 * u, odone_u = odone0 + 8 * u;
-    const int cnt = counts[1 + u];
-    const uint16_t* my_blk = blk + u * kMaxBlocks;
+    const uint32_t o_tmem = tmem + C::o_col(u) + lane_base;
+    const uint32_t pfull_u = pfull0 + 8 * u, odone_u = odone0 + 8 * u;
+    const int n = counts[1 + u];
+    const uint16_t* my_blk = blk + u * kMaxTiles;
     const int mshift = 16 + 2 * u + half;
     const float c = a.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
-    bool ok = cnt > 0;
-    for (int it = 0; it < cnt; ++it) {
-      if (!warp_wait(sfull_u, it & 1, abort, a.err)) { ok = false; break; }
+    bool ok = n > 0;
+    for (int it = 0; it < n; ++it) {
+      const int b = it & 1;
+      if (!warp_wait(sfull0 + 8 * (2 * u + b), (it >> 1) & 1, abort, a.err)) { ok = false; break; }
       ptx::tc_fence_after();
-      const uint32_t bj = my_blk[it];
-      const int j = bj & 4095;
-      const uint32_t n = bj >> 12;
-      const bool two = n == 3u;                    // tile slots 0 and 1 both used
-      const uint32_t e0 = list[2 * j];
-      const uint32_t e1 = (2 * j + 1 < L) ? list[2 * j + 1] : 0u;
-      const uint32_t ea = (n & 1u) ? e0 : e1;      // tile in S columns 0-63
-      const int use_a = tile_use(ea, mshift);
-      const int use_b = two ? tile_use(e1, mshift) : kUseSkip;
-      const uint64_t val_a = use_a == kUsePartial ? entry_valid_mask(ea, g) : ~0ull;
-      const uint64_t val_b = use_b == kUsePartial ? entry_valid_mask(e1, g) : ~0ull;
-      // Tile b's scores are read twice (max, then exponentials) instead of being kept
-      // live next to tile a's, which keeps the warpgroup within its register budget.
+      const uint32_t e = list[my_blk[it] & 0x1fffu];
+      const uint32_t s_tmem = tmem + C::s_col(u, b) + lane_base;
+      const int use = tile_use(e, mshift);
+      const uint64_t valid = use == kUsePartial ? entry_valid_mask(e, g) : ~0ull;
+      uint32_t r[64];
       float mx = -INFINITY;
-      if (use_b != kUseSkip) {
-        uint32_t rb[64];
-        tmem_ld64(s_tmem + 64, rb);
+      if (use != kUseSkip) {
+        tmem_ld64(s_tmem, r);
         ptx::tmem_wait_ld();
-        mx = tile_max(rb, use_b, val_b, mx);
-      }
-      uint32_t ra[64];
-      if (use_a != kUseSkip) {
-        tmem_ld64(s_tmem, ra);
-        ptx::tmem_wait_ld();
-        mx = tile_max(ra, use_a, val_a, mx);
+        mx = tile_max(r, use, valid, mx);
       }
       // The reference follows the running max exactly, so the row's largest probability
       // is 2^0 = 1, which bf16 holds exactly: rows dominated by one key lose nothing to
@@ -575,18 +559,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float alpha = grow ? ex2(m_run - m_new) : 1.0f;
       const float m_use = (m_new == -INFINITY) ? 0.0f : m_new;
       float sum = 0.f;
-      tile_exp(ra, use_a, val_a, c, m_use, sum, s_tmem);
-      if (two) {
-        uint32_t rb[64];
-        if (use_b != kUseSkip) {
-          tmem_ld64(s_tmem + 64, rb);
-          ptx::tmem_wait_ld();
-        }
-        tile_exp(rb, use_b, val_b, c, m_use, sum, s_tmem + 32);
-      }
+      tile_exp(r, use, valid, c, m_use, sum, s_tmem);
       l_run = l_run * alpha + sum;
       if (it > 0) {
-        // O must hold exactly the previous blocks before it is rescaled.
+        // The previous block's P.V must be complete: O is rescaled only over exactly the
+        // previous blocks, and P of this block is released only after it, so that the
+        // issuing thread never sees P phases two ahead of the products it has issued.
         if (!warp_wait(odone_u, (it - 1) & 1, abort, a.err)) { ok = false; break; }
         ptx::tc_fence_after();
         if (__any_sync(0xffffffffu, grow)) rescale_o<D>(o_tmem, alpha);
@@ -596,7 +574,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ptx::mbar_arrive(pfull_u);
       m_run = m_new;
     }
-    if (ok && warp_wait(odone_u, (cnt - 1) & 1, abort, a.err)) {
+    if (ok && warp_wait(odone_u, (n - 1) & 1, abort, a.err)) {
       ptx::tc_fence_after();
       const int r = row & 63;
       int n_tok = -1;
@@ -607,8 +585,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (t < g.T && y < g.Hs && xx < g.Ws) n_tok = (t * g.Hs + y) * g.Ws + xx;
       }
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
-      const int b = bh / g.H, h = bh - b * g.H;
-      uint4* dst = n_tok >= 0 ? reinterpret_cast<uint4*>(a.out + (((long long)b * g.N + n_tok) * g.H + h) * D) : nullptr;
+      const int bb = bh / g.H, h = bh - bb * g.H;
+      uint4* dst = n_tok >= 0 ? reinterpret_cast<uint4*>(a.out + (((long long)bb * g.N + n_tok) * g.H + h) * D) : nullptr;
 #pragma unroll 1
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t ov[32];
