@@ -280,16 +280,41 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(Geom g, const fl
   }
 }
 
-// ---- selection: one warp per (b, h, query tile) row, eight rows per block.
-template <int MODE, int KW>
+// ---- selection: one (b, h, query tile) row per WPR warps (1, 2 or 4), 8 / WPR rows per
+// block. Warp q of a row holds the keys of mask words [q KW, (q + 1) KW) in registers,
+// lane l the key of tile 32 w + l of each word w. Counts, maxima and tie prefixes of a row
+// are combined across its warps through a double-buffered shared exchange and a named
+// barrier per row (ids 1-8), so large rows need no more than 32 words per lane.
+
+// Row-wide combination of one 64-bit value per warp (sum or max), warp-uniform result.
+template <int WPR, bool kMax>
+__device__ __forceinline__ uint64_t row_combine(uint64_t v, volatile uint64_t* xb, int& par, int q, int rw) {
+  if (WPR == 1) return v;
+  if ((threadIdx.x & 31) == 0) xb[par * WPR + q] = v;
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + rw), "r"(WPR * 32) : "memory");
+  uint64_t r = kMax ? 0ull : 0ull;
+#pragma unroll
+  for (int k = 0; k < WPR; ++k) {
+    const uint64_t x = xb[par * WPR + k];
+    r = kMax ? (x > r ? x : r) : r + x;
+  }
+  par ^= 1;
+  return r;
+}
+
+template <int MODE, int KW, int WPR>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const float* __restrict__ S, int NKTP) {
   extern __shared__ __align__(16) uint32_t sm_u32[];
+  constexpr int kRows = kSelWarps / WPR;
   const Geom& g = a.g;
   const int NKT = g.NT, NQT = g.NT;
-  const int b = blockIdx.z, h = blockIdx.y, i0 = blockIdx.x * kSelWarps;
+  const int b = blockIdx.z, h = blockIdx.y;
   const long long bh = (long long)b * g.H + h;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rw = warp / WPR, q = warp % WPR;                 // row in block, warp in row
   uint32_t* coord = sm_u32;                                   // NKTP tile coordinates
+  volatile uint64_t* xb = reinterpret_cast<volatile uint64_t*>(sm_u32 + ((NKTP + 1) & ~1)) + rw * 2 * WPR;
+  int par = 0;
 
   for (int j = tid; j < NKT; j += kSelThreads) {
     int tt, ty, tx;
@@ -298,17 +323,17 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
   }
   __syncthreads();
 
-  const int i = i0 + warp;
-  if (i >= NQT) return;
+  const int i = blockIdx.x * kRows + rw;
+  if (i >= NQT) return;                                       // whole row: its warps leave together
   const long long rowid = bh * NQT + i;
   const float* srow = S + rowid * NKTP;
   uint32_t* mrow = a.mask + rowid * g.NW;
   if (a.dense[(long long)b * NQT + i]) {
-    for (int w = lane; w < g.NW; w += 32) {
+    for (int w = q * 32 + lane; w < g.NW; w += 32 * WPR) {
       const int rem = NKT - 32 * w;
       mrow[w] = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
     }
-    if (lane == 0) a.kv_count[rowid] = NKT;
+    if (q == 0 && lane == 0) a.kv_count[rowid] = NKT;
     return;
   }
 
@@ -324,26 +349,27 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
   }
 
   // Order-preserving integer keys of the candidates (tiles outside the window), held in
-  // registers: element j = 32*w + lane is kr[w]. 0 marks a window tile or a slot beyond NKT
-  // (no real score maps to 0 or 1).
+  // registers: element j = 32 (q KW + w) + lane is kr[w]. 0 marks a window tile or a slot
+  // beyond NKT (no real score maps to 0 or 1).
   uint32_t kr[KW];
   int ncand = 0;
 #pragma unroll
   for (int w = 0; w < KW; ++w) {
-    const int j = 32 * w + lane;
+    const int j = 32 * (q * KW + w) + lane;
     const bool cand = j < NKT && !in_window(ci, coord[j], kind, rad);
     kr[w] = cand ? order_key(srow[j]) : 0u;
-    if (w < g.NW) ncand += __popc(__ballot_sync(0xffffffffu, cand));
+    ncand += __popc(__ballot_sync(0xffffffffu, cand));
   }
+  ncand = (int)row_combine<WPR, false>((uint64_t)ncand, xb, par, q, rw);
   extra = max(0, min(extra, ncand));
-
-  // Threshold key thr and how many keys equal to it to take (need_eq, lowest index first):
-  // every key > thr is selected. extra == ncand selects every candidate.
-  // extra and ncand are warp-uniform by construction; the explicit broadcast from lane 0 is
+  // extra and ncand are row-uniform by construction; the explicit broadcast from lane 0 is
   // kept because builds without it (nvcc 12.9, -O3) selected every candidate of budget-mode
   // rows, a code-generation effect whose cause was not identified.
   extra = __shfl_sync(0xffffffffu, extra, 0);
   ncand = __shfl_sync(0xffffffffu, ncand, 0);
+
+  // Threshold key thr and how many keys equal to it to take (need_eq, lowest index first):
+  // every key > thr is selected. extra == ncand selects every candidate.
   uint32_t thr;
   int need_eq;
   if (extra == 0) {
@@ -353,14 +379,14 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
     thr = 1u;
     need_eq = 0;
   } else if (extra <= 32) {
-    // Few extra tiles: repeated warp argmax, the largest key first and the lowest tile
-    // index among equal keys; a chosen key becomes 0xffffffff (above any score's key) and
-    // thr = 0xfffffffe then selects exactly the chosen.
+    // Few extra tiles: repeated argmax over the row, the largest key first and the lowest
+    // tile index among equal keys; a chosen key becomes 0xffffffff (above any score's key)
+    // and thr = 0xfffffffe then selects exactly the chosen.
     for (int round = 0; round < extra; ++round) {
       uint64_t best = 0;
 #pragma unroll
       for (int w = 0; w < KW; ++w) {
-        const uint32_t j = 32u * w + lane;
+        const uint32_t j = 32u * (q * KW + w) + lane;
         const uint64_t v = ((uint64_t)kr[w] << 32) | (0xffffffffu - j);
         best = (kr[w] > 1u && kr[w] != 0xffffffffu && v > best) ? v : best;
       }
@@ -369,17 +395,18 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
         const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
         best = o > best ? o : best;
       }
+      best = row_combine<WPR, true>(best, xb, par, q, rw);
       const uint32_t jbest = 0xffffffffu - (uint32_t)best;
 #pragma unroll
       for (int w = 0; w < KW; ++w)
-        if (32u * w + lane == jbest) kr[w] = 0xffffffffu;      // chosen: above any score
+        if (32u * (q * KW + w) + lane == jbest) kr[w] = 0xffffffffu;      // chosen: above any score
     }
     thr = 0xfffffffeu;
     need_eq = 0;
   } else {
     // Many extra tiles: bitwise binary search for the largest thr with at least `extra`
-    // keys >= thr, counting with warp reductions; it stops early once exactly `extra`
-    // keys are >= the candidate, which then needs no tie pass.
+    // keys >= thr; it stops early once exactly `extra` keys are >= the candidate, which
+    // then needs no tie pass.
     uint32_t t = 0u;
     bool exact = false;
     for (int bit = 31; bit >= 0 && !exact; --bit) {
@@ -387,7 +414,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
       int c = 0;
 #pragma unroll
       for (int w = 0; w < KW; ++w) c += kr[w] >= cand_t ? 1 : 0;
-      c = __reduce_add_sync(0xffffffffu, c);
+      c = (int)row_combine<WPR, false>((uint64_t)__reduce_add_sync(0xffffffffu, c), xb, par, q, rw);
       if (c >= extra) t = cand_t;
       exact = c == extra;
     }
@@ -398,17 +425,34 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
       int gt = 0;
 #pragma unroll
       for (int w = 0; w < KW; ++w) gt += kr[w] > t ? 1 : 0;
+      gt = (int)row_combine<WPR, false>((uint64_t)__reduce_add_sync(0xffffffffu, gt), xb, par, q, rw);
       thr = t;
-      need_eq = extra - __reduce_add_sync(0xffffffffu, gt);
+      need_eq = extra - gt;
     }
   }
 
+  // Keys equal to thr in the warps before this one (index order runs warp by warp).
+  int eq_before = 0;
+  if (WPR > 1 && need_eq > 0) {
+    int eqc = 0;
+#pragma unroll
+    for (int w = 0; w < KW; ++w) {
+      const int j = 32 * (q * KW + w) + lane;
+      eqc += (j < NKT && kr[w] != 0u && kr[w] == thr) ? 1 : 0;
+    }
+    eqc = __reduce_add_sync(0xffffffffu, eqc);
+    // exclusive prefix over the row's warps: combine (count << 8 * q) sums, then unpack
+    const uint64_t packed = row_combine<WPR, false>((uint64_t)eqc << (16 * q), xb, par, q, rw);
+    for (int k = 0; k < q; ++k) eq_before += (int)((packed >> (16 * k)) & 0xffffu);
+  }
+
   // The row: window | key > thr | (key == thr, among the first need_eq in index order).
-  int count = 0, eq_before = 0;
+  int count = 0;
 #pragma unroll
   for (int w = 0; w < KW; ++w) {
-    if (w < g.NW) {
-      const int j = 32 * w + lane;
+    const int wg = q * KW + w;
+    if (wg < g.NW) {
+      const int j = 32 * wg + lane;
       const uint32_t k = kr[w];
       const bool inrow = j < NKT;
       bool sel = inrow && (k == 0u || k > thr);
@@ -418,31 +462,31 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
       sel = sel || (eq && rank < need_eq);
       eq_before += __popc(eqb);
       const uint32_t bits = __ballot_sync(0xffffffffu, sel);
-      if (lane == 0) mrow[w] = bits;
+      if (lane == 0) mrow[wg] = bits;
       count += __popc(bits);
     }
   }
-  if (lane == 0) a.kv_count[rowid] = count;
+  count = (int)row_combine<WPR, false>((uint64_t)count, xb, par, q, rw);
+  if (q == 0 && lane == 0) a.kv_count[rowid] = count;
 }
 
-template <int MODE, int KW>
-cudaError_t launch_select_kw(dim3 grid, size_t smem, const SelArgs& a, const float* S, int NKTP, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<MODE, KW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+template <int MODE, int KW, int WPR>
+cudaError_t launch_select_kw(const Geom& g, size_t smem, const SelArgs& a, const float* S, int NKTP, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<MODE, KW, WPR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  select_kernel<MODE, KW><<<grid, kSelThreads, smem, s>>>(a, S, NKTP);
+  const dim3 grid(ceil_div(g.NT, kSelWarps / WPR), g.H, g.B);
+  select_kernel<MODE, KW, WPR><<<grid, kSelThreads, smem, s>>>(a, S, NKTP);
   return cudaGetLastError();
 }
 
+// Words of a mask row per lane at most 32: rows of more than 32 words span 2 or 4 warps.
 template <int MODE>
-cudaError_t launch_select(int kw, dim3 grid, size_t smem, const SelArgs& a, const float* S, int NKTP,
-                          cudaStream_t s) {
-  switch (kw) {
-    case 8: return launch_select_kw<MODE, 8>(grid, smem, a, S, NKTP, s);
-    case 16: return launch_select_kw<MODE, 16>(grid, smem, a, S, NKTP, s);
-    case 32: return launch_select_kw<MODE, 32>(grid, smem, a, S, NKTP, s);
-    case 64: return launch_select_kw<MODE, 64>(grid, smem, a, S, NKTP, s);
-    default: return launch_select_kw<MODE, 128>(grid, smem, a, S, NKTP, s);
-  }
+cudaError_t launch_select(const Geom& g, size_t smem, const SelArgs& a, const float* S, int NKTP, cudaStream_t s) {
+  if (g.NW <= 8) return launch_select_kw<MODE, 8, 1>(g, smem, a, S, NKTP, s);
+  if (g.NW <= 16) return launch_select_kw<MODE, 16, 1>(g, smem, a, S, NKTP, s);
+  if (g.NW <= 32) return launch_select_kw<MODE, 32, 1>(g, smem, a, S, NKTP, s);
+  if (g.NW <= 64) return launch_select_kw<MODE, 32, 2>(g, smem, a, S, NKTP, s);
+  return launch_select_kw<MODE, 32, 4>(g, smem, a, S, NKTP, s);
 }
 
 template <int D>
@@ -505,12 +549,11 @@ cudaError_t build_mask_d(const Geom& g, const bsa_mask_params& p, const __nv_bfl
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  const size_t sel_smem = sizeof(uint32_t) * (size_t)NKTP;
-  dim3 grid(ceil_div(g.NT, kSelWarps), g.H, g.B);
-  // words of a mask row per lane, rounded up to the kernel's register array
-  const int kw = g.NW <= 8 ? 8 : g.NW <= 16 ? 16 : g.NW <= 32 ? 32 : g.NW <= 64 ? 64 : 128;
-  e = (p.budget_mode == 0) ? launch_select<kSelectFixed>(kw, grid, sel_smem, a, S, NKTP, s)
-                           : launch_select<kSelectBudget>(kw, grid, sel_smem, a, S, NKTP, s);
+  // coordinate table, then per row of the block a double-buffered exchange of one 64-bit
+  // value per warp
+  const size_t sel_smem = sizeof(uint32_t) * (size_t)((NKTP + 1) & ~1) + (size_t)kSelWarps * 2 * sizeof(uint64_t);
+  e = (p.budget_mode == 0) ? launch_select<kSelectFixed>(g, sel_smem, a, S, NKTP, s)
+                           : launch_select<kSelectBudget>(g, sel_smem, a, S, NKTP, s);
   if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();
