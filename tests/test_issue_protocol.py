@@ -1,0 +1,252 @@
+"""Discrete-event model of the attention kernel's pipeline protocol (CPU only).
+
+The attention kernel hands work between a TMA producer, one MMA-issuing thread per
+sub-unit and two softmax warpgroups through mbarriers that are tested by phase parity.
+This model replays that protocol on the unit lists of real masks under random
+interleavings and checks that it always finishes (no deadlock) and that every product
+reads the key/value tile it was meant to read (no stale ring stage).
+
+mbarrier semantics modelled: a phase completes when its expected arrival count is
+reached; a parity test for parity P succeeds when the current phase's parity differs from
+P, so a barrier two phases behind the awaited one looks complete (the hazard the kernel's
+issuers avoid by walking every entry of the union list in order). The tensor pipe runs
+products in issue order; a commit arrives once the products issued before it are done.
+
+A second, deliberately careless protocol (one issuer that tests a sub-unit's next entry
+without walking the others) is run too and must be caught, which shows the checker can
+see the hazard.
+"""
+import random
+
+import numpy as np
+import pytest
+
+import _cases as C
+from oracle import bsa_oracle as O
+
+NS = 4          # ring stages, one key tile each
+
+
+class Bar:
+    def __init__(self, count):
+        self.count, self.pending, self.k = count, count, 0
+
+    def arrive(self):
+        self.pending -= 1
+        if self.pending == 0:
+            self.k += 1
+            self.pending = self.count
+
+    def test(self, parity):
+        return (self.k & 1) != parity
+
+
+class Stale(Exception):
+    pass
+
+
+def units_from_mask(mask):
+    """Work units of one (b, h): the kernel's grouping of four consecutive rows per class
+    (rows retaining every key tile first), as (union list, used by A, used by B)."""
+    nt = mask.shape[0]
+    cnt = mask.sum(-1)
+    dense = [i for i in range(nt) if cnt[i] == nt]
+    local = [i for i in range(nt) if cnt[i] != nt]
+    out = []
+    for rows in (dense, local):
+        for u0 in range(0, len(rows), 4):
+            qs = rows[u0:u0 + 4] + [-1] * (4 - len(rows[u0:u0 + 4]))
+            mk = [mask[q] if q >= 0 else np.zeros(nt, bool) for q in qs]
+            union = np.nonzero(mk[0] | mk[1] | mk[2] | mk[3])[0]
+            out.append((len(union), [bool(mk[0][j] or mk[1][j]) for j in union],
+                        [bool(mk[2][j] or mk[3][j]) for j in union]))
+    return out
+
+
+def run_protocol(L, need_a, need_b, seed, careless=False):
+    """True if the unit finishes; False on deadlock; raises Stale on a wrong-tile read."""
+    rng = random.Random(seed)
+    need = [need_a, need_b]
+    has = [any(need_a), any(need_b)]
+    users = sum(has)
+    blk = [[i for i in range(L) if need[u][i]] for u in range(2)]
+    n = [len(b) for b in blk]
+    kfull, vfull = [Bar(1) for _ in range(NS)], [Bar(1) for _ in range(NS)]
+    kempty = [Bar(1 if careless else users) for _ in range(NS)]
+    vempty = [Bar(1 if careless else users) for _ in range(NS)]
+    sfull = [Bar(1) for _ in range(4)]
+    pfull, odone = [Bar(1) for _ in range(2)], [Bar(1) for _ in range(2)]
+    pipe, kload, vload = [], [], []
+    kdata, vdata = [None] * NS, [None] * NS
+    prod = [0, 'k']
+    ki, vi, qc, pc = [0, 0], [0, 0], [0, 0], [0, 0]
+    sm = [[0, 'wait_s'], [0, 'wait_s']]
+
+    def actions():
+        acts = []
+        i = prod[0]
+        if i < L:
+            s, ph = i % NS, ((i // NS) & 1) ^ 1
+            if prod[1] == 'k' and kempty[s].test(ph):
+                acts.append(('load_k',))
+            if prod[1] == 'v' and vempty[s].test(ph):
+                acts.append(('load_v',))
+        if kload:
+            acts.append(('tma_k',))
+        if vload:
+            acts.append(('tma_v',))
+        if pipe:
+            acts.append(('pipe',))
+        for u in range(2):
+            if not has[u]:
+                continue
+            if careless:
+                # one issuer per sub-unit that tests only its own next entries; the last
+                # user of a stage frees it
+                if qc[u] < n[u] and qc[u] - pc[u] < 2:
+                    e = blk[u][qc[u]]
+                    if kfull[e % NS].test((e // NS) & 1):
+                        acts.append(('qk', u))
+                if pc[u] < qc[u] and pfull[u].test(pc[u] & 1):
+                    e = blk[u][pc[u]]
+                    if vfull[e % NS].test((e // NS) & 1):
+                        acts.append(('pv', u))
+            else:
+                k = ki[u]
+                if k < L and kfull[k % NS].test((k // NS) & 1):
+                    if not need[u][k]:
+                        acts.append(('k_arrive', u))
+                    elif qc[u] - pc[u] < 2:
+                        acts.append(('qk', u))
+                v = vi[u]
+                if v < ki[u] and vfull[v % NS].test((v // NS) & 1):
+                    if not need[u][v]:
+                        acts.append(('v_arrive', u))
+                    elif pfull[u].test(pc[u] & 1):
+                        acts.append(('pv', u))
+            it, st = sm[u]
+            if it < n[u]:
+                if st == 'wait_s' and sfull[2 * u + (it & 1)].test((it >> 1) & 1):
+                    acts.append(('softmax_s', u))
+                if st == 'wait_o' and (it == 0 or odone[u].test((it - 1) & 1)):
+                    acts.append(('softmax_p', u))
+        return acts
+
+    def last_user(u, e, cursor):
+        o = 1 - u
+        return not need[o][e] or not has[o] or cursor[o] >= n[o] or blk[o][cursor[o]] > e
+
+    while True:
+        acts = actions()
+        finished = (prod[0] >= L and all(sm[u][0] >= n[u] for u in range(2))
+                    and all(pc[u] >= n[u] for u in range(2)))
+        if finished and not pipe and not kload and not vload:
+            return True
+        if not acts:
+            return False
+        a = rng.choice(acts)
+        kind = a[0]
+        if kind == 'load_k':
+            kload.append((prod[0] % NS, prod[0]))
+            prod[1] = 'v'
+        elif kind == 'load_v':
+            vload.append((prod[0] % NS, prod[0]))
+            prod[1] = 'k'
+            prod[0] += 1
+        elif kind == 'tma_k':
+            s, e = kload.pop(0)
+            kdata[s] = e
+            kfull[s].arrive()
+        elif kind == 'tma_v':
+            s, e = vload.pop(0)
+            vdata[s] = e
+            vfull[s].arrive()
+        elif kind == 'pipe':
+            op = pipe.pop(0)
+            if op[0] == 'commit':
+                op[1].arrive()
+            else:
+                _, which, s, e = op
+                if (kdata if which == 'k' else vdata)[s] != e:
+                    raise Stale(f"{which} product on entry {e} read stage {s} holding {(kdata if which == 'k' else vdata)[s]}")
+        elif kind == 'qk':
+            u = a[1]
+            e = blk[u][qc[u]]
+            s = e % NS
+            pipe += [('mma', 'k', s, e), ('commit', sfull[2 * u + (qc[u] & 1)])]
+            qc[u] += 1
+            if careless:
+                if last_user(u, e, qc):
+                    pipe.append(('commit', kempty[s]))
+            else:
+                pipe.append(('commit', kempty[s]))
+                ki[u] += 1
+        elif kind == 'k_arrive':
+            u = a[1]
+            kempty[ki[u] % NS].arrive()
+            ki[u] += 1
+        elif kind == 'pv':
+            u = a[1]
+            e = blk[u][pc[u]]
+            s = e % NS
+            pipe += [('mma', 'v', s, e), ('commit', odone[u])]
+            pc[u] += 1
+            if careless:
+                if last_user(u, e, pc):
+                    pipe.append(('commit', vempty[s]))
+            else:
+                pipe.append(('commit', vempty[s]))
+                vi[u] += 1
+        elif kind == 'v_arrive':
+            u = a[1]
+            vempty[vi[u] % NS].arrive()
+            vi[u] += 1
+        elif kind == 'softmax_s':
+            sm[a[1]][1] = 'wait_o'
+        elif kind == 'softmax_p':
+            u = a[1]
+            pfull[u].arrive()
+            sm[u] = [sm[u][0] + 1, 'wait_s']
+
+
+def _case_units(name):
+    w, q, k, v, diff = C.inputs(name)
+    ref = C.oracle_mask(w, O.reorder(O.to_f64(q), w.T, w.Hs, w.Ws),
+                        O.reorder(O.to_f64(k), w.T, w.Hs, w.Ws), diff.numpy())
+    m = ref["mask"]
+    return [u for b in range(m.shape[0]) for h in range(m.shape[1]) for u in units_from_mask(m[b, h])]
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiny_ragged", "small128", "ragged128", "budget128"])
+def test_two_issuer_protocol_finishes_and_reads_the_right_tiles(name):
+    for L, na, nb in _case_units(name):
+        for seed in range(12):
+            assert run_protocol(L, na, nb, seed), (name, L, seed)
+
+
+def test_random_sparse_unit_lists():
+    rng = np.random.default_rng(7)
+    for trial in range(150):
+        L = int(rng.integers(1, 40))
+        na = list(rng.random(L) < rng.uniform(0.1, 0.9))
+        nb = list(rng.random(L) < rng.uniform(0.1, 0.9))
+        for j in range(L):                       # every union entry has a user
+            if not (na[j] or nb[j]):
+                (na if rng.random() < 0.5 else nb)[j] = True
+        if trial % 5 == 0:                       # units without a second sub-unit
+            na, nb = [True] * L, [False] * L
+        for seed in range(4):
+            assert run_protocol(L, na, nb, seed), (trial, L, seed)
+
+
+def test_careless_protocol_is_caught():
+    """Testing only a sub-unit's own next entries lets it run two ring phases ahead of
+    the producer: the checker must report a deadlock or a stale-tile read."""
+    caught = 0
+    for L, na, nb in _case_units("budget128"):
+        for seed in range(12):
+            try:
+                caught += not run_protocol(L, na, nb, seed, careless=True)
+            except Stale:
+                caught += 1
+    assert caught > 0
