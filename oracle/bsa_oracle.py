@@ -17,6 +17,9 @@ It computes, plainly and in float64, what the method defines:
     pooled score, ties to the lower key index;
   * the entropy-to-budget-to-radius rule (Token Radius Attention, "Entropy-guided
     budgeting" and "Radius construction");
+  * a cumulative-mass variant of the extra tiles: beyond the window, the key tiles of
+    highest pooled probability until the row's retained pooled mass reaches a target
+    (Token Radius Attention summary: the keys needed to capture a target attention mass);
   * masked softmax attention over the retained tiles' valid keys, with a natural-log LSE,
     written back in raster token order.
 
@@ -37,6 +40,7 @@ import numpy as np
 TILE_EDGE = 4
 TILE_TOKENS = 64
 NEAR_TIE_REL = 1e-4
+MASS_NEAR_TIE = 1e-5
 
 
 # ----------------------------------------------------------------------------------------
@@ -225,6 +229,40 @@ def row_entropy(scores: np.ndarray) -> np.ndarray:
     return -plogp.sum(axis=-1)
 
 
+def pooled_probabilities(scores: np.ndarray) -> np.ndarray:
+    """Softmax over the last axis (all key tiles) of pooled scores, in float64."""
+    s = np.asarray(scores, dtype=np.float64)
+    e = np.exp(s - s.max(axis=-1, keepdims=True))
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def mass_extra(p_row: np.ndarray, scores_row: np.ndarray, window_row_: np.ndarray,
+               theta: float) -> tuple[int, bool]:
+    """Number of tiles outside the window that the cumulative-mass rule adds.
+
+    Reading of "the number of keys required to capture a target attention mass" (Token
+    Radius Attention summary) at tile granularity: the window is always kept; the tiles
+    outside it are taken in decreasing pooled score (ties to the lower index) until the
+    pooled probability of the whole row reaches theta, i.e. the smallest m with
+    mass(window) + mass(first m) >= theta (every tile outside the window when the target is
+    not reached). Returns (m, near) where near flags a row whose cumulative mass passes
+    within MASS_NEAR_TIE of the target at the crossing, where float32 sums may decide
+    either way.
+    """
+    R = theta - float(p_row[window_row_].sum())
+    cand = np.nonzero(~window_row_)[0]
+    if R <= 0.0 or cand.size == 0:
+        return 0, abs(R) < MASS_NEAR_TIE
+    order = cand[np.lexsort((cand, -scores_row[cand]))]
+    cum = np.cumsum(p_row[order])
+    m = int(np.searchsorted(cum, R, side="left")) + 1
+    if m > cand.size:
+        return int(cand.size), abs(cum[-1] - R) < MASS_NEAR_TIE
+    near = abs(cum[m - 1] - R) < MASS_NEAR_TIE or (m >= 2 and abs(R - cum[m - 2]) < MASS_NEAR_TIE) \
+        or (m == 1 and R < MASS_NEAR_TIE)
+    return m, bool(near)
+
+
 def entropy_budgets(H_row: np.ndarray, tau: float, NKT: int) -> tuple[np.ndarray, np.ndarray]:
     """Per-query-tile budgets of one (b, h): b_i proportional to exp(H_i).
 
@@ -265,9 +303,11 @@ def build_mask(qt: np.ndarray, kt: np.ndarray, difficulty: np.ndarray, *, T: int
     (HetA-DiT); give every other query tile its local window plus extra tiles by pooled
     score (fixed top-k, or an entropy-derived budget, Token Radius Attention).
 
-    Fixed mode: row = window(kind, radius) U top-k tiles outside the window (k capped at the
-    number of tiles outside it). Budget mode: row = decayed window of radius r_i U the top
-    (b_i - |window|) tiles outside it. Dense rows: every key tile.
+    Fixed mode (budget_mode 0): row = window(kind, radius) U top-k tiles outside the window
+    (k capped at the number of tiles outside it). Entropy budget (1): row = decayed window
+    of radius r_i U the top (b_i - |window|) tiles outside it. Cumulative mass (2): row =
+    window(kind, radius) U the fewest best tiles outside it that bring the row's pooled
+    probability to budget_target. Dense rows: every key tile.
 
     Returns dict(mask bool [B,H,NQT,NKT], count int [B,H,NQT], near_tie bool [B,H,NQT],
     qbar, kbar, scores, dense bool [B,NQT], budget, budget_x).
@@ -315,8 +355,23 @@ def build_mask(qt: np.ndarray, kt: np.ndarray, difficulty: np.ndarray, *, T: int
                     row[top_outside(S[b, h, i], Wi, m)] = True
                     mask[b, h, i] = row
                     near[b, h, i] = near_half or boundary_near_tie(S[b, h, i], Wi, m)
+    elif budget_mode == 2:
+        W = window(window_kind, radius, T, Hs, Ws)
+        theta = float(np.float32(budget_target))
+        P = pooled_probabilities(S)
+        for b in range(B):
+            for h in range(H):
+                for i in range(NQT):
+                    if dense[b, i]:
+                        mask[b, h, i, :] = True
+                        continue
+                    m, near_mass = mass_extra(P[b, h, i], S[b, h, i], W[i], theta)
+                    row = W[i].copy()
+                    row[top_outside(S[b, h, i], W[i], m)] = True
+                    mask[b, h, i] = row
+                    near[b, h, i] = near_mass or boundary_near_tie(S[b, h, i], W[i], m)
     else:
-        raise ValueError("budget_mode must be 0 or 1")
+        raise ValueError("budget_mode must be 0, 1 or 2")
     return dict(mask=mask, count=mask.sum(axis=-1).astype(np.int64), near_tie=near,
                 qbar=qbar, kbar=kbar, scores=S, dense=dense, budget=budget,
                 budget_x=budget_x)

@@ -442,6 +442,91 @@ def test_full_forward_tiny_is_dense():
     np.testing.assert_allclose(res["O"], ref.numpy(), rtol=1e-11, atol=1e-12)
 
 
+# ------------------------------------------------------------------------------ cumulative mass
+def _mass_mask(qt, kt, NT, T, Hs, Ws, theta, kind=1, radius=1):
+    return O.build_mask(qt, kt, np.zeros((1, NT), np.float32), T=T, Hs=Hs, Ws=Ws,
+                        window_kind=kind, radius=radius, topk=0, dense_fraction=0.0,
+                        budget_mode=2, budget_target=theta)
+
+
+def test_mass_uniform_scores_closed_form():
+    """Identical kbar: every pooled probability is 1/NKT, so the rule adds
+    ceil(theta * NKT - |window|) tiles (none when the window already holds theta), the
+    lowest-indexed ones outside the window."""
+    T, Hs, Ws, d = 8, 16, 16, 4
+    NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
+    e1 = np.zeros(d); e1[0] = 1.0
+    qt, kt = _planted(T, Hs, Ws, 1, d, [e1] * NT, 0.3 * e1)
+    W = O.window(1, 1, T, Hs, Ws)
+    for theta in (0.125, 0.5, 0.75, 1.0):
+        th = float(np.float32(theta))
+        res = _mass_mask(qt, kt, NT, T, Hs, Ws, theta)
+        for i in range(NT):
+            m = max(0, math.ceil(th * NT - W[i].sum() - 1e-9))
+            outside = [j for j in range(NT) if not W[i, j]]
+            assert set(np.nonzero(res["mask"][0, 0, i])[0]) == set(np.nonzero(W[i])[0]) | set(outside[:m])
+
+
+def test_mass_limits():
+    """theta = 1 keeps every tile; a target below the window's own mass keeps the window."""
+    T, Hs, Ws, d = 8, 16, 16, 8
+    NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
+    rng = np.random.default_rng(5)
+    qt = rng.standard_normal((1, 2, NT, 64, d)); kt = rng.standard_normal((1, 2, NT, 64, d))
+    full = _mass_mask(qt, kt, NT, T, Hs, Ws, 1.0)
+    assert full["mask"].all()
+    W = O.window(1, 1, T, Hs, Ws)
+    tiny = _mass_mask(qt, kt, NT, T, Hs, Ws, 1e-12)
+    assert np.array_equal(tiny["mask"][0, 0], W) and np.array_equal(tiny["mask"][0, 1], W)
+
+
+def test_mass_planted_dominant_tile():
+    """One key tile whose score dwarfs the rest carries almost all the pooled mass: a target
+    of one half adds exactly that tile (or nothing when it lies in the window)."""
+    T, Hs, Ws, d = 8, 16, 16, 4
+    NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
+    e1 = np.zeros(d); e1[0] = 1.0
+    star = 17
+    kvals = [e1 * (40.0 if j == star else 0.0) for j in range(NT)]
+    qt, kt = _planted(T, Hs, Ws, 1, d, kvals, e1)
+    res = _mass_mask(qt, kt, NT, T, Hs, Ws, 0.5)
+    W = O.window(1, 1, T, Hs, Ws)
+    for i in range(NT):
+        assert set(np.nonzero(res["mask"][0, 0, i])[0]) == set(np.nonzero(W[i])[0]) | {star}
+
+
+def test_mass_monotone_and_brute_force():
+    """Rows grow with theta, and each row equals a brute-force reading of the definition:
+    the shortest prefix of the (score desc, index asc) order outside the window whose mass,
+    with the window's, reaches theta."""
+    T, Hs, Ws, d = 6, 10, 9, 8
+    NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
+    rng = np.random.default_rng(9)
+    qt = 2 * rng.standard_normal((1, 1, NT, 64, d)); kt = 2 * rng.standard_normal((1, 1, NT, 64, d))
+    prev = None
+    W = O.window(0, 1, T, Hs, Ws)
+    for theta in (0.2, 0.4, 0.6, 0.8, 0.95):
+        res = _mass_mask(qt, kt, NT, T, Hs, Ws, theta, kind=0, radius=1)
+        cnt = res["count"][0, 0]
+        if prev is not None:
+            assert np.all(cnt >= prev)
+        prev = cnt
+        S = res["scores"][0, 0]
+        th = float(np.float32(theta))
+        for i in range(NT):
+            e = [math.exp(x - max(S[i])) for x in S[i]]
+            z = sum(e)
+            p = [x / z for x in e]
+            mass = sum(p[j] for j in range(NT) if W[i, j])
+            keep = {j for j in range(NT) if W[i, j]}
+            for j in sorted((j for j in range(NT) if not W[i, j]), key=lambda j: (-S[i, j], j)):
+                if mass >= th:
+                    break
+                keep.add(j)
+                mass += p[j]
+            assert set(np.nonzero(res["mask"][0, 0, i])[0]) == keep
+
+
 # ------------------------------------------------------------------------------ planted mistakes
 def test_pins_catch_planted_pool_divisor(monkeypatch):
     """Dividing by 64 instead of the valid count must break the raster-mean pin."""
@@ -470,3 +555,12 @@ def test_pins_catch_planted_tie_break(monkeypatch):
     monkeypatch.setattr(O, "top_outside", bad_top)
     with pytest.raises(AssertionError):
         test_topk_ties_go_to_lower_index()
+
+
+def test_pins_catch_planted_window_mass(monkeypatch):
+    """Forgetting the window's own mass (counting only the added tiles toward the target)
+    must break the closed-form mass pin."""
+    real = O.mass_extra
+    monkeypatch.setattr(O, "mass_extra", lambda p, s, w, t: real(p * np.where(w, 0.0, 1.0), s, w, t))
+    with pytest.raises(AssertionError):
+        test_mass_uniform_scores_closed_form()
