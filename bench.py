@@ -80,6 +80,35 @@ def _peaks():
     return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
 
 
+def _tile_valid_counts(g):
+    """Valid tokens of every tile (edge tiles of a grid that is not a multiple of 4 hold
+    fewer than 64)."""
+    import numpy as np
+    nT, nY, nX = (g.T + 3) // 4, (g.Hs + 3) // 4, (g.Ws + 3) // 4
+    vt = np.minimum(4, g.T - 4 * np.arange(nT))
+    vy = np.minimum(4, g.Hs - 4 * np.arange(nY))
+    vx = np.minimum(4, g.Ws - 4 * np.arange(nX))
+    return (vt[:, None, None] * vy[None, :, None] * vx[None, None, :]).reshape(-1)
+
+
+def _valid_token_flops(g, mask_i32):
+    """4 d sum over retained (query tile, key tile) pairs of n_valid(q) n_valid(k): the
+    FLOPs of the valid tokens only, printed beside the tile-granular headline."""
+    import numpy as np
+    bits = mask_i32.cpu().numpy().view(np.uint32)                   # [B, H, NQT, NW]
+    nv = _tile_valid_counts(g).astype(np.float64)
+    words = np.arange(g.NT) // 32
+    sh = np.arange(g.NT) % 32
+    keep = (bits[..., words] >> sh) & 1                              # [B, H, NQT, NKT]
+    return 4.0 * g.d * float(np.einsum("bhqk,q,k->", keep.astype(np.float64), nv, nv))
+
+
+def _mask_bytes(g):
+    """Algorithmic bytes of the mask build: the valid Q and K tokens read once (the pooling
+    pass), the bitmask and kv_count written."""
+    return 2 * g.B * g.N * g.H * g.d * 2 + g.B * g.H * g.NT * (g.NW + 1) * 4
+
+
 def _workload_desc(w, retention):
     return {
         "workload": (f"Wan-1.3B-480p-shaped attention call: B={w.B} heads={w.H} d={w.d} "
@@ -307,6 +336,7 @@ def run_ours(args):
     if bsa.read_error(bufs.ws) != 0:
         raise SystemExit("kernel error word set")
     retained = int(bufs.kv_count.sum().item())
+    mask_snapshot = bufs.mask.clone()          # the dense comparison below rewrites the mask
     dense_pairs = g.B * g.H * g.NT * g.NT
     flops_call = 4.0 * 64 * 64 * g.d * retained
     retention = retained / dense_pairs
@@ -342,7 +372,9 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     clocks = sampler.stop() if sampler else None
     elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end))
-    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in attn_ev]))
+    attn_each = np.array([a.elapsed_time(b) for a, b in attn_ev])
+    attn_ms = float(np.mean(attn_each))
+    attn_pct = {f"p{q}": float(np.percentile(attn_each, q)) for q in (10, 50, 90)}
     attn_ms = max_over_ranks(attn_ms)
     ms_step = elapsed_ms / args.steps
     total_flops = sum_over_ranks(flops_call) * args.steps
@@ -420,6 +452,7 @@ def run_ours(args):
     peak = peaks["bf16_sustained"] if capped else peaks["bf16"]
     other = peaks["bf16"] if capped else peaks["bf16_sustained"]
     attn_tflops = flops_call / (attn_ms * 1e-3) / 1e12
+    valid_flops = _valid_token_flops(g, mask_snapshot)
     traffic, traffic_src = _traffic()
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -427,7 +460,9 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": _workload_desc(w, retention),
         "attn_ms_per_call": attn_ms,
+        "attn_ms_per_call_percentiles": attn_pct,
         "attn_effective_tflops": attn_tflops,
+        "attn_valid_token_tflops": valid_flops / (attn_ms * 1e-3) / 1e12,
         "attn_frac_of_nominal_bf16_peak": attn_tflops / NOMINAL_BF16_TFLOPS,
         "dense_path": {"ms_per_call": dense_ms, "effective_tflops": dense_tflops,
                        "sparse_speedup": dense_ms / attn_ms},
@@ -475,6 +510,7 @@ def run_report(args):
     from bsa_synth import generate_difficulty, generate_qkv
 
     dev = torch.device("cuda", 0)
+    peaks = _peaks()
     torch.cuda.set_device(dev)
     cache = {}
     for name, w in _report_workloads():
@@ -492,23 +528,28 @@ def run_report(args):
         bsa.forward(g, p, q, k, v, diff, b)
         torch.cuda.synchronize()
         retained = int(b.kv_count.sum().item())
+        valid_flops = _valid_token_flops(g, b.mask)
         stages = {"reorder_qkv": lambda: [bsa.reorder(g, x, y) for x, y in ((q, b.qt), (k, b.kt), (v, b.vt))],
                   "build_mask": lambda: bsa.build_mask(g, p, b.qt, b.kt, diff, b.mask, b.kv_count, b.ws),
                   "sparse_attn": lambda: bsa.sparse_attn_fwd(g, b.qt, b.kt, b.vt, b.mask, b.kv_count, None,
                                                              b.out, b.lse, b.ws)}
-        res = {}
+        res, pct = {}, {}
         for st, fn in stages.items():
             for _ in range(max(3, args.warmup)):
                 fn()
             n = max(5, min(args.steps, 30))
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
             torch.cuda.synchronize()
-            e0.record()
-            for _ in range(n):
+            for e0, e1 in evs:
+                e0.record()
                 fn()
-            e1.record()
+                e1.record()
             torch.cuda.synchronize()
-            res[st] = e0.elapsed_time(e1) / n
+            each = [e0.elapsed_time(e1) for e0, e1 in evs]
+            res[st] = sum(each) / n
+            if st == "sparse_attn":
+                srt = sorted(each)
+                pct = {f"p{q}": srt[min(n - 1, int(round(q / 100 * (n - 1))))] for q in (10, 50, 90)}
         err = bsa.read_error(b.ws)
         flops = 4.0 * 64 * 64 * g.d * retained
         dense_pairs = g.B * g.H * g.NT * g.NT
@@ -534,6 +575,12 @@ def run_report(args):
             "attn_effective_tflops": flops / (res["sparse_attn"] * 1e-3) / 1e12,
             "step_effective_tflops": flops / (sum(res.values()) * 1e-3) / 1e12,
             "reorder_gbs": qkv_bytes / (res["reorder_qkv"] * 1e-3) / 1e9,
+            "reorder_frac_of_8tbs": qkv_bytes / (res["reorder_qkv"] * 1e-3) / 8e12,
+            "reorder_frac_of_measured_copy": qkv_bytes / (res["reorder_qkv"] * 1e-3) / (peaks["hbm"] * 1e9),
+            "mask_gbs": _mask_bytes(g) / (res["build_mask"] * 1e-3) / 1e9,
+            "mask_frac_of_8tbs": _mask_bytes(g) / (res["build_mask"] * 1e-3) / 8e12,
+            "attn_valid_token_tflops": valid_flops / (res["sparse_attn"] * 1e-3) / 1e12,
+            "attn_ms_percentiles": pct,
             "dense_ms": dense_ms,
             "dense_effective_tflops": 4.0 * 64 * 64 * g.d * dense_pairs / (dense_ms * 1e-3) / 1e12,
             "sparse_speedup_vs_own_dense": dense_ms / res["sparse_attn"],

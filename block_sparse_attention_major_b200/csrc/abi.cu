@@ -37,6 +37,10 @@ bool valid_params(const bsa_geom* g, const bsa_mask_params* p) {
   } else if (p->budget_mode == 1) {
     if (p->window_kind != 1) return false;
     if (!(p->budget_target > 0.0f && p->budget_target <= 1.0f)) return false;
+  } else if (p->budget_mode == 2) {
+    if (p->window_kind != 0 && p->window_kind != 1) return false;
+    if (p->radius < 0) return false;
+    if (!(p->budget_target > 0.0f && p->budget_target <= 1.0f)) return false;
   } else {
     return false;
   }

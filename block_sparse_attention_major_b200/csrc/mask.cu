@@ -12,8 +12,10 @@
 //  select    per (b, h, query tile): the local support - a cube window or a window whose
 //            spatial radius decays with the frame-tile distance (Token Radius Attention
 //            summary, "Radius construction") - plus the best tiles outside it by pooled
-//            score: a fixed top-k, or the remainder of a budget derived from the entropy
-//            (Token Radius Attention summary, "Entropy-guided budgeting").
+//            score: a fixed top-k, the remainder of a budget derived from the entropy
+//            (Token Radius Attention summary, "Entropy-guided budgeting"), or as many as
+//            it takes for the row's pooled probability to reach a target mass (the same
+//            summary: keys needed to capture a target attention mass).
 //
 // Selection works per row and per warp on order-preserving integer keys of
 // the fp32 scores: a few extra tiles by repeated warp argmax (largest key, then lowest
@@ -100,12 +102,13 @@ __global__ void __launch_bounds__(256) route_kernel(Geom g, const float* __restr
 }
 
 // ------------------------------------------------------------------------ selection
-enum SelMode { kSelectFixed = 0, kSelectBudget = 2 };
+enum SelMode { kSelectFixed = 0, kSelectMass = 1, kSelectBudget = 2 };
 
 struct SelArgs {
   Geom g;
   int window_kind, radius, topk;
-  float scale;                 // 1/sqrt(d), used by the entropy only
+  float scale;                 // 1/sqrt(d), for the entropy and the pooled probabilities
+  float theta;                 // cumulative-mass mode: target pooled probability of a row
   const float* qbar;
   const float* kbar;
   const uint8_t* dense;
@@ -302,6 +305,27 @@ __device__ __forceinline__ uint64_t row_combine(uint64_t v, volatile uint64_t* x
   return r;
 }
 
+// Row-wide float sum. The butterfly leaves each lane with its own rounding of the total, so
+// lane 0's value is broadcast first: every warp of the row then branches identically.
+template <int WPR>
+__device__ __forceinline__ float row_sum_f(float v, volatile uint64_t* xb, int& par, int q, int rw) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  v = __shfl_sync(0xffffffffu, v, 0);
+  if (WPR == 1) return v;
+  if ((threadIdx.x & 31) == 0) xb[par * WPR + q] = __float_as_uint(v);
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + rw), "r"(WPR * 32) : "memory");
+  float r = 0.0f;
+#pragma unroll
+  for (int k = 0; k < WPR; ++k) r += __uint_as_float((uint32_t)xb[par * WPR + k]);
+  par ^= 1;
+  return r;
+}
+
+__device__ __forceinline__ float order_key_inverse(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 template <int MODE, int KW, int WPR>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const float* __restrict__ S, int NKTP) {
   extern __shared__ __align__(16) uint32_t sm_u32[];
@@ -341,6 +365,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
   int kind = a.window_kind, rad = a.radius, extra;
   if (MODE == kSelectFixed) {
     extra = a.topk;
+  } else if (MODE == kSelectMass) {
+    extra = 0;                 // set by the mass search below
   } else {
     const int2 pl = a.plan[rowid];
     kind = 1;
@@ -353,14 +379,47 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
   // beyond NKT (no real score maps to 0 or 1).
   uint32_t kr[KW];
   int ncand = 0;
+  float mass_need = 0.0f;     // cumulative-mass mode: pooled mass still to collect (unnormalised)
+  if (MODE == kSelectMass) {
+    // Pooled probabilities e_j / Z with e_j = 2^((s_j - max) * scale * log2 e). The keys are
+    // the fp32 bits of e_j: positive floats, so their order is the order of the scores.
+    float mx = -INFINITY;
 #pragma unroll
-  for (int w = 0; w < KW; ++w) {
-    const int j = 32 * (q * KW + w) + lane;
-    const bool cand = j < NKT && !in_window(ci, coord[j], kind, rad);
-    kr[w] = cand ? order_key(srow[j]) : 0u;
-    ncand += __popc(__ballot_sync(0xffffffffu, cand));
+    for (int w = 0; w < KW; ++w) {
+      const int j = 32 * (q * KW + w) + lane;
+      if (j < NKT) mx = fmaxf(mx, srow[j]);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    mx = order_key_inverse((uint32_t)row_combine<WPR, true>((uint64_t)order_key(mx), xb, par, q, rw));
+    const float c = a.scale * 1.4426950408889634f;
+    float z = 0.0f, zw = 0.0f;
+#pragma unroll
+    for (int w = 0; w < KW; ++w) {
+      const int j = 32 * (q * KW + w) + lane;
+      const bool inrow = j < NKT;
+      const bool inw = inrow && in_window(ci, coord[j], kind, rad);
+      const float e = inrow ? exp2f((srow[j] - mx) * c) : 0.0f;
+      z += e;
+      zw += inw ? e : 0.0f;
+      const bool cand = inrow && !inw;
+      kr[w] = cand ? max(__float_as_uint(e), 1u) : 0u;
+      ncand += __popc(__ballot_sync(0xffffffffu, cand));
+    }
+    z = row_sum_f<WPR>(z, xb, par, q, rw);
+    zw = row_sum_f<WPR>(zw, xb, par, q, rw);
+    mass_need = a.theta * z - zw;
+  } else {
+#pragma unroll
+    for (int w = 0; w < KW; ++w) {
+      const int j = 32 * (q * KW + w) + lane;
+      const bool cand = j < NKT && !in_window(ci, coord[j], kind, rad);
+      kr[w] = cand ? order_key(srow[j]) : 0u;
+      ncand += __popc(__ballot_sync(0xffffffffu, cand));
+    }
   }
   ncand = (int)row_combine<WPR, false>((uint64_t)ncand, xb, par, q, rw);
+  if (MODE == kSelectMass) extra = mass_need > 0.0f ? ncand : 0;   // refined by the mass search
   extra = max(0, min(extra, ncand));
   // extra and ncand are row-uniform by construction; the explicit broadcast from lane 0 is
   // kept because builds without it (nvcc 12.9, -O3) selected every candidate of budget-mode
@@ -372,7 +431,43 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
   // every key > thr is selected. extra == ncand selects every candidate.
   uint32_t thr;
   int need_eq;
-  if (extra == 0) {
+  if (MODE == kSelectMass) {
+    // Smallest set of best candidates whose mass reaches mass_need: the largest key t with
+    // mass(keys >= t) >= mass_need, every key above t, then the keys equal to t (equal
+    // masses) in index order until the need is met. All candidates if it cannot be met.
+    float total = 0.0f;
+#pragma unroll
+    for (int w = 0; w < KW; ++w) total += kr[w] != 0u ? __uint_as_float(kr[w]) : 0.0f;
+    total = row_sum_f<WPR>(total, xb, par, q, rw);
+    if (extra == 0) {
+      thr = 0xffffffffu;
+      need_eq = 0;
+    } else if (total < mass_need) {
+      thr = 0u;
+      need_eq = 0;
+    } else {
+      uint32_t t = 0u;
+      for (int bit = 30; bit >= 0; --bit) {
+        const uint32_t cand_t = t | (1u << bit);
+        float m = 0.0f;
+#pragma unroll
+        for (int w = 0; w < KW; ++w) m += kr[w] >= cand_t ? __uint_as_float(kr[w]) : 0.0f;
+        if (row_sum_f<WPR>(m, xb, par, q, rw) >= mass_need) t = cand_t;
+      }
+      float above = 0.0f;
+      int eqc = 0;
+#pragma unroll
+      for (int w = 0; w < KW; ++w) {
+        above += kr[w] > t ? __uint_as_float(kr[w]) : 0.0f;
+        eqc += kr[w] == t ? 1 : 0;
+      }
+      above = row_sum_f<WPR>(above, xb, par, q, rw);
+      eqc = (int)row_combine<WPR, false>((uint64_t)__reduce_add_sync(0xffffffffu, eqc), xb, par, q, rw);
+      const int need = (int)ceilf((mass_need - above) / __uint_as_float(t));
+      thr = t;
+      need_eq = __shfl_sync(0xffffffffu, max(1, min(need, eqc)), 0);
+    }
+  } else if (extra == 0) {
     thr = 0xffffffffu;
     need_eq = 0;
   } else if (extra == ncand) {
@@ -537,6 +632,7 @@ cudaError_t build_mask_d(const Geom& g, const bsa_mask_params& p, const __nv_bfl
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
+  a.theta = p.budget_target;
   const long long rows = (long long)g.B * g.H * g.NT;
   if (p.budget_mode == 1) {
     entropy_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(g, S, NKTP, a.scale, entropy);
@@ -552,7 +648,8 @@ cudaError_t build_mask_d(const Geom& g, const bsa_mask_params& p, const __nv_bfl
   // coordinate table, then per row of the block a double-buffered exchange of one 64-bit
   // value per warp
   const size_t sel_smem = sizeof(uint32_t) * (size_t)((NKTP + 1) & ~1) + (size_t)kSelWarps * 2 * sizeof(uint64_t);
-  e = (p.budget_mode == 0) ? launch_select<kSelectFixed>(g, sel_smem, a, S, NKTP, s)
+  e = p.budget_mode == 0   ? launch_select<kSelectFixed>(g, sel_smem, a, S, NKTP, s)
+      : p.budget_mode == 2 ? launch_select<kSelectMass>(g, sel_smem, a, S, NKTP, s)
                            : launch_select<kSelectBudget>(g, sel_smem, a, S, NKTP, s);
   if (e != cudaSuccess) return e;
   count_launches(1);

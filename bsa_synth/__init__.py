@@ -55,8 +55,9 @@ class Workload:
     radius: int = 1
     topk: int = 0
     dense_fraction: float = 0.0   # rho: share of query tiles routed to dense attention
-    budget_mode: int = 0          # 0: window + fixed top-k, 1: entropy-derived budget
-    budget_target: float = 0.0    # tau: target retained fraction in budget mode
+    budget_mode: int = 0          # 0: window + fixed top-k, 1: entropy-derived budget,
+                                  # 2: cumulative pooled mass
+    budget_target: float = 0.0    # tau (mode 1: target retained fraction), theta (mode 2: mass)
 
     @property
     def N(self) -> int:

@@ -68,8 +68,14 @@ typedef struct bsa_geom {
  *                 the pooled-score softmax, b_i = clamp(floor(tau*NKT*NQT*exp(H_i) /
  *                 sum_i' exp(H_i') + 1/2), 1, NKT); the window is the decayed window of the
  *                 largest radius that fits b_i, topped up to b_i tiles by pooled score
- *                 (window_kind must be 1)
- *   budget_target tau in (0,1] for budget_mode 1 */
+ *                 (window_kind must be 1);
+ *                 2: cumulative mass: the window (window_kind, radius), then the tiles
+ *                 outside it in decreasing pooled score (ties to the lower index) until
+ *                 the row's pooled probability, softmax over all key tiles of the pooled
+ *                 scores, reaches theta (Token Radius Attention summary: the keys needed
+ *                 to capture a target attention mass); every tile outside the window when
+ *                 theta is not reached; topk is ignored
+ *   budget_target tau in (0,1] for budget_mode 1, theta in (0,1] for budget_mode 2 */
 typedef struct bsa_mask_params {
     int window_kind;
     int radius;

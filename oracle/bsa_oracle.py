@@ -246,20 +246,21 @@ def mass_extra(p_row: np.ndarray, scores_row: np.ndarray, window_row_: np.ndarra
     pooled probability of the whole row reaches theta, i.e. the smallest m with
     mass(window) + mass(first m) >= theta (every tile outside the window when the target is
     not reached). Returns (m, near) where near flags a row whose cumulative mass passes
-    within MASS_NEAR_TIE of the target at the crossing, where float32 sums may decide
-    either way.
+    within the band of the target at the crossing, where float32 sums may decide either
+    way. The band is MASS_NEAR_TIE plus twice the worst-case relative error of a float32
+    sum of NKT positive terms (about NKT * 2^-24 of the total, which is at most 1).
     """
+    band = MASS_NEAR_TIE + p_row.shape[0] * 2.0 ** -23
     R = theta - float(p_row[window_row_].sum())
     cand = np.nonzero(~window_row_)[0]
     if R <= 0.0 or cand.size == 0:
-        return 0, abs(R) < MASS_NEAR_TIE
+        return 0, abs(R) < band
     order = cand[np.lexsort((cand, -scores_row[cand]))]
     cum = np.cumsum(p_row[order])
     m = int(np.searchsorted(cum, R, side="left")) + 1
     if m > cand.size:
-        return int(cand.size), abs(cum[-1] - R) < MASS_NEAR_TIE
-    near = abs(cum[m - 1] - R) < MASS_NEAR_TIE or (m >= 2 and abs(R - cum[m - 2]) < MASS_NEAR_TIE) \
-        or (m == 1 and R < MASS_NEAR_TIE)
+        return int(cand.size), abs(cum[-1] - R) < band
+    near = abs(cum[m - 1] - R) < band or (m >= 2 and abs(R - cum[m - 2]) < band) or (m == 1 and R < band)
     return m, bool(near)
 
 

@@ -24,6 +24,9 @@ SMALL_D128 = {
     "budget128": Workload("budget128", B=1, H=2, d=128, T=12, Hs=16, Ws=20, seed=1012,
                           window_kind=1, radius=0, topk=0, dense_fraction=0.0,
                           budget_mode=1, budget_target=0.19),
+    "mass128": Workload("mass128", B=2, H=2, d=128, T=8, Hs=14, Ws=20, seed=1013,
+                        window_kind=0, radius=1, topk=0, dense_fraction=0.2,
+                        budget_mode=2, budget_target=0.5),
 }
 
 

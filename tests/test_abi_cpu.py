@@ -95,6 +95,8 @@ def test_null_and_misaligned_pointers_rejected_on_host(lib):
     dict(dense_fraction=1.5), dict(dense_fraction=-0.1), dict(window_kind=2), dict(radius=-1),
     dict(topk=-3), dict(budget_mode=2), dict(budget_mode=1, window_kind=0, budget_target=0.1),
     dict(budget_mode=1, window_kind=1, budget_target=0.0),
+    dict(budget_mode=3, budget_target=0.5), dict(budget_mode=2, budget_target=1.5),
+    dict(budget_mode=2, budget_target=0.5, radius=-1), dict(budget_mode=2, budget_target=0.5, window_kind=2),
 ])
 def test_invalid_mask_params_rejected_on_host(lib, bad):
     import block_sparse_attention_major_b200 as bsa

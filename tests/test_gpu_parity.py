@@ -14,7 +14,7 @@ from oracle import bsa_oracle as O
 
 pytestmark = pytest.mark.gpu
 
-SMALL = ["tiny", "tiny_s", "tiny_ragged", "small128", "ragged128", "budget128"]
+SMALL = ["tiny", "tiny_s", "tiny_ragged", "small128", "ragged128", "budget128", "mass128"]
 
 
 def _bsa():
@@ -95,6 +95,16 @@ def test_mask_wan5b_rho_sweep(rho):
 def test_mask_wan14b_heads():
     w, g, gm, ref, cmp, _, _ = _mask_case("wan14b", heads=[0, 39])
     assert cmp["n_unflagged"] == 0, cmp
+
+
+@pytest.mark.parametrize("theta", [0.3, 0.7])
+def test_mask_mass_wan13b_heads(theta):
+    """Cumulative-mass selection on the 1.3B-shaped call (its window, rho = 0.2)."""
+    w, g, gm, ref, cmp, _, _ = _mask_case("wan13b", heads=[0, 11],
+                                          overrides=(("budget_mode", 2), ("budget_target", theta)))
+    assert cmp["n_unflagged"] == 0, cmp
+    assert cmp["n_diff"] <= max(1, cmp["n_rows"] // 200), cmp
+    print(f"theta={theta}: retained={gm.mean():.4f} flagged={cmp['n_flagged']} differing={cmp['n_diff']}")
 
 
 @pytest.mark.parametrize("tau", [0.09, 0.19])
@@ -259,7 +269,7 @@ def test_attention_wan13b_sampled_rows():
 
 
 # ----------------------------------------------------------------------------- whole path
-@pytest.mark.parametrize("name", ["tiny_ragged", "small128", "budget128", "wan13b"])
+@pytest.mark.parametrize("name", ["tiny_ragged", "small128", "budget128", "mass128", "wan13b"])
 def test_forward_path(name):
     """reorder -> build_mask -> sparse attention on the GPU vs the oracle's whole path."""
     bsa = _bsa()
