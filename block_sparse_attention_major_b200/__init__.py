@@ -85,6 +85,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
                                                           vp, vp]
         lib.bsa_launch_count.restype = ctypes.c_uint64
         lib.bsa_launch_count.argtypes = []
+        lib.bsa_selftest_bounded_wait.restype = ctypes.c_int
+        lib.bsa_selftest_bounded_wait.argtypes = [ctypes.c_longlong, vp, vp]
         if path is None:
             _lib = lib
         return lib
@@ -184,6 +186,14 @@ def clear_error(ws: torch.Tensor, stream=None) -> None:
 
 def launch_count() -> int:
     return int(load_library().bsa_launch_count())
+
+
+def selftest_bounded_wait(err: torch.Tensor, limit_cycles: int = 20_000_000, stream=None) -> None:
+    """Run the bounded-wait self-test: a wait that nothing completes gives up after
+    limit_cycles SM cycles and sets BSA_KERR_WAIT_TIMEOUT in err (int32 [1], device)."""
+    _need(err, torch.int32, (1,), "err")
+    _check(load_library().bsa_selftest_bounded_wait(ctypes.c_longlong(limit_cycles), _ptr(err), _stream(stream)),
+           "bsa_selftest_bounded_wait")
 
 
 def reorder(g: Geometry, x: torch.Tensor, xt: torch.Tensor | None = None, stream=None) -> torch.Tensor:

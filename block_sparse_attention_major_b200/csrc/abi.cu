@@ -65,6 +65,10 @@ int status_of(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; 
 
 using namespace bsa;
 
+namespace bsa {
+cudaError_t launch_wait_selftest(long long limit_cycles, uint32_t* err, cudaStream_t s);   // selftest.cu
+}
+
 extern "C" {
 
 const char* bsa_status_string(int status) {
@@ -173,5 +177,13 @@ int bsa_sparse_attn_fwd_fixed_scratch(const bsa_geom* g, const void* qt, const v
 }
 
 uint64_t bsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int bsa_selftest_bounded_wait(long long limit_cycles, uint32_t* err, void* stream) {
+  if (!err || (reinterpret_cast<uintptr_t>(err) & 3u) != 0) return BSA_ERR_INVALID_ARG;
+  if (limit_cycles <= 0 || limit_cycles > 4000000000LL) return BSA_ERR_INVALID_ARG;
+  const int dev = device_ok();
+  if (dev != BSA_OK) return dev;
+  return status_of(bsa::launch_wait_selftest(limit_cycles, err, static_cast<cudaStream_t>(stream)));
+}
 
 }  // extern "C"

@@ -186,6 +186,16 @@ int bsa_sparse_attn_fwd_fixed_scratch(const bsa_geom* g, const void* qt, const v
  * threads). Host-side counter, for accounting only. */
 uint64_t bsa_launch_count(void);
 
+/* Self-test of the kernels' bounded waits (no counterpart in the papers). Launches one
+ * warp that waits, with the same bounded mbarrier wait the attention kernel uses, on a
+ * barrier that nothing ever arrives on, giving up after `limit_cycles` SM cycles (> 0, at
+ * most 4e9). On time-out the wait sets BSA_KERR_WAIT_TIMEOUT in *err (device memory, 4-byte
+ * aligned, OR-ed in) and the kernel returns: the CUDA context stays usable. This is how a
+ * lost arrival (a producer that never delivers) surfaces to the caller, checked without
+ * faulting or hanging a GPU. Asynchronous on `stream`; returns BSA_ERR_INVALID_ARG for a
+ * null or misaligned err or an out-of-range limit. */
+int bsa_selftest_bounded_wait(long long limit_cycles, uint32_t* err, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

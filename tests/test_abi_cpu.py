@@ -119,3 +119,11 @@ def test_binding_fails_loudly_without_library(tmp_path):
 
 def test_launch_counter_starts_at_zero_without_launches(lib):
     assert lib.bsa_launch_count() == 0
+
+
+def test_selftest_arguments_rejected_on_host(lib):
+    al = ctypes.c_void_p(0x1000)
+    assert lib.bsa_selftest_bounded_wait(ctypes.c_longlong(1000), None, None) == 1
+    assert lib.bsa_selftest_bounded_wait(ctypes.c_longlong(1000), ctypes.c_void_p(0x1002), None) == 1
+    assert lib.bsa_selftest_bounded_wait(ctypes.c_longlong(0), al, None) == 1
+    assert lib.bsa_selftest_bounded_wait(ctypes.c_longlong(5_000_000_000), al, None) == 1
