@@ -151,64 +151,73 @@ __device__ int decayed_window_size(const Geom& g, int tt, int ty, int tx, int r)
   return s;
 }
 
-// ---- pooled scores: one 64 x 64 tile of S = qbar kbar^T (unscaled) per block, for one
-// (b, h). Register-blocked SIMT SGEMM: each thread owns a 4 x 4 sub-tile and reads one
-// float4 of each transposed operand per step of the d-loop (2 shared loads per 16 FMAs).
-// Each output is summed over d in increasing order, so the scores are deterministic.
-constexpr int kScoreTile = 64;
+// ---- pooled scores: one 128 x 128 tile of S = qbar kbar^T (unscaled) per block, for one
+// (b, h). Register-blocked SIMT SGEMM: each of the 256 threads owns an 8 x 8 sub-tile, split
+// as rows {4 ty + r, 64 + 4 ty + r} and columns {4 tx + c, 64 + 4 tx + c} so that its four
+// float4 shared loads per d step are broadcast or conflict-free (4 loads per 64 FMAs). The d
+// dimension is staged through shared memory 32 at a time, transposed. Each output is
+// summed over d in increasing order, so the scores are deterministic.
+constexpr int kScoreTile = 128;
+constexpr int kScoreK = 32;
 constexpr int kScorePad = kScoreTile + 4;
 
 template <int D>
-__global__ void __launch_bounds__(256) score_kernel(Geom g, const float* __restrict__ qbar,
+__global__ void __launch_bounds__(256, 2) score_kernel(Geom g, const float* __restrict__ qbar,
                                                     const float* __restrict__ kbar, float* __restrict__ S,
                                                     int NKTP) {
-  extern __shared__ __align__(16) float smem[];
-  float* sA = smem;                          // [D][kScorePad]: sA[c][r] = qbar[i0 + r][c]
-  float* sB = smem + D * kScorePad;          // [D][kScorePad]: sB[c][r] = kbar[j0 + r][c]
+  __shared__ __align__(16) float sA[kScoreK][kScorePad];   // sA[c][r] = qbar[i0 + r][k0 + c]
+  __shared__ __align__(16) float sB[kScoreK][kScorePad];   // sB[c][r] = kbar[j0 + r][k0 + c]
   const int i0 = blockIdx.x * kScoreTile, j0 = blockIdx.y * kScoreTile;
   const long long bh = blockIdx.z;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const float4* q4 = reinterpret_cast<const float4*>(qbar + (bh * g.NT) * D);
   const float4* k4 = reinterpret_cast<const float4*>(kbar + (bh * g.NT) * D);
-  for (int e = tid; e < kScoreTile * (D / 4); e += 256) {
-    const int r = e / (D / 4), c4 = e % (D / 4);
-    float4 va = make_float4(0.f, 0.f, 0.f, 0.f), vb = va;
-    if (i0 + r < g.NT) va = q4[(long long)(i0 + r) * (D / 4) + c4];
-    if (j0 + r < g.NT) vb = k4[(long long)(j0 + r) * (D / 4) + c4];
-    sA[(4 * c4 + 0) * kScorePad + r] = va.x;
-    sA[(4 * c4 + 1) * kScorePad + r] = va.y;
-    sA[(4 * c4 + 2) * kScorePad + r] = va.z;
-    sA[(4 * c4 + 3) * kScorePad + r] = va.w;
-    sB[(4 * c4 + 0) * kScorePad + r] = vb.x;
-    sB[(4 * c4 + 1) * kScorePad + r] = vb.y;
-    sB[(4 * c4 + 2) * kScorePad + r] = vb.z;
-    sB[(4 * c4 + 3) * kScorePad + r] = vb.w;
+  float acc[8][8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
+  for (int k0 = 0; k0 < D; k0 += kScoreK) {
+#pragma unroll
+    for (int t = 0; t < kScoreTile * kScoreK / 4 / 256; ++t) {
+      const int e = tid + 256 * t;
+      const int r = e / (kScoreK / 4), c4 = e % (kScoreK / 4);
+      float4 va = make_float4(0.f, 0.f, 0.f, 0.f), vb = va;
+      if (i0 + r < g.NT) va = q4[(long long)(i0 + r) * (D / 4) + k0 / 4 + c4];
+      if (j0 + r < g.NT) vb = k4[(long long)(j0 + r) * (D / 4) + k0 / 4 + c4];
+      sA[4 * c4 + 0][r] = va.x;
+      sA[4 * c4 + 1][r] = va.y;
+      sA[4 * c4 + 2][r] = va.z;
+      sA[4 * c4 + 3][r] = va.w;
+      sB[4 * c4 + 0][r] = vb.x;
+      sB[4 * c4 + 1][r] = vb.y;
+      sB[4 * c4 + 2][r] = vb.z;
+      sB[4 * c4 + 3][r] = vb.w;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int c = 0; c < kScoreK; ++c) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&sA[c][4 * ty]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&sA[c][64 + 4 * ty]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&sB[c][4 * tx]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&sB[c][64 + 4 * tx]);
+      const float qv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float kv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) acc[r][cc] = fmaf(qv[r], kv[cc], acc[r][cc]);
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  const int tx = tid & 15, ty = tid >> 4;
-  float acc[4][4];
 #pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
-#pragma unroll 8
-  for (int c = 0; c < D; ++c) {
-    const float4 qa = *reinterpret_cast<const float4*>(sA + c * kScorePad + 4 * ty);
-    const float4 kb = *reinterpret_cast<const float4*>(sB + c * kScorePad + 4 * tx);
-    const float qv[4] = {qa.x, qa.y, qa.z, qa.w};
-    const float kv[4] = {kb.x, kb.y, kb.z, kb.w};
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) acc[r][cc] = fmaf(qv[r], kv[cc], acc[r][cc]);
-  }
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int i = i0 + 4 * ty + r;
-    const int j = j0 + 4 * tx;
-    if (i < g.NT && j < NKTP)
-      *reinterpret_cast<float4*>(S + (bh * g.NT + i) * (long long)NKTP + j) =
-          make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+  for (int r = 0; r < 8; ++r) {
+    const int i = i0 + (r < 4 ? 4 * ty + r : 64 + 4 * ty + (r - 4));
+    if (i >= g.NT) continue;
+    float* row = S + (bh * g.NT + i) * (long long)NKTP;
+    const int j_lo = j0 + 4 * tx, j_hi = j0 + 64 + 4 * tx;
+    if (j_lo < NKTP) *reinterpret_cast<float4*>(row + j_lo) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+    if (j_hi < NKTP) *reinterpret_cast<float4*>(row + j_hi) = make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
   }
 }
 
@@ -623,10 +632,7 @@ cudaError_t build_mask_d(const Geom& g, const bsa_mask_params& p, const __nv_bfl
 
   float* S = reinterpret_cast<float*>(ws + L.scores);
   const int NKTP = (g.NT + 3) & ~3;
-  const size_t score_smem = 2 * D * kScorePad * sizeof(float);
-  e = cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)score_smem);
-  if (e != cudaSuccess) return e;
-  score_kernel<D><<<dim3(ceil_div(g.NT, kScoreTile), ceil_div(g.NT, kScoreTile), g.B * g.H), 256, score_smem, s>>>(
+  score_kernel<D><<<dim3(ceil_div(g.NT, kScoreTile), ceil_div(g.NT, kScoreTile), g.B * g.H), 256, 0, s>>>(
       g, qbar, kbar, S, NKTP);
   count_launches(1);
   e = cudaGetLastError();
