@@ -27,6 +27,11 @@ SMALL_D128 = {
     "mass128": Workload("mass128", B=2, H=2, d=128, T=8, Hs=14, Ws=20, seed=1013,
                         window_kind=0, radius=1, topk=0, dense_fraction=0.2,
                         budget_mode=2, budget_target=0.5),
+    # edge cases: a grid of one (partial) tile, and the largest supported tile count
+    "one_tile": Workload("one_tile", B=1, H=2, d=64, T=3, Hs=3, Ws=3, seed=1014,
+                         window_kind=0, radius=1, topk=2, dense_fraction=0.0),
+    "max_tiles": Workload("max_tiles", B=1, H=1, d=64, T=64, Hs=64, Ws=64, seed=1015,
+                          window_kind=0, radius=1, topk=4, dense_fraction=0.05),
 }
 
 

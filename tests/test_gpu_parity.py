@@ -293,6 +293,47 @@ def test_forward_path(name):
     C.assert_attention_close(st)
 
 
+def test_forward_path_one_tile():
+    """A grid of a single partial tile (27 tokens): one mask word, one query tile per unit,
+    no second sub-unit; the whole path against the oracle on every row."""
+    bsa = _bsa()
+    w, q, k, v, diff = C.inputs("one_tile")
+    g = C.geometry(w)
+    assert g.NT == 1
+    b = bsa.forward(g, C.params(w), q.cuda(), k.cuda(), v.cuda(), diff.cuda())
+    torch.cuda.synchronize()
+    assert bsa.read_error(b.ws) == 0
+    qt64, kt64, vt64 = (O.reorder(O.to_f64(x), w.T, w.Hs, w.Ws) for x in (q, k, v))
+    mref = C.oracle_mask(w, qt64, kt64, diff.numpy())
+    assert np.array_equal(C.gpu_mask_bool(b.mask, g.NT), mref["mask"])
+    rows = [(0, h, 0) for h in range(w.H)]
+    ref = O.attention_tiles(qt64, kt64, vt64, mref["mask"], rows, T=w.T, Hs=w.Hs, Ws=w.Ws)
+    C.assert_attention_close(C.compare_attention(w, b.out, b.lse, ref))
+
+
+def test_forward_path_max_tiles():
+    """The largest supported grid (4096 tiles: 128 mask words per row, rows spanning four
+    selection warps, union lists at their limit): masks on every row, attention on
+    sampled rows."""
+    bsa = _bsa()
+    w, q, k, v, diff = C.inputs("max_tiles")
+    g = C.geometry(w)
+    assert g.NT == 4096
+    b = bsa.forward(g, C.params(w), q.cuda(), k.cuda(), v.cuda(), diff.cuda())
+    torch.cuda.synchronize()
+    assert bsa.read_error(b.ws) == 0
+    qt64, kt64, vt64 = (O.reorder(O.to_f64(x), w.T, w.Hs, w.Ws) for x in (q, k, v))
+    mref = C.oracle_mask(w, qt64, kt64, diff.numpy())
+    cmp = C.compare_masks(C.gpu_mask_bool(b.mask, g.NT), mref)
+    assert cmp["n_unflagged"] == 0, cmp
+    rng = np.random.default_rng(17)
+    dense_rows = np.nonzero(mref["dense"][0])[0]
+    rows = [(0, 0, int(i)) for i in rng.integers(g.NT, size=12)] + [(0, 0, int(dense_rows[0]))]
+    ref = O.attention_tiles(qt64, kt64, vt64, mref["mask"], rows, T=w.T, Hs=w.Hs, Ws=w.Ws)
+    st = C.compare_attention(w, b.out, b.lse, ref, skip_rows=cmp["diff_rows"])
+    C.assert_attention_close(st)
+
+
 @pytest.mark.parametrize("name,overrides", [("wan14b", ()), ("hunyuan", (("budget_target", 0.14),))])
 def test_forward_path_full_size(name, overrides):
     """Whole path on the 14B- and Hunyuan-shaped calls; the oracle checks two heads."""
