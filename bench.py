@@ -383,41 +383,72 @@ def run_ours(args):
         raise SystemExit("kernel error word set")
 
     # ---------------------------------------------------------------- end to end (host buffers)
+    # Every step copies its inputs from pinned host memory and reads its output and LSE back.
+    # Two sets of device inputs and outputs let the copy in of step s+1 (one stream) and the
+    # copy back of step s-1 (another stream) run on the copy engines while step s's kernels
+    # run; events order every reuse of a buffer.
     e2e = None
     if not args.no_e2e:
         q_p, k_p, v_p, d_p = (x.pin_memory() for x in (q_h, k_h, v_h, diff_h))
-        out_p = torch.empty(bufs.out.shape, dtype=bufs.out.dtype).pin_memory()
-        lse_p = torch.empty(bufs.lse.shape, dtype=bufs.lse.dtype).pin_memory()
-        qd, kd, vd, dd = (torch.empty_like(x, device=dev) for x in (q_h, k_h, v_h, diff_h))
+        ins = [tuple(torch.empty_like(x, device=dev) for x in (q_h, k_h, v_h, diff_h)) for _ in range(2)]
+        outb = [bufs, bsa.Buffers(g, dev)]
+        outs = [(torch.empty(bufs.out.shape, dtype=bufs.out.dtype).pin_memory(),
+                 torch.empty(bufs.lse.shape, dtype=bufs.lse.dtype).pin_memory()) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         e2e_steps = max(3, min(args.steps, 60))
 
-        def e2e_step():
-            qd.copy_(q_p, non_blocking=True)
-            kd.copy_(k_p, non_blocking=True)
-            vd.copy_(v_p, non_blocking=True)
-            dd.copy_(d_p, non_blocking=True)
-            bsa.forward(g, p, qd, kd, vd, dd, bufs)
-            out_p.copy_(bufs.out, non_blocking=True)
-            lse_p.copy_(bufs.lse, non_blocking=True)
+        def e2e_run(n, start):
+            s_in.wait_event(start)
+            s_out.wait_event(start)
+            computed, returned = [None, None], [None, None]
+            for step in range(n):
+                j = step % 2
+                qd, kd, vd, dd = ins[j]
+                with torch.cuda.stream(s_in):
+                    if computed[j] is not None:          # step - 2 has read these inputs
+                        s_in.wait_event(computed[j])
+                    for dst, src in zip((qd, kd, vd, dd), (q_p, k_p, v_p, d_p)):
+                        dst.copy_(src, non_blocking=True)
+                    arrived = ev()
+                    arrived.record(s_in)
+                stream.wait_event(arrived)
+                if returned[j] is not None:              # step - 2's output has been read back
+                    stream.wait_event(returned[j])
+                bsa.forward(g, p, qd, kd, vd, dd, outb[j])
+                computed[j] = ev()
+                computed[j].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(computed[j])
+                    outs[j][0].copy_(outb[j].out, non_blocking=True)
+                    outs[j][1].copy_(outb[j].lse, non_blocking=True)
+                    returned[j] = ev()
+                    returned[j].record(s_out)
+            for r in returned:
+                if r is not None:
+                    stream.wait_event(r)
 
-        for _ in range(args.warmup):
-            e2e_step()
+        w0 = ev()
+        w0.record(stream)
+        e2e_run(args.warmup, w0)
         torch.cuda.synchronize(dev)
         barrier()
         torch.cuda.synchronize(dev)
         a, b = ev(), ev()
         a.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
+        e2e_run(e2e_steps, a)
         b.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
         e2e_ms = max_over_ranks(a.elapsed_time(b))
         h2d = sum(x.numel() * x.element_size() for x in (q_h, k_h, v_h, diff_h))
-        d2h = out_p.numel() * out_p.element_size() + lse_p.numel() * lse_p.element_size()
+        d2h = outs[0][0].numel() * outs[0][0].element_size() + outs[0][1].numel() * outs[0][1].element_size()
         e2e = {"value": sum_over_ranks(flops_call) * e2e_steps / (e2e_ms * 1e-3) / 1e12,
                "unit": "TFLOP/s", "ms_per_step": e2e_ms / e2e_steps,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+               "overlap": "copy in of step s+1 and copy back of step s-1 overlap step s's kernels"}
+        if bsa.read_error(outb[1].ws) != 0:
+            raise SystemExit("kernel error word set")
+        del ins, outb
 
     # ---------------------------------------------------------------- own dense path (rho = 1)
     pd = bsa.MaskParams(w.window_kind, w.radius, w.topk, 1.0, 0, 0.0)
