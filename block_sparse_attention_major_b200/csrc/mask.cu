@@ -17,11 +17,12 @@
 //            it takes for the row's pooled probability to reach a target mass (the same
 //            summary: keys needed to capture a target attention mass).
 //
-// Selection works per row and per warp on order-preserving integer keys of
-// the fp32 scores: a few extra tiles by repeated warp argmax (largest key, then lowest
-// tile index), many by a bitwise binary search for the threshold key followed by an
-// index-ordered pass over tied keys. Both reproduce "highest score, ties to the lower
-// index" exactly and use no atomics.
+// Selection works per row (one to four warps) on order-preserving integer keys: the fp32
+// bits of the scores mapped to unsigned order, or, in cumulative-mass mode, the bits of the
+// row's positive pooled probabilities. A few extra tiles are found by repeated argmax
+// (largest key, then lowest tile index), many by a bitwise binary search for the threshold
+// key (on counts, or on mass) followed by an index-ordered pass over tied keys. Both
+// reproduce "highest score, ties to the lower index" exactly and use no atomics.
 #include "common.cuh"
 
 #include <math.h>
@@ -304,7 +305,7 @@ __device__ __forceinline__ uint64_t row_combine(uint64_t v, volatile uint64_t* x
   if (WPR == 1) return v;
   if ((threadIdx.x & 31) == 0) xb[par * WPR + q] = v;
   asm volatile("bar.sync %0, %1;" ::"r"(1 + rw), "r"(WPR * 32) : "memory");
-  uint64_t r = kMax ? 0ull : 0ull;
+  uint64_t r = 0ull;
 #pragma unroll
   for (int k = 0; k < WPR; ++k) {
     const uint64_t x = xb[par * WPR + k];
