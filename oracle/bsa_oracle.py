@@ -167,6 +167,9 @@ def window(kind: int, r: int, T: int, Hs: int, Ws: int) -> np.ndarray:
     kind 1 (temporal distance decay, Token Radius Attention "Radius construction"):
         |dt| <= r and max(|dy|, |dx|) <= r - |dt|: the spatial radius shrinks by one per
         frame-tile of distance.
+    kind 2 (token-level circular support of radius r in tokens, see in_token_support):
+        the key tiles that hold a token of some query token's support; attention inside
+        these tiles is then masked token by token (attention_tiles, token_rho).
     """
     c = tile_coords(T, Hs, Ws)
     dt = np.abs(c[:, None, 0] - c[None, :, 0])
@@ -176,7 +179,9 @@ def window(kind: int, r: int, T: int, Hs: int, Ws: int) -> np.ndarray:
         return np.maximum(np.maximum(dt, dy), dx) <= r
     if kind == 1:
         return (dt <= r) & (np.maximum(dy, dx) <= r - dt)
-    raise ValueError("window kind must be 0 or 1")
+    if kind == 2:
+        return token_window(r, T, Hs, Ws)
+    raise ValueError("window kind must be 0, 1 or 2")
 
 
 def window_row(kind: int, r: int, i: int, T: int, Hs: int, Ws: int) -> np.ndarray:
@@ -188,6 +193,46 @@ def window_row(kind: int, r: int, i: int, T: int, Hs: int, Ws: int) -> np.ndarra
     if kind == 0:
         return np.maximum(np.maximum(dt, dy), dx) <= r
     return (dt <= r) & (np.maximum(dy, dx) <= r - dt)
+
+
+def slot_coords(T: int, Hs: int, Ws: int) -> np.ndarray:
+    """Token coordinates (t, y, x) of every slot of every tile, int [NT, 64, 3] (padding
+    slots get the coordinates they would have; use slot_valid to drop them)."""
+    c = tile_coords(T, Hs, Ws)
+    r = np.arange(TILE_TOKENS)
+    off = np.stack([r // 16, (r // 4) % 4, r % 4], axis=1)               # (dt, dy, dx)
+    return c[:, None, :] * TILE_EDGE + off[None, :, :]
+
+
+def in_token_support(n: np.ndarray, m: np.ndarray, rho: int) -> np.ndarray:
+    """Whether key token m lies in the circular support of query token n (broadcasting over
+    leading axes of the [..., 3] coordinate arrays).
+
+    Reading of Token Radius Attention ("Radius construction": query-centred circular
+    neighbourhoods whose base radius is applied across frames with temporal distance decay)
+    at token level: frame distance |dt| <= rho and in-plane Euclidean distance at most
+    rho - |dt|, i.e. dy^2 + dx^2 <= (rho - |dt|)^2.
+    """
+    dt = np.abs(m[..., 0] - n[..., 0])
+    d2 = (m[..., 1] - n[..., 1]) ** 2 + (m[..., 2] - n[..., 2]) ** 2
+    return (dt <= rho) & (d2 <= (rho - dt) ** 2)
+
+
+def token_window(rho: int, T: int, Hs: int, Ws: int) -> np.ndarray:
+    """Tile window of the token-level circular support, bool [NQT, NKT]: key tile j is in
+    query tile i's window when some valid token of j lies in the support of some valid
+    token of i (brute force over token pairs)."""
+    xy = slot_coords(T, Hs, Ws)
+    valid = slot_valid(T, Hs, Ws)
+    NT = xy.shape[0]
+    keys = xy[valid]                                                      # [Nvalid, 3]
+    key_tile = np.repeat(np.arange(NT), valid.sum(axis=1))
+    W = np.zeros((NT, NT), dtype=bool)
+    for i in range(NT):
+        q = xy[i][valid[i]]                                               # [nq, 3]
+        hit = in_token_support(q[:, None, :], keys[None, :, :], rho).any(axis=0)
+        W[i, np.unique(key_tile[hit])] = True
+    return W
 
 
 def top_outside(scores_row: np.ndarray, excluded: np.ndarray, m: int) -> np.ndarray:
@@ -323,8 +368,10 @@ def build_mask(qt: np.ndarray, kt: np.ndarray, difficulty: np.ndarray, *, T: int
     near = np.zeros((B, H, NQT), dtype=bool)
     budget = np.zeros((B, H, NQT), dtype=np.int64)
     budget_x = np.zeros((B, H, NQT), dtype=np.float64)
+    window_mask = np.zeros((NQT, NKT), dtype=bool)
     if budget_mode == 0:
         W = window(window_kind, radius, T, Hs, Ws)
+        window_mask = W
         for b in range(B):
             for h in range(H):
                 for i in range(NQT):
@@ -337,6 +384,8 @@ def build_mask(qt: np.ndarray, kt: np.ndarray, difficulty: np.ndarray, *, T: int
                     mask[b, h, i] = row
                     near[b, h, i] = boundary_near_tie(S[b, h, i], W[i], m)
     elif budget_mode == 1:
+        if window_kind != 1:
+            raise ValueError("the entropy budget uses the decayed window (window_kind 1)")
         Hent = row_entropy(S)
         for b in range(B):
             for h in range(H):
@@ -358,6 +407,7 @@ def build_mask(qt: np.ndarray, kt: np.ndarray, difficulty: np.ndarray, *, T: int
                     near[b, h, i] = near_half or boundary_near_tie(S[b, h, i], Wi, m)
     elif budget_mode == 2:
         W = window(window_kind, radius, T, Hs, Ws)
+        window_mask = W
         theta = float(np.float32(budget_target))
         P = pooled_probabilities(S)
         for b in range(B):
@@ -375,7 +425,7 @@ def build_mask(qt: np.ndarray, kt: np.ndarray, difficulty: np.ndarray, *, T: int
         raise ValueError("budget_mode must be 0, 1 or 2")
     return dict(mask=mask, count=mask.sum(axis=-1).astype(np.int64), near_tie=near,
                 qbar=qbar, kbar=kbar, scores=S, dense=dense, budget=budget,
-                budget_x=budget_x)
+                budget_x=budget_x, window=window_mask)
 
 
 def pack_bitmask(mask: np.ndarray) -> np.ndarray:
@@ -402,16 +452,24 @@ def unpack_bitmask(bits: np.ndarray, NKT: int) -> np.ndarray:
 # ----------------------------------------------------------------------------------------
 def attention_tiles(qt: np.ndarray, kt: np.ndarray, vt: np.ndarray, mask: np.ndarray,
                     rows: list[tuple[int, int, int]], *, T: int, Hs: int, Ws: int,
-                    scale: float | None = None, return_weights: bool = False) -> dict:
+                    scale: float | None = None, return_weights: bool = False,
+                    token_rho: int | None = None, window: np.ndarray | None = None,
+                    dense: np.ndarray | None = None) -> dict:
     """Masked softmax attention for the listed (b, h, query tile) rows, in float64.
 
     For each valid query token of tile i: s = q . k * scale over the valid tokens of the
     retained key tiles; weights = softmax(s) (max subtracted); o = weights @ v;
     lse = log(sum exp(s)). Output per row: o [64, d] (padding slots zero), lse [64].
+
+    With token_rho (window kind 2), a query token of a local (non-dense) row sees, in the
+    key tiles of its tile's window (window [NQT, NKT]), only the tokens of its circular
+    support (in_token_support); tiles retained outside the window (the extras) are seen
+    whole. dense [B, NQT] marks rows that see every valid token.
     """
     d = qt.shape[-1]
     sc = (1.0 / math.sqrt(d)) if scale is None else scale
     valid = slot_valid(T, Hs, Ws)
+    coords = slot_coords(T, Hs, Ws) if token_rho is not None else None
     res = {}
     for (b, h, i) in rows:
         kept = np.nonzero(mask[b, h, i])[0]
@@ -427,6 +485,14 @@ def attention_tiles(qt: np.ndarray, kt: np.ndarray, vt: np.ndarray, mask: np.nda
         V = np.concatenate(vals, axis=0)
         q = np.asarray(qt[b, h, i], dtype=np.float64)
         s = (q @ K.T) * sc                                               # [64, nk]
+        if token_rho is not None and not (dense is not None and dense[b, i]):
+            ids = np.concatenate(key_ids, axis=0)                        # [nk, 2] (tile, slot)
+            in_win = window[i, ids[:, 0]]
+            kc = coords[ids[:, 0], ids[:, 1]]                            # [nk, 3]
+            sup = in_token_support(coords[i][:, None, :], kc[None, :, :], token_rho)
+            allowed = sup | ~in_win[None, :]
+            allowed[~valid[i]] = True                                    # padding rows: any finite value
+            s = np.where(allowed, s, -np.inf)
         mx = s.max(axis=1, keepdims=True)
         e = np.exp(s - mx)
         z = e.sum(axis=1, keepdims=True)

@@ -527,6 +527,98 @@ def test_mass_monotone_and_brute_force():
             assert set(np.nonzero(res["mask"][0, 0, i])[0]) == keep
 
 
+# ------------------------------------------------------------------------------ token-level circular support
+def _golden_token_support():
+    rows = []
+    with open(os.path.join(os.path.dirname(__file__), "golden", "token_support_sizes.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                rows.append(tuple(int(x) for x in line.split()))
+    return rows
+
+
+@pytest.mark.parametrize("rho,disc,size", _golden_token_support())
+def test_token_support_interior_size(rho, disc, size):
+    """Counted by brute force around an interior token: the lattice-point counts."""
+    n = np.array([20, 20, 20])
+    r = np.arange(-8, 9)
+    box = np.stack(np.meshgrid(r, r, r, indexing="ij"), axis=-1).reshape(-1, 3) + n
+    inside = O.in_token_support(n[None, :], box, rho)
+    assert inside.sum() == size
+    same_frame = inside & (box[:, 0] == n[0])
+    assert same_frame.sum() == disc
+
+
+def test_token_support_symmetric():
+    rng = np.random.default_rng(3)
+    a = rng.integers(0, 12, size=(500, 3))
+    b = rng.integers(0, 12, size=(500, 3))
+    for rho in (0, 1, 2, 4):
+        assert np.array_equal(O.in_token_support(a, b, rho), O.in_token_support(b, a, rho))
+
+
+def _valid_box(T, Hs, Ws):
+    """Per tile, the [lo, hi] token range along t, y, x of its valid slots."""
+    c = O.tile_coords(T, Hs, Ws) * 4
+    hi = np.minimum(c + 3, np.array([T - 1, Hs - 1, Ws - 1]))
+    return c, hi
+
+
+@pytest.mark.parametrize("grid", [(8, 16, 16), (6, 10, 9), (13, 7, 11)])
+@pytest.mark.parametrize("rho", [0, 1, 2, 3, 5])
+def test_token_window_matches_interval_closed_form(grid, rho):
+    """The valid tokens of a tile form a box, and a larger frame distance only shrinks the
+    in-plane radius, so tile j is in tile i's window iff the smallest frame gap g_t and the
+    smallest row/column gaps g_y, g_x between their boxes satisfy g_t <= rho and
+    g_y^2 + g_x^2 <= (rho - g_t)^2."""
+    T, Hs, Ws = grid
+    lo, hi = _valid_box(T, Hs, Ws)
+    gap = np.maximum(0, np.maximum(lo[None, :, :] - hi[:, None, :], lo[:, None, :] - hi[None, :, :]))
+    gt, gy, gx = gap[..., 0], gap[..., 1], gap[..., 2]
+    expect = (gt <= rho) & (gy ** 2 + gx ** 2 <= (rho - gt) ** 2)
+    assert np.array_equal(O.token_window(rho, T, Hs, Ws), expect)
+
+
+def test_token_window_attention_matches_brute_force():
+    """Window kind 2 with top-k extras: the attention equals a softmax over the explicit
+    token mask (support inside window tiles, whole extra tiles, every key for dense rows)."""
+    T, Hs, Ws, d, H = 6, 10, 9, 8, 2
+    rng = np.random.default_rng(31)
+    NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
+    qt = rng.standard_normal((1, H, NT, 64, d)); kt = rng.standard_normal((1, H, NT, 64, d))
+    vt = rng.standard_normal((1, H, NT, 64, d))
+    valid = O.slot_valid(T, Hs, Ws)
+    for t in (qt, kt, vt):
+        t[:, :, ~valid] = 0.0
+    diff = rng.random((1, NT)).astype(np.float32)
+    rho = 2
+    m = O.build_mask(qt, kt, diff, T=T, Hs=Hs, Ws=Ws, window_kind=2, radius=rho, topk=2,
+                     dense_fraction=0.25)
+    rows = [(0, h, i) for h in range(H) for i in range(NT)]
+    res = O.attention_tiles(qt, kt, vt, m["mask"], rows, T=T, Hs=Hs, Ws=Ws, token_rho=rho,
+                            window=m["window"], dense=m["dense"])
+    xy = O.slot_coords(T, Hs, Ws)
+    keys = [(j, s_) for j in range(NT) for s_ in range(64) if valid[j, s_]]
+    for (b, h, i) in rows:
+        for r in range(64):
+            if not valid[i, r]:
+                continue
+            logits, vals = [], []
+            for (j, s_) in keys:
+                if not m["mask"][b, h, i, j]:
+                    continue
+                local = m["window"][i, j] and not m["dense"][b, i]
+                if local and not O.in_token_support(xy[i, r], xy[j, s_], rho):
+                    continue
+                logits.append(float(qt[b, h, i, r] @ kt[b, h, j, s_]) / math.sqrt(d))
+                vals.append(vt[b, h, j, s_])
+            lg = np.array(logits)
+            w = np.exp(lg - lg.max())
+            o = (w[:, None] * np.array(vals)).sum(0) / w.sum()
+            np.testing.assert_allclose(res[(b, h, i)]["o"][r], o, rtol=1e-10, atol=1e-12)
+            assert abs(res[(b, h, i)]["lse"][r] - (lg.max() + math.log(w.sum()))) < 1e-10
+
+
 # ------------------------------------------------------------------------------ planted mistakes
 def test_pins_catch_planted_pool_divisor(monkeypatch):
     """Dividing by 64 instead of the valid count must break the raster-mean pin."""
@@ -564,3 +656,14 @@ def test_pins_catch_planted_window_mass(monkeypatch):
     monkeypatch.setattr(O, "mass_extra", lambda p, s, w, t: real(p * np.where(w, 0.0, 1.0), s, w, t))
     with pytest.raises(AssertionError):
         test_mass_uniform_scores_closed_form()
+
+
+def test_pins_catch_planted_square_support(monkeypatch):
+    """A square (Chebyshev) support instead of the circular one must break the size pin."""
+    def square(n, m, rho):
+        dt = np.abs(m[..., 0] - n[..., 0])
+        cheb = np.maximum(np.abs(m[..., 1] - n[..., 1]), np.abs(m[..., 2] - n[..., 2]))
+        return (dt <= rho) & (cheb <= rho - dt)
+    monkeypatch.setattr(O, "in_token_support", square)
+    with pytest.raises(AssertionError):
+        test_token_support_interior_size(2, 13, 25)
