@@ -549,6 +549,17 @@ def test_token_support_interior_size(rho, disc, size):
     assert same_frame.sum() == disc
 
 
+@pytest.mark.parametrize("grid", [(8, 16, 16), (6, 10, 9), (13, 7, 11)])
+def test_slot_coords_match_raster_tokens(grid):
+    """Each valid slot's (t, y, x) gives back its raster token index (t Hs + y) Ws + x."""
+    T, Hs, Ws = grid
+    xy = O.slot_coords(T, Hs, Ws)
+    tok = O.slot_tokens(T, Hs, Ws)
+    valid = O.slot_valid(T, Hs, Ws)
+    n = (xy[..., 0] * Hs + xy[..., 1]) * Ws + xy[..., 2]
+    assert np.array_equal(n[valid], tok[valid])
+
+
 def test_token_support_symmetric():
     rng = np.random.default_rng(3)
     a = rng.integers(0, 12, size=(500, 3))
