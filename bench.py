@@ -530,6 +530,8 @@ def _report_workloads():
     out += [(f"wan5b_rho{r}", WORKLOADS["wan5b"].with_(dense_fraction=r)) for r in WAN5B_RHO_SWEEP]
     out.append(("wan14b", WORKLOADS["wan14b"]))
     out += [(f"hunyuan_tau{t}", WORKLOADS["hunyuan"].with_(budget_target=t)) for t in HUNYUAN_TAU_SWEEP]
+    # cumulative-mass selection on the 1.3B-shaped call (its window and dense share)
+    out += [(f"wan13b_mass{t}", WORKLOADS["wan13b"].with_(budget_mode=2, budget_target=t)) for t in (0.5, 0.8)]
     return out
 
 
