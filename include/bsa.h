@@ -135,8 +135,9 @@ int bsa_unreorder(const bsa_geom* g, const void* xt, void* x, void* stream);
  *   kv_count   : int32 [B, H, NQT] output; retained key tiles per row
  *   ws, ws_bytes : device workspace of at least bsa_workspace_bytes(g, p) bytes
  * Steps: mean of each tile's valid tokens (fp32); pooled scores qbar.kbar (fp32, ranked
- * unscaled; the 1/sqrt(d) scale enters the entropy only); routing; window; extra tiles
- * by pooled score. Deterministic: repeated calls give identical bits. */
+ * unscaled; the 1/sqrt(d) scale enters the entropy and the pooled probabilities of the
+ * cumulative-mass mode only); routing; window; extra tiles by pooled score.
+ * Deterministic: repeated calls give identical bits. */
 int bsa_build_mask(const bsa_geom* g, const bsa_mask_params* p, const void* qt,
                    const void* kt, const float* difficulty, uint32_t* mask,
                    int32_t* kv_count, void* ws, size_t ws_bytes, void* stream);
