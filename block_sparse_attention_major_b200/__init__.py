@@ -136,9 +136,28 @@ class MaskParams:
                                self.budget_mode, self.budget_target)
 
 
-def _stream(stream) -> ctypes.c_void_p:
-    s = torch.cuda.current_stream() if stream is None else stream
+def _stream(stream, device: torch.device) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    if s.device != device:
+        raise ValueError(f"stream is on {s.device}, the tensors on {device}")
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def _device_of(*tensors: torch.Tensor | None) -> torch.device:
+    """The one device of the given tensors (None entries skipped). The library launches on
+    the current device with the pointers it is given, so tensors of two devices, or of a
+    device other than the one the call runs on, are refused here."""
+    devs = [t.device for t in tensors if t is not None]
+    if not devs or any(d != devs[0] for d in devs):
+        raise ValueError(f"tensors of one call must share one device, got {sorted(set(map(str, devs)))}")
+    return devs[0]
+
+
+def _run(what: str, device: torch.device, stream, call) -> None:
+    """call(stream_handle) with `device` current, so that the library's launches, its
+    device queries and the stream all refer to the device that holds the tensors."""
+    with torch.cuda.device(device):
+        _check(call(_stream(stream, device)), what)
 
 
 def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
@@ -154,6 +173,12 @@ def _need(t: torch.Tensor, dtype, shape, name: str) -> None:
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+def _need_ws(ws: torch.Tensor) -> None:
+    if (not isinstance(ws, torch.Tensor) or not ws.is_cuda or ws.dtype != torch.uint8 or ws.dim() != 1
+            or not ws.is_contiguous()):
+        raise ValueError("ws must be a contiguous 1-D uint8 CUDA tensor (see alloc_workspace)")
 
 
 def _check(status: int, what: str) -> None:
@@ -181,7 +206,8 @@ def read_error(ws: torch.Tensor) -> int:
 
 
 def clear_error(ws: torch.Tensor, stream=None) -> None:
-    _check(load_library().bsa_clear_error(_ptr(ws), _stream(stream)), "bsa_clear_error")
+    _need_ws(ws)
+    _run("bsa_clear_error", ws.device, stream, lambda s: load_library().bsa_clear_error(_ptr(ws), s))
 
 
 def launch_count() -> int:
@@ -192,8 +218,8 @@ def selftest_bounded_wait(err: torch.Tensor, limit_cycles: int = 20_000_000, str
     """Run the bounded-wait self-test: a wait that nothing completes gives up after
     limit_cycles SM cycles and sets BSA_KERR_WAIT_TIMEOUT in err (int32 [1], device)."""
     _need(err, torch.int32, (1,), "err")
-    _check(load_library().bsa_selftest_bounded_wait(ctypes.c_longlong(limit_cycles), _ptr(err), _stream(stream)),
-           "bsa_selftest_bounded_wait")
+    _run("bsa_selftest_bounded_wait", err.device, stream,
+         lambda s: load_library().bsa_selftest_bounded_wait(ctypes.c_longlong(limit_cycles), _ptr(err), s))
 
 
 def reorder(g: Geometry, x: torch.Tensor, xt: torch.Tensor | None = None, stream=None) -> torch.Tensor:
@@ -201,8 +227,8 @@ def reorder(g: Geometry, x: torch.Tensor, xt: torch.Tensor | None = None, stream
     if xt is None:
         xt = torch.empty((g.B, g.H, g.NT, 64, g.d), dtype=torch.bfloat16, device=x.device)
     _need(xt, torch.bfloat16, (g.B, g.H, g.NT, 64, g.d), "xt")
-    _check(load_library().bsa_reorder(ctypes.byref(g.c()), _ptr(x), _ptr(xt), _stream(stream)),
-           "bsa_reorder")
+    _run("bsa_reorder", _device_of(x, xt), stream,
+         lambda s: load_library().bsa_reorder(ctypes.byref(g.c()), _ptr(x), _ptr(xt), s))
     return xt
 
 
@@ -211,8 +237,8 @@ def unreorder(g: Geometry, xt: torch.Tensor, x: torch.Tensor | None = None, stre
     if x is None:
         x = torch.empty((g.B, g.N, g.H, g.d), dtype=torch.bfloat16, device=xt.device)
     _need(x, torch.bfloat16, (g.B, g.N, g.H, g.d), "x")
-    _check(load_library().bsa_unreorder(ctypes.byref(g.c()), _ptr(xt), _ptr(x), _stream(stream)),
-           "bsa_unreorder")
+    _run("bsa_unreorder", _device_of(xt, x), stream,
+         lambda s: load_library().bsa_unreorder(ctypes.byref(g.c()), _ptr(xt), _ptr(x), s))
     return x
 
 
@@ -232,11 +258,12 @@ def build_mask(g: Geometry, p: MaskParams, qt: torch.Tensor, kt: torch.Tensor,
     _need(kv_count, torch.int32, (g.B, g.H, g.NT), "kv_count")
     if ws is None:
         ws = alloc_workspace(g, dev)
+    _need_ws(ws)
     pc = p.c()
-    _check(load_library().bsa_build_mask(ctypes.byref(g.c()), ctypes.byref(pc), _ptr(qt), _ptr(kt),
-                                         _ptr(difficulty), _ptr(mask), _ptr(kv_count), _ptr(ws),
-                                         ctypes.c_size_t(ws.numel()), _stream(stream)),
-           "bsa_build_mask")
+    _run("bsa_build_mask", _device_of(qt, kt, difficulty, mask, kv_count, ws), stream,
+         lambda s: load_library().bsa_build_mask(ctypes.byref(g.c()), ctypes.byref(pc), _ptr(qt), _ptr(kt),
+                                                 _ptr(difficulty), _ptr(mask), _ptr(kv_count), _ptr(ws),
+                                                 ctypes.c_size_t(ws.numel()), s))
     return mask, kv_count
 
 
@@ -259,12 +286,13 @@ def sparse_attn_fwd(g: Geometry, qt: torch.Tensor, kt: torch.Tensor, vt: torch.T
         _need(lse, torch.float32, (g.B, g.H, g.N), "lse")
     if ws is None:
         ws = alloc_workspace(g, dev)
+    _need_ws(ws)
     sc = 1.0 / math.sqrt(g.d) if scale is None else float(scale)
-    _check(load_library().bsa_sparse_attn_fwd(ctypes.byref(g.c()), _ptr(qt), _ptr(kt), _ptr(vt),
-                                              _ptr(mask), _ptr(kv_count), ctypes.c_float(sc),
-                                              _ptr(out), _ptr(lse), _ptr(ws),
-                                              ctypes.c_size_t(ws.numel()), _stream(stream)),
-           "bsa_sparse_attn_fwd")
+    _run("bsa_sparse_attn_fwd", _device_of(qt, kt, vt, mask, kv_count, out, lse, ws), stream,
+         lambda s: load_library().bsa_sparse_attn_fwd(ctypes.byref(g.c()), _ptr(qt), _ptr(kt), _ptr(vt),
+                                                      _ptr(mask), _ptr(kv_count), ctypes.c_float(sc),
+                                                      _ptr(out), _ptr(lse), _ptr(ws),
+                                                      ctypes.c_size_t(ws.numel()), s))
     return out, lse
 
 
@@ -301,10 +329,11 @@ def sparse_attn_fwd_fixed_scratch(g: Geometry, qt: torch.Tensor, kt: torch.Tenso
     if kernel_errors is not None:
         _need(kernel_errors, torch.int32, (1,), "kernel_errors")
     sc = 1.0 / math.sqrt(g.d) if scale is None else float(scale)
-    _check(load_library().bsa_sparse_attn_fwd_fixed_scratch(
-        ctypes.byref(g.c()), _ptr(qt), _ptr(kt), _ptr(vt), _ptr(mask), _ptr(kv_count),
-        ctypes.c_float(sc), _ptr(out), _ptr(lse), _ptr(kernel_errors), _stream(stream)),
-        "bsa_sparse_attn_fwd_fixed_scratch")
+    _run("bsa_sparse_attn_fwd_fixed_scratch", _device_of(qt, kt, vt, mask, kv_count, out, lse, kernel_errors),
+         stream,
+         lambda s: load_library().bsa_sparse_attn_fwd_fixed_scratch(
+             ctypes.byref(g.c()), _ptr(qt), _ptr(kt), _ptr(vt), _ptr(mask), _ptr(kv_count),
+             ctypes.c_float(sc), _ptr(out), _ptr(lse), _ptr(kernel_errors), s))
     return out, lse
 
 

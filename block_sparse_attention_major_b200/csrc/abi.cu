@@ -17,6 +17,11 @@ bool valid_geom(const bsa_geom* g) {
   if (g->B < 1 || g->H < 1 || g->T < 1 || g->Hs < 1 || g->Ws < 1) return false;
   if (g->d != 64 && g->d != 128) return false;
   if (g->Hs > 4096 || g->Ws > 4096 || g->T > 4096) return false;   // 10-bit tile coordinates
+  // A grid of more than 64 * kMaxTiles tokens has more than kMaxTiles tiles; rejecting it
+  // here keeps the token count in make_geom within int range.
+  if ((long long)g->T * g->Hs * g->Ws > 64LL * kMaxTiles) return false;
+  // The mask builder puts B, H and B*H on grid axes limited to 65535 blocks.
+  if ((long long)g->B * g->H > 65535) return false;
   const Geom G = make_geom(*g);
   if (G.NT > kMaxTiles) return false;
   const long long rows = (long long)g->B * g->H * G.NT * 64;

@@ -43,7 +43,8 @@ extern "C" {
 #endif
 
 /* Shape of one attention call. d (head dim) must be 64 or 128; B, H >= 1;
- * T, Hs, Ws >= 1 with NT <= 4096 tiles and B*H*NT*64 < 2^31 tile rows. */
+ * T, Hs, Ws >= 1 and at most 4096 each, with NT <= 4096 tiles, B*H <= 65535 and
+ * B*H*NT*64 < 2^31 tile rows. */
 typedef struct bsa_geom {
     int B;   /* batch items */
     int H;   /* attention heads */

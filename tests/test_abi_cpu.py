@@ -59,6 +59,9 @@ def test_tile_grid_and_workspace(lib):
 @pytest.mark.parametrize("bad", [
     dict(d=96), dict(d=0), dict(B=0), dict(H=0), dict(T=0), dict(Ws=-1),
     dict(T=400, Hs=400, Ws=400),                      # more than 4096 tiles
+    dict(T=4096, Hs=4096, Ws=4096),                   # token count beyond int range
+    dict(T=4097),                                     # more than 4096 per axis
+    dict(B=2, H=40000),                               # B*H above the 65535 grid limit
 ])
 def test_invalid_geometry_rejected_on_host(lib, bad):
     import block_sparse_attention_major_b200 as bsa
@@ -70,6 +73,16 @@ def test_invalid_geometry_rejected_on_host(lib, bad):
     buf = ctypes.create_string_buffer(64)
     assert lib.bsa_reorder(ctypes.byref(g), buf, buf, None) == 1
     assert lib.bsa_unreorder(ctypes.byref(g), buf, buf, None) == 1
+
+
+def test_largest_head_count_accepted_on_host(lib):
+    """B*H = 65535 heads of one tile is a valid geometry (the grid limit is inclusive)."""
+    import block_sparse_attention_major_b200 as bsa
+    g = bsa.bsa_geom(1, 65535, 64, 4, 4, 4)
+    nt = ctypes.c_int(0)
+    assert lib.bsa_tile_grid(ctypes.byref(g), None, None, None, ctypes.byref(nt)) == 0
+    assert nt.value == 1
+    assert lib.bsa_workspace_bytes(ctypes.byref(g), None) > 0
 
 
 def test_null_and_misaligned_pointers_rejected_on_host(lib):
@@ -115,6 +128,111 @@ def test_binding_fails_loudly_without_library(tmp_path):
     import block_sparse_attention_major_b200 as bsa
     with pytest.raises(RuntimeError):
         bsa.load_library(str(tmp_path / "missing.so"))
+
+
+def test_binding_refuses_mixed_devices():
+    """Tensors of one call must share a device: the library launches on the current device
+    with the pointers it is given, so a tensor elsewhere is refused before any call."""
+    import torch
+    import block_sparse_attention_major_b200 as bsa
+    a = torch.zeros(4)
+    m = torch.empty(4, device="meta")
+    assert bsa._device_of(a, None, a) == torch.device("cpu")
+    with pytest.raises(ValueError, match="share one device"):
+        bsa._device_of(a, m)
+    with pytest.raises(ValueError, match="share one device"):
+        bsa._device_of(None, None)
+
+
+@pytest.mark.parametrize("ws", ["host", "float", "2d", "strided"])
+def test_binding_refuses_a_bad_workspace(ws):
+    """The workspace must be device memory: a host tensor, or one of another dtype or shape,
+    is refused by the binding before the library sees its pointer."""
+    import torch
+    import block_sparse_attention_major_b200 as bsa
+    t = {"host": torch.zeros(1024, dtype=torch.uint8),
+         "float": torch.zeros(256, dtype=torch.float32),
+         "2d": torch.zeros(4, 256, dtype=torch.uint8),
+         "strided": torch.zeros(2048, dtype=torch.uint8)[::2]}[ws]
+    with pytest.raises(ValueError, match="ws must be"):
+        bsa._need_ws(t)
+    with pytest.raises(ValueError, match="ws must be"):
+        bsa.clear_error(t)
+
+
+def test_binding_wrappers_marshal_every_entry_point(monkeypatch):
+    """Every wrapper, driven on the CPU through a fake library and a fake current stream:
+    each reaches its C entry point once, with the stream of the tensors' device and the
+    pointers of the tensors it was given."""
+    import contextlib
+    import torch
+    import block_sparse_attention_major_b200 as bsa
+
+    calls = []
+
+    class FakeLib:
+        def __getattr__(self, name):
+            def f(*args):
+                calls.append((name, args))
+                return 0
+            return f
+
+    class FakeStream:
+        device = torch.device("cpu")
+        cuda_stream = 0x5000
+
+    monkeypatch.setattr(bsa, "load_library", lambda path=None: FakeLib())
+    monkeypatch.setattr(bsa, "_need", lambda t, dtype, shape, name: None)
+    monkeypatch.setattr(bsa, "_need_ws", lambda ws: None)
+    monkeypatch.setattr(torch.cuda, "device", lambda d: contextlib.nullcontext())
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda d=None: FakeStream())
+    g = bsa.Geometry(1, 2, 64, 8, 16, 16)
+    p = bsa.MaskParams(1, 2, 3, 0.25, 0, 0.0)
+    tiled = torch.zeros(g.B, g.H, g.NT, 64, g.d, dtype=torch.bfloat16)
+    raster = torch.zeros(g.B, g.N, g.H, g.d, dtype=torch.bfloat16)
+    mask = torch.zeros(g.B, g.H, g.NT, g.NW, dtype=torch.int32)
+    cnt = torch.zeros(g.B, g.H, g.NT, dtype=torch.int32)
+    diff = torch.zeros(g.B, g.NT)
+    ws = torch.zeros(4096, dtype=torch.uint8)
+    out = torch.zeros_like(raster)
+    lse = torch.zeros(g.B, g.H, g.N)
+    err = torch.zeros(1, dtype=torch.int32)
+
+    bsa.reorder(g, raster, tiled)
+    bsa.unreorder(g, tiled, raster)
+    bsa.build_mask(g, p, tiled, tiled, diff, mask, cnt, ws)
+    bsa.sparse_attn_fwd(g, tiled, tiled, tiled, mask, cnt, None, out, lse, ws)
+    bsa.sparse_attn_fwd_fixed_scratch(g, tiled, tiled, tiled, mask, cnt, None, out, lse, err)
+    bsa.clear_error(ws)
+    bsa.selftest_bounded_wait(err)
+    names = [c[0] for c in calls]
+    assert names == ["bsa_reorder", "bsa_unreorder", "bsa_build_mask", "bsa_sparse_attn_fwd",
+                     "bsa_sparse_attn_fwd_fixed_scratch", "bsa_clear_error", "bsa_selftest_bounded_wait"]
+    for name, args in calls:
+        assert args[-1].value == FakeStream.cuda_stream, name
+    ptr = lambda t: t.data_ptr()
+    assert [a.value for a in calls[0][1][1:3]] == [ptr(raster), ptr(tiled)]
+    assert [a.value for a in calls[1][1][1:3]] == [ptr(tiled), ptr(raster)]
+    bm = calls[2][1]
+    assert [a.value for a in bm[2:8]] == [ptr(tiled), ptr(tiled), ptr(diff), ptr(mask), ptr(cnt), ptr(ws)]
+    assert bm[8].value == ws.numel()
+    fw = calls[3][1]
+    assert abs(fw[6].value - 0.125) < 1e-7                 # 1/sqrt(64)
+    assert [a.value for a in (fw[7], fw[8], fw[9])] == [ptr(out), ptr(lse), ptr(ws)]
+    assert calls[4][1][9].value == ptr(err)
+
+    # a tensor of another device in the same call is refused before the library is called
+    calls.clear()
+    with pytest.raises(ValueError, match="share one device"):
+        bsa.sparse_attn_fwd(g, tiled, tiled, tiled.to("meta"), mask, cnt, None, out, lse, ws)
+    assert calls == []
+
+    # so is a stream of another device
+    class OtherStream(FakeStream):
+        device = torch.device("meta")
+    with pytest.raises(ValueError, match="stream is on"):
+        bsa.reorder(g, raster, tiled, stream=OtherStream())
+    assert calls == []
 
 
 def test_launch_counter_starts_at_zero_without_launches(lib):

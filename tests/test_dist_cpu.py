@@ -36,7 +36,7 @@ def _worker(rank, world, port, out):
 
 def test_reduce_over_two_gloo_ranks():
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:        # no fork of a multi-threaded process
         out = m.dict()
         mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
         res = dict(out)
