@@ -359,7 +359,14 @@ def forward(g: Geometry, p: MaskParams, q: torch.Tensor, k: torch.Tensor, v: tor
     """The whole path: reorder Q, K, V; build the mask; block-sparse attention.
 
     Returns the buffers; out / lse hold the attention output and LSE in raster order.
+    Window kind 2 (token-level circular support) is refused: its attention masks the tokens
+    outside the support inside window tiles, which the attention kernel does not do yet.
+    build_mask accepts kind 2; sparse_attn_fwd then attends whole retained tiles.
     """
+    if p.window_kind == 2:
+        raise ValueError("forward(): window kind 2 needs token-level masking inside window tiles, "
+                         "which the attention kernel does not apply yet; build_mask + "
+                         "sparse_attn_fwd give the tile-granular result")
     b = bufs or Buffers(g, q.device)
     reorder(g, q, b.qt, stream)
     reorder(g, k, b.kt, stream)

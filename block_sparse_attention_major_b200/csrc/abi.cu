@@ -4,6 +4,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "window.cuh"
 
 namespace bsa {
 
@@ -33,18 +34,24 @@ bool valid_geom(const bsa_geom* g) {
 
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Window kinds 0 and 1 take a radius in tiles, kind 2 a radius in tokens (window.cuh).
+bool valid_window(int kind, int radius) {
+  if (kind != 0 && kind != 1 && kind != 2) return false;
+  if (radius < 0) return false;
+  return kind != 2 || radius <= kMaxTokenRadius;
+}
+
 bool valid_params(const bsa_geom* g, const bsa_mask_params* p) {
   if (!p) return false;
   if (!(p->dense_fraction >= 0.0f && p->dense_fraction <= 1.0f)) return false;
   if (p->budget_mode == 0) {
-    if (p->window_kind != 0 && p->window_kind != 1) return false;
-    if (p->radius < 0 || p->topk < 0) return false;
+    if (!valid_window(p->window_kind, p->radius)) return false;
+    if (p->topk < 0) return false;
   } else if (p->budget_mode == 1) {
     if (p->window_kind != 1) return false;
     if (!(p->budget_target > 0.0f && p->budget_target <= 1.0f)) return false;
   } else if (p->budget_mode == 2) {
-    if (p->window_kind != 0 && p->window_kind != 1) return false;
-    if (p->radius < 0) return false;
+    if (!valid_window(p->window_kind, p->radius)) return false;
     if (!(p->budget_target > 0.0f && p->budget_target <= 1.0f)) return false;
   } else {
     return false;

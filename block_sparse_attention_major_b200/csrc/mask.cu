@@ -9,9 +9,10 @@
 //  entropy   (budget mode) entropy of each row's softmax of the scaled scores
 //  budget    (budget mode) per row: the tile budget, the window radius it affords and the
 //            number of extra tiles
-//  select    per (b, h, query tile): the local support - a cube window or a window whose
+//  select    per (b, h, query tile): the local support - a cube window, a window whose
 //            spatial radius decays with the frame-tile distance (Token Radius Attention
-//            summary, "Radius construction") - plus the best tiles outside it by pooled
+//            summary, "Radius construction"), or the tiles touched by a token-level
+//            circular support (window.cuh) - plus the best tiles outside it by pooled
 //            score: a fixed top-k, the remainder of a budget derived from the entropy
 //            (Token Radius Attention summary, "Entropy-guided budgeting"), or as many as
 //            it takes for the row's pooled probability to reach a target mass (the same
@@ -24,6 +25,7 @@
 // key (on counts, or on mass) followed by an index-ordered pass over tied keys. Both
 // reproduce "highest score, ties to the lower index" exactly and use no atomics.
 #include "common.cuh"
+#include "window.cuh"
 
 #include <math.h>
 
@@ -122,18 +124,6 @@ struct SelArgs {
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t u = __float_as_uint(f == 0.0f ? 0.0f : f);      // +0 and -0 tie
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-__device__ __forceinline__ uint32_t pack_coord(int tt, int ty, int tx) {
-  return ((uint32_t)tt << 20) | ((uint32_t)ty << 10) | (uint32_t)tx;
-}
-
-__device__ __forceinline__ bool in_window(uint32_t ci, uint32_t cj, int kind, int r) {
-  const int dt = abs((int)(ci >> 20) - (int)(cj >> 20));
-  const int dy = abs((int)((ci >> 10) & 1023u) - (int)((cj >> 10) & 1023u));
-  const int dx = abs((int)(ci & 1023u) - (int)(cj & 1023u));
-  if (kind == 0) return max(dt, max(dy, dx)) <= r;
-  return dt <= r && max(dy, dx) <= r - dt;
 }
 
 // Number of tiles in [c - s, c + s] clipped to [0, n).
@@ -336,7 +326,14 @@ __device__ __forceinline__ float order_key_inverse(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-template <int MODE, int KW, int WPR>
+// TOK: the window is the token-level support (kind 2), a separate instantiation so that the
+// tile-window kinds keep their own register allocation.
+template <int MODE, int KW, int WPR, bool TOK>
+__device__ __forceinline__ bool sel_in_window(uint32_t ci, uint32_t cj, int kind, int r) {
+  return TOK ? in_token_window(ci, cj, r) : in_tile_window(ci, cj, kind, r);
+}
+
+template <int MODE, int KW, int WPR, bool TOK>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const float* __restrict__ S, int NKTP) {
   extern __shared__ __align__(16) uint32_t sm_u32[];
   constexpr int kRows = kSelWarps / WPR;
@@ -408,7 +405,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
     for (int w = 0; w < KW; ++w) {
       const int j = 32 * (q * KW + w) + lane;
       const bool inrow = j < NKT;
-      const bool inw = inrow && in_window(ci, coord[j], kind, rad);
+      const bool inw = inrow && sel_in_window<MODE, KW, WPR, TOK>(ci, coord[j], kind, rad);
       const float e = inrow ? exp2f((srow[j] - mx) * c) : 0.0f;
       z += e;
       zw += inw ? e : 0.0f;
@@ -423,7 +420,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
 #pragma unroll
     for (int w = 0; w < KW; ++w) {
       const int j = 32 * (q * KW + w) + lane;
-      const bool cand = j < NKT && !in_window(ci, coord[j], kind, rad);
+      const bool cand = j < NKT && !sel_in_window<MODE, KW, WPR, TOK>(ci, coord[j], kind, rad);
       kr[w] = cand ? order_key(srow[j]) : 0u;
       ncand += __popc(__ballot_sync(0xffffffffu, cand));
     }
@@ -575,23 +572,24 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
   if (q == 0 && lane == 0) a.kv_count[rowid] = count;
 }
 
-template <int MODE, int KW, int WPR>
+template <int MODE, int KW, int WPR, bool TOK>
 cudaError_t launch_select_kw(const Geom& g, size_t smem, const SelArgs& a, const float* S, int NKTP, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<MODE, KW, WPR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<MODE, KW, WPR, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid(ceil_div(g.NT, kSelWarps / WPR), g.H, g.B);
-  select_kernel<MODE, KW, WPR><<<grid, kSelThreads, smem, s>>>(a, S, NKTP);
+  select_kernel<MODE, KW, WPR, TOK><<<grid, kSelThreads, smem, s>>>(a, S, NKTP);
   return cudaGetLastError();
 }
 
 // Words of a mask row per lane at most 32: rows of more than 32 words span 2 or 4 warps.
-template <int MODE>
+template <int MODE, bool TOK>
 cudaError_t launch_select(const Geom& g, size_t smem, const SelArgs& a, const float* S, int NKTP, cudaStream_t s) {
-  if (g.NW <= 8) return launch_select_kw<MODE, 8, 1>(g, smem, a, S, NKTP, s);
-  if (g.NW <= 16) return launch_select_kw<MODE, 16, 1>(g, smem, a, S, NKTP, s);
-  if (g.NW <= 32) return launch_select_kw<MODE, 32, 1>(g, smem, a, S, NKTP, s);
-  if (g.NW <= 64) return launch_select_kw<MODE, 32, 2>(g, smem, a, S, NKTP, s);
-  return launch_select_kw<MODE, 32, 4>(g, smem, a, S, NKTP, s);
+  if (g.NW <= 8) return launch_select_kw<MODE, 8, 1, TOK>(g, smem, a, S, NKTP, s);
+  if (g.NW <= 16) return launch_select_kw<MODE, 16, 1, TOK>(g, smem, a, S, NKTP, s);
+  if (g.NW <= 32) return launch_select_kw<MODE, 32, 1, TOK>(g, smem, a, S, NKTP, s);
+  if (g.NW <= 64) return launch_select_kw<MODE, 32, 2, TOK>(g, smem, a, S, NKTP, s);
+  return launch_select_kw<MODE, 32, 4, TOK>(g, smem, a, S, NKTP, s);
 }
 
 template <int D>
@@ -655,9 +653,16 @@ cudaError_t build_mask_d(const Geom& g, const bsa_mask_params& p, const __nv_bfl
   // coordinate table, then per row of the block a double-buffered exchange of one 64-bit
   // value per warp
   const size_t sel_smem = sizeof(uint32_t) * (size_t)((NKTP + 1) & ~1) + (size_t)kSelWarps * 2 * sizeof(uint64_t);
-  e = p.budget_mode == 0   ? launch_select<kSelectFixed>(g, sel_smem, a, S, NKTP, s)
-      : p.budget_mode == 2 ? launch_select<kSelectMass>(g, sel_smem, a, S, NKTP, s)
-                           : launch_select<kSelectBudget>(g, sel_smem, a, S, NKTP, s);
+  // the budget mode always uses the decayed tile window (kind 1)
+  const bool tok = p.window_kind == 2;
+  if (p.budget_mode == 0)
+    e = tok ? launch_select<kSelectFixed, true>(g, sel_smem, a, S, NKTP, s)
+            : launch_select<kSelectFixed, false>(g, sel_smem, a, S, NKTP, s);
+  else if (p.budget_mode == 2)
+    e = tok ? launch_select<kSelectMass, true>(g, sel_smem, a, S, NKTP, s)
+            : launch_select<kSelectMass, false>(g, sel_smem, a, S, NKTP, s);
+  else
+    e = launch_select<kSelectBudget, false>(g, sel_smem, a, S, NKTP, s);
   if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();

@@ -59,7 +59,18 @@ typedef struct bsa_geom {
  *   window_kind   0: cube window, max(|dt|,|dy|,|dx|) <= radius (tile units)
  *                 1: window with temporal decay, |dt| <= radius and
  *                    max(|dy|,|dx|) <= radius - |dt|
- *   radius        window radius in tiles (>= 0); ignored when budget_mode = 1
+ *                 2: the tiles touched by a token-level circular support with temporal
+ *                    decay (Token Radius Attention summary: query-centred circular
+ *                    neighbourhoods, base radius applied across frames with decay): key
+ *                    token m supports query token n when |t_m - t_n| <= radius and
+ *                    (y_m - y_n)^2 + (x_m - x_n)^2 <= (radius - |t_m - t_n|)^2, in tokens;
+ *                    key tile j is a window tile of query tile i when a valid token of j
+ *                    supports a valid token of i. Budget modes 0 and 2 only. The mask is
+ *                    tile-granular: bsa_sparse_attn_fwd attends every valid token of each
+ *                    retained tile (it does not yet mask the tokens outside the support
+ *                    inside window tiles)
+ *   radius        window radius (>= 0): in tiles for kinds 0 and 1, in tokens (at most
+ *                 32767) for kind 2; ignored when budget_mode = 1
  *   topk          extra key tiles outside the window, by pooled score, ties to the lower
  *                 tile index; capped at the number of tiles outside the window (>= 0)
  *   dense_fraction rho in [0,1]: the floor(rho*NQT + 1/2) query tiles of highest

@@ -27,6 +27,13 @@ SMALL_D128 = {
     "mass128": Workload("mass128", B=2, H=2, d=128, T=8, Hs=14, Ws=20, seed=1013,
                         window_kind=0, radius=1, topk=0, dense_fraction=0.2,
                         budget_mode=2, budget_target=0.5),
+    # token-level circular support (window kind 2, radius in tokens): fixed top-k on the
+    # 8 x 16 x 16 grid, cumulative mass on a ragged grid
+    "token128": Workload("token128", B=1, H=2, d=128, T=8, Hs=16, Ws=16, seed=1016,
+                         window_kind=2, radius=6, topk=3, dense_fraction=0.25),
+    "token_mass": Workload("token_mass", B=2, H=2, d=64, T=7, Hs=13, Ws=10, seed=1017,
+                           window_kind=2, radius=5, topk=0, dense_fraction=0.2,
+                           budget_mode=2, budget_target=0.5),
     # edge cases: a grid of one (partial) tile, and the largest supported tile count
     "one_tile": Workload("one_tile", B=1, H=2, d=64, T=3, Hs=3, Ws=3, seed=1014,
                          window_kind=0, radius=1, topk=2, dense_fraction=0.0),

@@ -105,11 +105,14 @@ def test_null_and_misaligned_pointers_rejected_on_host(lib):
 
 
 @pytest.mark.parametrize("bad", [
-    dict(dense_fraction=1.5), dict(dense_fraction=-0.1), dict(window_kind=2), dict(radius=-1),
+    dict(dense_fraction=1.5), dict(dense_fraction=-0.1), dict(window_kind=-1), dict(radius=-1),
     dict(topk=-3), dict(budget_mode=2), dict(budget_mode=1, window_kind=0, budget_target=0.1),
     dict(budget_mode=1, window_kind=1, budget_target=0.0),
     dict(budget_mode=3, budget_target=0.5), dict(budget_mode=2, budget_target=1.5),
-    dict(budget_mode=2, budget_target=0.5, radius=-1), dict(budget_mode=2, budget_target=0.5, window_kind=2),
+    dict(budget_mode=2, budget_target=0.5, radius=-1), dict(budget_mode=2, budget_target=0.5, window_kind=3),
+    dict(window_kind=2, radius=32768), dict(window_kind=2, radius=-1), dict(window_kind=3),
+    dict(budget_mode=1, window_kind=2, budget_target=0.2),
+    dict(budget_mode=2, budget_target=0.5, window_kind=2, radius=40000),
 ])
 def test_invalid_mask_params_rejected_on_host(lib, bad):
     import block_sparse_attention_major_b200 as bsa
@@ -122,6 +125,16 @@ def test_invalid_mask_params_rejected_on_host(lib, bad):
     al = ctypes.c_void_p(0x1000)
     assert lib.bsa_build_mask(ctypes.byref(g), ctypes.byref(p), al, al, al, al, al,
                               ctypes.c_void_p(0x10000), 1 << 30, None) == 1
+
+
+def test_forward_refuses_token_window():
+    """forward() does not hand a kind-2 mask to an attention that would attend whole tiles."""
+    import torch
+    import block_sparse_attention_major_b200 as bsa
+    g = bsa.Geometry(1, 1, 64, 4, 4, 4)
+    x = torch.zeros(1, 64, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="window kind 2"):
+        bsa.forward(g, bsa.MaskParams(2, 6, 1), x, x, x, torch.zeros(1, 1))
 
 
 def test_binding_fails_loudly_without_library(tmp_path):

@@ -359,3 +359,21 @@ def test_forward_path_full_size(name, overrides):
     st = C.compare_attention(w, b.out, b.lse, ref, skip_rows=skip)
     print(name, st, cmp["n_diff"], "retained", float(gm.mean()))
     C.assert_attention_close(st)
+
+
+# ----------------------------------------------------------------------------- window kind 2
+@pytest.mark.parametrize("name,overrides", [
+    ("token128", ()), ("token_mass", ()),
+    ("wan13b", (("window_kind", 2), ("radius", 6))),          # 4 r + 2 tokens for r = 1
+])
+def test_mask_token_window(name, overrides):
+    """Masks whose local support is the token-level circular support (radius in tokens):
+    bit-exact against the oracle, whose window is a brute force over token pairs."""
+    heads = [0, 11] if name == "wan13b" else None
+    w, g, gm, ref, cmp, _, _ = _mask_case(name, heads=heads, overrides=overrides)
+    assert cmp["n_unflagged"] == 0, cmp
+    assert cmp["n_diff"] <= max(1, cmp["n_rows"] // 200), cmp
+    local = ~ref["dense"][:, None, :, None]
+    assert np.all(gm >= (ref["window"][None, None] & local)), "a window tile is missing"
+    print(f"{name}: retained={gm.mean():.4f} window={ref['window'].mean():.4f} "
+          f"flagged={cmp['n_flagged']} differing={cmp['n_diff']}")

@@ -1,0 +1,17 @@
+// Host build of the mask builder's window predicate (csrc/window.cuh), for the CPU tests:
+// enumerates the window of every query tile of a T x Hs x Ws grid as a [NT, NT] byte
+// matrix. The tests compare it with the oracle's own enumeration.
+#include "window.cuh"
+
+extern "C" int window_tiles(int T, int Hs, int Ws, int kind, int r, unsigned char* out) {
+  const int nT = (T + 3) / 4, nY = (Hs + 3) / 4, nX = (Ws + 3) / 4;
+  const int NT = nT * nY * nX;
+  for (int i = 0; i < NT; ++i) {
+    const uint32_t ci = bsa::pack_coord(i / (nY * nX), (i / nX) % nY, i % nX);
+    for (int j = 0; j < NT; ++j) {
+      const uint32_t cj = bsa::pack_coord(j / (nY * nX), (j / nX) % nY, j % nX);
+      out[(long long)i * NT + j] = bsa::in_window(ci, cj, kind, r) ? 1 : 0;
+    }
+  }
+  return NT;
+}
