@@ -3,18 +3,23 @@
 The attention kernel hands work between a TMA producer, one MMA-issuing thread per
 sub-unit and two softmax warpgroups through mbarriers that are tested by phase parity.
 This model replays that protocol on the unit lists of real masks under random
-interleavings and checks that it always finishes (no deadlock) and that every product
-reads the key/value tile it was meant to read (no stale ring stage).
+interleavings and checks that it always finishes (no deadlock) and that every read sees
+what it should: each product the key/value tile of its entry (no stale ring stage), the
+softmax S of its own block, each P.V the P of its own block, O holding exactly the blocks
+before it at each P.V and rescale, and every block at the epilogue.
 
 mbarrier semantics modelled: a phase completes when its expected arrival count is
 reached; a parity test for parity P succeeds when the current phase's parity differs from
-P, so a barrier two phases behind the awaited one looks complete (the hazard the kernel's
-issuers avoid by walking every entry of the union list in order). The tensor pipe runs
-products in issue order; a commit arrives once the products issued before it are done.
+P, so a barrier two phases behind the awaited one looks complete. Each issuing thread's
+products run in its issue order, and its commit arrives once the products it issued
+before the commit are done; nothing orders the two issuers' products against each other.
 
-A second, deliberately careless protocol (one issuer that tests a sub-unit's next entry
-without walking the others) is run too and must be caught, which shows the checker can
-see the hazard.
+The protocol: S-full barriers per (sub-unit, S buffer), one P-ready and one P.V-done
+barrier per sub-unit, and a softmax that waits for the previous block's P.V before it
+releases P (and rescales O, when the row max grew). Deliberately broken variants must be
+caught, which shows the checker can see the hazards: issuers that test only their own next
+entries (ring stages), a softmax that releases P without that wait, an epilogue that waits
+one block early, and QK products three blocks ahead of P.V.
 """
 import random
 
@@ -63,8 +68,21 @@ def units_from_mask(mask):
     return out
 
 
-def run_protocol(L, need_a, need_b, seed, careless=False):
-    """True if the unit finishes; False on deadlock; raises Stale on a wrong-tile read."""
+def run_protocol(L, need_a, need_b, seed, careless=False, no_wait=False):
+    """True if the unit finishes; False on deadlock; raises Stale on a wrong read.
+
+    Besides the ring stages, the model tracks what each S buffer holds (S of block it after
+    its QK product, P of block it after the softmax released it) and how many P.V
+    products O has absorbed, and checks every read against them: the softmax reads S of
+    its own block, a P.V reads P of its own block and adds to O holding exactly the
+    blocks before it, a rescale sees O holding exactly the blocks before it, and the
+    epilogue sees every block. From its second block on, a softmax waits for the previous
+    P.V (then may rescale O) before it releases P.
+
+    careless: one issuer per sub-unit that tests only its own next entries (ring hazard).
+    no_wait: the softmax releases P without that wait (it can then run two P-ready phases
+    ahead of the issuer).
+    """
     rng = random.Random(seed)
     need = [need_a, need_b]
     has = [any(need_a), any(need_b)]
@@ -74,13 +92,22 @@ def run_protocol(L, need_a, need_b, seed, careless=False):
     kfull, vfull = [Bar(1) for _ in range(NS)], [Bar(1) for _ in range(NS)]
     kempty = [Bar(1 if careless else users) for _ in range(NS)]
     vempty = [Bar(1 if careless else users) for _ in range(NS)]
-    sfull = [Bar(1) for _ in range(4)]
-    pfull, odone = [Bar(1) for _ in range(2)], [Bar(1) for _ in range(2)]
-    pipe, kload, vload = [], [], []
+    sfull = [Bar(1) for _ in range(4)]          # 2u + b
+    pfull = [Bar(1) for _ in range(2)]          # u
+    odone = [Bar(1) for _ in range(2)]          # u
+    pipe, kload, vload = [[], []], [], []     # one product queue per issuing thread
     kdata, vdata = [None] * NS, [None] * NS
+    sbuf = [[None, None], [None, None]]         # ('S', it) or ('P', it)
+    oblocks = [0, 0]                            # P.V products absorbed by O
     prod = [0, 'k']
     ki, vi, qc, pc = [0, 0], [0, 0], [0, 0], [0, 0]
     sm = [[0, 'wait_s'], [0, 'wait_s']]
+
+    def pbar(u, it):
+        return pfull[u], it & 1
+
+    def obar(u, it):
+        return odone[u], it & 1
 
     def actions():
         acts = []
@@ -95,19 +122,19 @@ def run_protocol(L, need_a, need_b, seed, careless=False):
             acts.append(('tma_k',))
         if vload:
             acts.append(('tma_v',))
-        if pipe:
-            acts.append(('pipe',))
+        for u in range(2):
+            if pipe[u]:
+                acts.append(('pipe', u))
         for u in range(2):
             if not has[u]:
                 continue
             if careless:
-                # one issuer per sub-unit that tests only its own next entries; the last
-                # user of a stage frees it
                 if qc[u] < n[u] and qc[u] - pc[u] < 2:
                     e = blk[u][qc[u]]
                     if kfull[e % NS].test((e // NS) & 1):
                         acts.append(('qk', u))
-                if pc[u] < qc[u] and pfull[u].test(pc[u] & 1):
+                bar, par = pbar(u, pc[u])
+                if pc[u] < qc[u] and bar.test(par):
                     e = blk[u][pc[u]]
                     if vfull[e % NS].test((e // NS) & 1):
                         acts.append(('pv', u))
@@ -122,14 +149,24 @@ def run_protocol(L, need_a, need_b, seed, careless=False):
                 if v < ki[u] and vfull[v % NS].test((v // NS) & 1):
                     if not need[u][v]:
                         acts.append(('v_arrive', u))
-                    elif pfull[u].test(pc[u] & 1):
-                        acts.append(('pv', u))
+                    else:
+                        bar, par = pbar(u, pc[u])
+                        if bar.test(par):
+                            acts.append(('pv', u))
             it, st = sm[u]
             if it < n[u]:
                 if st == 'wait_s' and sfull[2 * u + (it & 1)].test((it >> 1) & 1):
                     acts.append(('softmax_s', u))
-                if st == 'wait_o' and (it == 0 or odone[u].test((it - 1) & 1)):
+                if st == 'wait_o':
+                    bar, par = obar(u, it - 1)
+                    if bar.test(par):
+                        acts.append(('softmax_rescale', u))
+                if st == 'release':
                     acts.append(('softmax_p', u))
+            elif st != 'done':
+                bar, par = obar(u, n[u] - 1)
+                if n[u] == 0 or bar.test(par):
+                    acts.append(('epilogue', u))
         return acts
 
     def last_user(u, e, cursor):
@@ -138,9 +175,9 @@ def run_protocol(L, need_a, need_b, seed, careless=False):
 
     while True:
         acts = actions()
-        finished = (prod[0] >= L and all(sm[u][0] >= n[u] for u in range(2))
+        finished = (prod[0] >= L and all(sm[u][1] == 'done' or not has[u] for u in range(2))
                     and all(pc[u] >= n[u] for u in range(2)))
-        if finished and not pipe and not kload and not vload:
+        if finished and not pipe[0] and not pipe[1] and not kload and not vload:
             return True
         if not acts:
             return False
@@ -162,24 +199,36 @@ def run_protocol(L, need_a, need_b, seed, careless=False):
             vdata[s] = e
             vfull[s].arrive()
         elif kind == 'pipe':
-            op = pipe.pop(0)
+            op = pipe[a[1]].pop(0)
             if op[0] == 'commit':
                 op[1].arrive()
+            elif op[0] == 'qk':
+                _, u, it, s, e = op
+                if kdata[s] != e:
+                    raise Stale(f"QK of entry {e} read K stage {s} holding {kdata[s]}")
+                if it >= 2 and oblocks[u] < it - 1:
+                    raise Stale(f"S of block {it} overwrote P of block {it - 2} before its P.V")
+                sbuf[u][it & 1] = ('S', it)
             else:
-                _, which, s, e = op
-                if (kdata if which == 'k' else vdata)[s] != e:
-                    raise Stale(f"{which} product on entry {e} read stage {s} holding {(kdata if which == 'k' else vdata)[s]}")
+                _, u, it, s, e = op
+                if vdata[s] != e:
+                    raise Stale(f"P.V of entry {e} read V stage {s} holding {vdata[s]}")
+                if sbuf[u][it & 1] != ('P', it):
+                    raise Stale(f"P.V of block {it} read {sbuf[u][it & 1]}")
+                if oblocks[u] != it:
+                    raise Stale(f"P.V of block {it} added to O holding {oblocks[u]} blocks")
+                oblocks[u] += 1
         elif kind == 'qk':
             u = a[1]
             e = blk[u][qc[u]]
             s = e % NS
-            pipe += [('mma', 'k', s, e), ('commit', sfull[2 * u + (qc[u] & 1)])]
+            pipe[u] += [('qk', u, qc[u], s, e), ('commit', sfull[2 * u + (qc[u] & 1)])]
             qc[u] += 1
             if careless:
                 if last_user(u, e, qc):
-                    pipe.append(('commit', kempty[s]))
+                    pipe[u].append(('commit', kempty[s]))
             else:
-                pipe.append(('commit', kempty[s]))
+                pipe[u].append(('commit', kempty[s]))
                 ki[u] += 1
         elif kind == 'k_arrive':
             u = a[1]
@@ -189,24 +238,41 @@ def run_protocol(L, need_a, need_b, seed, careless=False):
             u = a[1]
             e = blk[u][pc[u]]
             s = e % NS
-            pipe += [('mma', 'v', s, e), ('commit', odone[u])]
+            pipe[u] += [('pv', u, pc[u], s, e), ('commit', obar(u, pc[u])[0])]
             pc[u] += 1
             if careless:
                 if last_user(u, e, pc):
-                    pipe.append(('commit', vempty[s]))
+                    pipe[u].append(('commit', vempty[s]))
             else:
-                pipe.append(('commit', vempty[s]))
+                pipe[u].append(('commit', vempty[s]))
                 vi[u] += 1
         elif kind == 'v_arrive':
             u = a[1]
             vempty[vi[u] % NS].arrive()
             vi[u] += 1
         elif kind == 'softmax_s':
-            sm[a[1]][1] = 'wait_o'
+            u = a[1]
+            it = sm[u][0]
+            if sbuf[u][it & 1] != ('S', it):
+                raise Stale(f"softmax of block {it} read {sbuf[u][it & 1]}")
+            sm[u][1] = 'wait_o' if it > 0 and not no_wait else 'release'
+        elif kind == 'softmax_rescale':
+            u = a[1]
+            if oblocks[u] != sm[u][0]:
+                raise Stale(f"rescale at block {sm[u][0]} saw O holding {oblocks[u]} blocks")
+            sm[u][1] = 'release'
         elif kind == 'softmax_p':
             u = a[1]
-            pfull[u].arrive()
-            sm[u] = [sm[u][0] + 1, 'wait_s']
+            it = sm[u][0]
+            sbuf[u][it & 1] = ('P', it)
+            bar, _ = pbar(u, it)
+            bar.arrive()
+            sm[u] = [it + 1, 'wait_s']
+        elif kind == 'epilogue':
+            u = a[1]
+            if oblocks[u] != n[u]:
+                raise Stale(f"epilogue read O holding {oblocks[u]} of {n[u]} blocks")
+            sm[u][1] = 'done'
 
 
 def _case_units(name):
@@ -247,6 +313,45 @@ def test_careless_protocol_is_caught():
         for seed in range(12):
             try:
                 caught += not run_protocol(L, na, nb, seed, careless=True)
+            except Stale:
+                caught += 1
+    assert caught > 0
+
+
+def test_release_without_waiting_is_caught():
+    """Without the wait for the previous P.V, a softmax can complete two phases of its
+    single P-ready barrier before the issuer tests the first: the parity test aliases, and
+    the checker must report a deadlock or a wrong read."""
+    caught = 0
+    for L, na, nb in _case_units("budget128"):
+        for seed in range(12):
+            try:
+                caught += not run_protocol(L, na, nb, seed, no_wait=True)
+            except Stale:
+                caught += 1
+    assert caught > 0
+
+
+@pytest.mark.parametrize("mutation", ["epilogue_one_block_early", "qk_three_blocks_ahead"])
+def test_broken_waits_are_caught(mutation):
+    """The same checker on two one-line mistakes: an epilogue that waits for the last P.V
+    but one, and QK products allowed three blocks ahead of P.V (S would overwrite P before
+    its product)."""
+    import inspect
+    import textwrap
+    src = inspect.getsource(run_protocol)
+    a, b = {
+        "epilogue_one_block_early": ("bar, par = obar(u, n[u] - 1)", "bar, par = obar(u, max(n[u] - 2, 0))"),
+        "qk_three_blocks_ahead": ("elif qc[u] - pc[u] < 2:", "elif qc[u] - pc[u] < 3:"),
+    }[mutation]
+    assert a in src
+    ns = dict(globals())
+    exec(textwrap.dedent(src.replace(a, b)), ns)
+    caught = 0
+    for L, na, nb in _case_units("budget128"):
+        for seed in range(12):
+            try:
+                caught += not ns["run_protocol"](L, na, nb, seed)
             except Stale:
                 caught += 1
     assert caught > 0
