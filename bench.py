@@ -605,6 +605,10 @@ def run_report(args):
             "workload": name, "B": g.B, "H": g.H, "d": g.d, "grid": [g.T, g.Hs, g.Ws], "tiles": g.NT,
             "retained_tile_fraction": retained / dense_pairs, "ms": res,
             "ms_step": sum(res.values()),
+            # a step whose mask is rebuilt every m calls and reused in between (forward's
+            # rebuild_mask): the measured stage times with the mask build amortised
+            "ms_step_mask_rebuilt_every": {m: res["reorder_qkv"] + res["sparse_attn"] + res["build_mask"] / m
+                                           for m in (1, 2, 4, 8)},
             "attn_effective_tflops": flops / (res["sparse_attn"] * 1e-3) / 1e12,
             "step_effective_tflops": flops / (sum(res.values()) * 1e-3) / 1e12,
             "reorder_gbs": qkv_bytes / (res["reorder_qkv"] * 1e-3) / 1e9,

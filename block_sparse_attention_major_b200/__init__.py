@@ -355,10 +355,14 @@ class Buffers:
 
 def forward(g: Geometry, p: MaskParams, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
             difficulty: torch.Tensor, bufs: Buffers | None = None, scale: float | None = None,
-            stream=None) -> Buffers:
+            stream=None, rebuild_mask: bool = True) -> Buffers:
     """The whole path: reorder Q, K, V; build the mask; block-sparse attention.
 
     Returns the buffers; out / lse hold the attention output and LSE in raster order.
+    rebuild_mask=False skips the mask build and attends through the mask (and counts) that
+    an earlier call left in `bufs`: the reuse of a previous step's routing and sparsity
+    (HetA-DiT reuses the preceding denoising step's estimates; MOD-DiT keeps historical
+    sparsity). How often to rebuild is the caller's choice.
     Window kind 2 (token-level circular support) is refused: its attention masks the tokens
     outside the support inside window tiles, which the attention kernel does not do yet.
     build_mask accepts kind 2; sparse_attn_fwd then attends whole retained tiles.
@@ -367,17 +371,22 @@ def forward(g: Geometry, p: MaskParams, q: torch.Tensor, k: torch.Tensor, v: tor
         raise ValueError("forward(): window kind 2 needs token-level masking inside window tiles, "
                          "which the attention kernel does not apply yet; build_mask + "
                          "sparse_attn_fwd give the tile-granular result")
+    if not rebuild_mask and bufs is None:
+        raise ValueError("rebuild_mask=False attends through the mask held in bufs: pass the "
+                         "Buffers of an earlier call")
     b = bufs or Buffers(g, q.device)
     reorder(g, q, b.qt, stream)
     reorder(g, k, b.kt, stream)
     reorder(g, v, b.vt, stream)
-    build_mask(g, p, b.qt, b.kt, difficulty, b.mask, b.kv_count, b.ws, stream)
+    if rebuild_mask:
+        build_mask(g, p, b.qt, b.kt, difficulty, b.mask, b.kv_count, b.ws, stream)
     sparse_attn_fwd(g, b.qt, b.kt, b.vt, b.mask, b.kv_count, scale, b.out, b.lse, b.ws,
                     stream=stream)
     return b
 
 
 # kernels launched by forward(): 3 reorders; pool, route, score and select (plus entropy
-# and budget in budget mode); 3 scheduler kernels and the attention kernel
-def launches_per_forward(p: MaskParams) -> int:
-    return 3 + 4 + (2 if p.budget_mode == 1 else 0) + 4
+# and budget in budget mode) unless the mask is reused; 3 scheduler kernels and the
+# attention kernel
+def launches_per_forward(p: MaskParams, rebuild_mask: bool = True) -> int:
+    return 3 + ((4 + (2 if p.budget_mode == 1 else 0)) if rebuild_mask else 0) + 4

@@ -248,6 +248,48 @@ def test_binding_wrappers_marshal_every_entry_point(monkeypatch):
     assert calls == []
 
 
+def test_forward_mask_reuse_skips_the_build(monkeypatch):
+    """forward(rebuild_mask=False) reorders and attends through the buffers' mask without
+    calling the mask builder; without earlier buffers it refuses."""
+    import contextlib
+    import types
+    import torch
+    import block_sparse_attention_major_b200 as bsa
+
+    calls = []
+
+    class FakeLib:
+        def __getattr__(self, name):
+            return lambda *args: calls.append(name) or 0
+
+    class FakeStream:
+        device = torch.device("cpu")
+        cuda_stream = 0x5000
+
+    monkeypatch.setattr(bsa, "load_library", lambda path=None: FakeLib())
+    monkeypatch.setattr(bsa, "_need", lambda t, dtype, shape, name: None)
+    monkeypatch.setattr(bsa, "_need_ws", lambda ws: None)
+    monkeypatch.setattr(torch.cuda, "device", lambda d: contextlib.nullcontext())
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda d=None: FakeStream())
+    g = bsa.Geometry(1, 2, 64, 8, 16, 16)
+    p = bsa.MaskParams(1, 1, 2, 0.25)
+    t = lambda *shape, dt=torch.bfloat16: torch.zeros(*shape, dtype=dt)
+    b = types.SimpleNamespace(qt=t(1, 2, g.NT, 64, 64), kt=t(1, 2, g.NT, 64, 64), vt=t(1, 2, g.NT, 64, 64),
+                              mask=t(1, 2, g.NT, g.NW, dt=torch.int32), kv_count=t(1, 2, g.NT, dt=torch.int32),
+                              out=t(1, g.N, 2, 64), lse=t(1, 2, g.N, dt=torch.float32),
+                              ws=t(4096, dt=torch.uint8))
+    x = t(1, g.N, 2, 64)
+    d = t(1, g.NT, dt=torch.float32)
+    bsa.forward(g, p, x, x, x, d, bufs=b)
+    assert calls == ["bsa_reorder"] * 3 + ["bsa_build_mask", "bsa_sparse_attn_fwd"]
+    calls.clear()
+    bsa.forward(g, p, x, x, x, d, bufs=b, rebuild_mask=False)
+    assert calls == ["bsa_reorder"] * 3 + ["bsa_sparse_attn_fwd"]
+    assert bsa.launches_per_forward(p, rebuild_mask=False) == bsa.launches_per_forward(p) - 4
+    with pytest.raises(ValueError, match="earlier call"):
+        bsa.forward(g, p, x, x, x, d, rebuild_mask=False)
+
+
 def test_launch_counter_starts_at_zero_without_launches(lib):
     assert lib.bsa_launch_count() == 0
 

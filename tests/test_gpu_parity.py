@@ -377,3 +377,32 @@ def test_mask_token_window(name, overrides):
     assert np.all(gm >= (ref["window"][None, None] & local)), "a window tile is missing"
     print(f"{name}: retained={gm.mean():.4f} window={ref['window'].mean():.4f} "
           f"flagged={cmp['n_flagged']} differing={cmp['n_diff']}")
+
+
+def test_forward_mask_reuse():
+    """forward(rebuild_mask=False) attends a new call's inputs through the mask an earlier
+    call built: against the oracle's attention on the new inputs under the oracle's mask of
+    the earlier inputs (rows where the GPU's earlier mask differs at a near-tie skipped)."""
+    bsa = _bsa()
+    wa, qa, ka, va, da = C.inputs("small128")
+    wb, qb, kb, vb, db = C.inputs("small128", (("seed", wa.seed + 7),))
+    g = C.geometry(wa)
+    p = C.params(wa)
+    b = bsa.forward(g, p, qa.cuda(), ka.cuda(), va.cuda(), da.cuda())
+    mask_a, cnt_a = b.mask.clone(), b.kv_count.clone()
+    n0 = bsa.launch_count()
+    bsa.forward(g, p, qb.cuda(), kb.cuda(), vb.cuda(), db.cuda(), bufs=b, rebuild_mask=False)
+    torch.cuda.synchronize()
+    assert bsa.launch_count() - n0 == bsa.launches_per_forward(p, rebuild_mask=False)
+    assert torch.equal(b.mask, mask_a) and torch.equal(b.kv_count, cnt_a)
+    assert bsa.read_error(b.ws) == 0
+    qa64, ka64 = (O.reorder(O.to_f64(x), wa.T, wa.Hs, wa.Ws) for x in (qa, ka))
+    mref = C.oracle_mask(wa, qa64, ka64, da.numpy())
+    cmp = C.compare_masks(C.gpu_mask_bool(mask_a, g.NT), mref)
+    assert cmp["n_unflagged"] == 0, cmp
+    qb64, kb64, vb64 = (O.reorder(O.to_f64(x), wb.T, wb.Hs, wb.Ws) for x in (qb, kb, vb))
+    rows = [(bb, h, i) for bb in range(wb.B) for h in range(wb.H) for i in range(g.NT)]
+    ref = O.attention_tiles(qb64, kb64, vb64, mref["mask"], rows, T=wb.T, Hs=wb.Hs, Ws=wb.Ws)
+    st = C.compare_attention(wb, b.out, b.lse, ref, skip_rows=cmp["diff_rows"])
+    print(st)
+    C.assert_attention_close(st)
