@@ -1,7 +1,11 @@
 // C ABI of libbsa: argument validation, workspace sizing and dispatch to the kernels.
-// No entry point allocates, synchronises or copies between host and device.
+// No entry point allocates, synchronises or copies between host and device. Each entry
+// point that enqueues work is an NVTX range named after it (a no-op unless a profiler is
+// attached), so that profiles and ncu's NVTX filters can tell the calls apart.
 #include <atomic>
 #include <math.h>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "common.cuh"
 #include "window.cuh"
@@ -33,6 +37,14 @@ bool valid_geom(const bsa_geom* g) {
 }
 
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// NVTX range for the lifetime of one entry point call.
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
 
 // Window kinds 0 and 1 take a radius in tiles, kind 2 a radius in tokens (window.cuh).
 bool valid_window(int kind, int radius) {
@@ -111,6 +123,7 @@ size_t bsa_workspace_bytes(const bsa_geom* g, const bsa_mask_params* p) {
 }
 
 int bsa_clear_error(void* ws, void* stream) {
+  const CallRange range("bsa_clear_error");
   if (!ws) return BSA_ERR_INVALID_ARG;
   const int dev = device_ok();
   if (dev != BSA_OK) return dev;
@@ -118,6 +131,7 @@ int bsa_clear_error(void* ws, void* stream) {
 }
 
 int bsa_reorder(const bsa_geom* g, const void* x, void* xt, void* stream) {
+  const CallRange range("bsa_reorder");
   if (!valid_geom(g) || !aligned16(x) || !aligned16(xt)) return BSA_ERR_INVALID_ARG;
   const int dev = device_ok();
   if (dev != BSA_OK) return dev;
@@ -126,6 +140,7 @@ int bsa_reorder(const bsa_geom* g, const void* x, void* xt, void* stream) {
 }
 
 int bsa_unreorder(const bsa_geom* g, const void* xt, void* x, void* stream) {
+  const CallRange range("bsa_unreorder");
   if (!valid_geom(g) || !aligned16(x) || !aligned16(xt)) return BSA_ERR_INVALID_ARG;
   const int dev = device_ok();
   if (dev != BSA_OK) return dev;
@@ -136,6 +151,7 @@ int bsa_unreorder(const bsa_geom* g, const void* xt, void* x, void* stream) {
 int bsa_build_mask(const bsa_geom* g, const bsa_mask_params* p, const void* qt, const void* kt,
                    const float* difficulty, uint32_t* mask, int32_t* kv_count, void* ws, size_t ws_bytes,
                    void* stream) {
+  const CallRange range("bsa_build_mask");
   if (!valid_geom(g) || !valid_params(g, p)) return BSA_ERR_INVALID_ARG;
   if (!aligned16(qt) || !aligned16(kt) || !aligned16(difficulty) || !aligned16(mask) || !aligned16(kv_count))
     return BSA_ERR_INVALID_ARG;
@@ -151,6 +167,7 @@ int bsa_build_mask(const bsa_geom* g, const bsa_mask_params* p, const void* qt, 
 int bsa_sparse_attn_fwd(const bsa_geom* g, const void* qt, const void* kt, const void* vt, const uint32_t* mask,
                         const int32_t* kv_count, float softmax_scale, void* out, float* lse, void* ws,
                         size_t ws_bytes, void* stream) {
+  const CallRange range("bsa_sparse_attn_fwd");
   if (!valid_geom(g)) return BSA_ERR_INVALID_ARG;
   if (!aligned16(qt) || !aligned16(kt) || !aligned16(vt) || !aligned16(mask) || !aligned16(kv_count) ||
       !aligned16(out))
@@ -170,6 +187,7 @@ int bsa_sparse_attn_fwd(const bsa_geom* g, const void* qt, const void* kt, const
 int bsa_sparse_attn_fwd_fixed_scratch(const bsa_geom* g, const void* qt, const void* kt, const void* vt,
                                       const uint32_t* mask, const int32_t* kv_count, float softmax_scale,
                                       void* out, float* lse, uint32_t* kernel_errors, void* stream) {
+  const CallRange range("bsa_sparse_attn_fwd_fixed_scratch");
   if (!valid_geom(g)) return BSA_ERR_INVALID_ARG;
   if (!aligned16(qt) || !aligned16(kt) || !aligned16(vt) || !aligned16(mask) || !aligned16(kv_count) ||
       !aligned16(out))
@@ -191,6 +209,7 @@ int bsa_sparse_attn_fwd_fixed_scratch(const bsa_geom* g, const void* qt, const v
 uint64_t bsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int bsa_selftest_bounded_wait(long long limit_cycles, uint32_t* err, void* stream) {
+  const CallRange range("bsa_selftest_bounded_wait");
   if (!err || (reinterpret_cast<uintptr_t>(err) & 3u) != 0) return BSA_ERR_INVALID_ARG;
   if (limit_cycles <= 0 || limit_cycles > 4000000000LL) return BSA_ERR_INVALID_ARG;
   const int dev = device_ok();
