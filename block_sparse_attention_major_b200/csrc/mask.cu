@@ -328,7 +328,7 @@ __device__ __forceinline__ float order_key_inverse(uint32_t k) {
 
 // TOK: the window is the token-level support (kind 2), a separate instantiation so that the
 // tile-window kinds keep their own register allocation.
-template <int MODE, int KW, int WPR, bool TOK>
+template <bool TOK>
 __device__ __forceinline__ bool sel_in_window(uint32_t ci, uint32_t cj, int kind, int r) {
   return TOK ? in_token_window(ci, cj, r) : in_tile_window(ci, cj, kind, r);
 }
@@ -405,7 +405,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
     for (int w = 0; w < KW; ++w) {
       const int j = 32 * (q * KW + w) + lane;
       const bool inrow = j < NKT;
-      const bool inw = inrow && sel_in_window<MODE, KW, WPR, TOK>(ci, coord[j], kind, rad);
+      const bool inw = inrow && sel_in_window<TOK>(ci, coord[j], kind, rad);
       const float e = inrow ? exp2f((srow[j] - mx) * c) : 0.0f;
       z += e;
       zw += inw ? e : 0.0f;
@@ -420,7 +420,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
 #pragma unroll
     for (int w = 0; w < KW; ++w) {
       const int j = 32 * (q * KW + w) + lane;
-      const bool cand = j < NKT && !sel_in_window<MODE, KW, WPR, TOK>(ci, coord[j], kind, rad);
+      const bool cand = j < NKT && !sel_in_window<TOK>(ci, coord[j], kind, rad);
       kr[w] = cand ? order_key(srow[j]) : 0u;
       ncand += __popc(__ballot_sync(0xffffffffu, cand));
     }
