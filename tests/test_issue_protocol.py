@@ -16,7 +16,9 @@ before the commit are done; nothing orders the two issuers' products against eac
 
 The protocol: S-full barriers per (sub-unit, S buffer), one P-ready and one P.V-done
 barrier per sub-unit, and a softmax that waits for the previous block's P.V before it
-releases P (and rescales O, when the row max grew). Deliberately broken variants must be
+releases P (and rescales O, when the row max grew). Each sub-unit's softmax runs as four
+independent warps, each with its own rows, so warps of one sub-unit may be at different
+blocks. Deliberately broken variants must be
 caught, which shows the checker can see the hazards: issuers that test only their own next
 entries (ring stages), a softmax that releases P without that wait, an epilogue that waits
 one block early, and QK products three blocks ahead of P.V.
@@ -30,6 +32,7 @@ import _cases as C
 from oracle import bsa_oracle as O
 
 NS = 4          # ring stages, one key tile each
+WARPS = 4       # softmax warps per sub-unit; each warp's 32 threads arrive on P-ready
 
 
 class Bar:
@@ -93,15 +96,16 @@ def run_protocol(L, need_a, need_b, seed, careless=False, no_wait=False):
     kempty = [Bar(1 if careless else users) for _ in range(NS)]
     vempty = [Bar(1 if careless else users) for _ in range(NS)]
     sfull = [Bar(1) for _ in range(4)]          # 2u + b
-    pfull = [Bar(1) for _ in range(2)]          # u
+    pfull = [Bar(WARPS) for _ in range(2)]      # u (one arrival per warp stands for its 32)
     odone = [Bar(1) for _ in range(2)]          # u
     pipe, kload, vload = [[], []], [], []     # one product queue per issuing thread
     kdata, vdata = [None] * NS, [None] * NS
-    sbuf = [[None, None], [None, None]]         # ('S', it) or ('P', it)
+    sbuf = [[[None] * WARPS for _ in range(2)] for _ in range(2)]   # per warp's rows: ('S', it) / ('P', it)
     oblocks = [0, 0]                            # P.V products absorbed by O
     prod = [0, 'k']
     ki, vi, qc, pc = [0, 0], [0, 0], [0, 0], [0, 0]
-    sm = [[0, 'wait_s'], [0, 'wait_s']]
+    # one agent per softmax warp: [block, state]; each warp owns a quarter of the rows
+    sm = [[[0, 'wait_s'] for _ in range(WARPS)] for _ in range(2)]
 
     def pbar(u, it):
         return pfull[u], it & 1
@@ -153,20 +157,21 @@ def run_protocol(L, need_a, need_b, seed, careless=False, no_wait=False):
                         bar, par = pbar(u, pc[u])
                         if bar.test(par):
                             acts.append(('pv', u))
-            it, st = sm[u]
-            if it < n[u]:
-                if st == 'wait_s' and sfull[2 * u + (it & 1)].test((it >> 1) & 1):
-                    acts.append(('softmax_s', u))
-                if st == 'wait_o':
-                    bar, par = obar(u, it - 1)
-                    if bar.test(par):
-                        acts.append(('softmax_rescale', u))
-                if st == 'release':
-                    acts.append(('softmax_p', u))
-            elif st != 'done':
-                bar, par = obar(u, n[u] - 1)
-                if n[u] == 0 or bar.test(par):
-                    acts.append(('epilogue', u))
+            for w in range(WARPS):
+                it, st = sm[u][w]
+                if it < n[u]:
+                    if st == 'wait_s' and sfull[2 * u + (it & 1)].test((it >> 1) & 1):
+                        acts.append(('softmax_s', u, w))
+                    if st == 'wait_o':
+                        bar, par = obar(u, it - 1)
+                        if bar.test(par):
+                            acts.append(('softmax_rescale', u, w))
+                    if st == 'release':
+                        acts.append(('softmax_p', u, w))
+                elif st != 'done':
+                    bar, par = obar(u, n[u] - 1)
+                    if n[u] == 0 or bar.test(par):
+                        acts.append(('epilogue', u, w))
         return acts
 
     def last_user(u, e, cursor):
@@ -175,7 +180,7 @@ def run_protocol(L, need_a, need_b, seed, careless=False, no_wait=False):
 
     while True:
         acts = actions()
-        finished = (prod[0] >= L and all(sm[u][1] == 'done' or not has[u] for u in range(2))
+        finished = (prod[0] >= L and all(sm[u][w][1] == 'done' or not has[u] for u in range(2) for w in range(WARPS))
                     and all(pc[u] >= n[u] for u in range(2)))
         if finished and not pipe[0] and not pipe[1] and not kload and not vload:
             return True
@@ -208,12 +213,12 @@ def run_protocol(L, need_a, need_b, seed, careless=False, no_wait=False):
                     raise Stale(f"QK of entry {e} read K stage {s} holding {kdata[s]}")
                 if it >= 2 and oblocks[u] < it - 1:
                     raise Stale(f"S of block {it} overwrote P of block {it - 2} before its P.V")
-                sbuf[u][it & 1] = ('S', it)
+                sbuf[u][it & 1] = [('S', it)] * WARPS
             else:
                 _, u, it, s, e = op
                 if vdata[s] != e:
                     raise Stale(f"P.V of entry {e} read V stage {s} holding {vdata[s]}")
-                if sbuf[u][it & 1] != ('P', it):
+                if sbuf[u][it & 1] != [('P', it)] * WARPS:
                     raise Stale(f"P.V of block {it} read {sbuf[u][it & 1]}")
                 if oblocks[u] != it:
                     raise Stale(f"P.V of block {it} added to O holding {oblocks[u]} blocks")
@@ -251,28 +256,28 @@ def run_protocol(L, need_a, need_b, seed, careless=False, no_wait=False):
             vempty[vi[u] % NS].arrive()
             vi[u] += 1
         elif kind == 'softmax_s':
-            u = a[1]
-            it = sm[u][0]
-            if sbuf[u][it & 1] != ('S', it):
-                raise Stale(f"softmax of block {it} read {sbuf[u][it & 1]}")
-            sm[u][1] = 'wait_o' if it > 0 and not no_wait else 'release'
+            u, w = a[1], a[2]
+            it = sm[u][w][0]
+            if sbuf[u][it & 1][w] != ('S', it):
+                raise Stale(f"softmax warp {w} of block {it} read {sbuf[u][it & 1][w]}")
+            sm[u][w][1] = 'wait_o' if it > 0 and not no_wait else 'release'
         elif kind == 'softmax_rescale':
-            u = a[1]
-            if oblocks[u] != sm[u][0]:
-                raise Stale(f"rescale at block {sm[u][0]} saw O holding {oblocks[u]} blocks")
-            sm[u][1] = 'release'
+            u, w = a[1], a[2]
+            if oblocks[u] != sm[u][w][0]:
+                raise Stale(f"rescale at block {sm[u][w][0]} saw O holding {oblocks[u]} blocks")
+            sm[u][w][1] = 'release'
         elif kind == 'softmax_p':
-            u = a[1]
-            it = sm[u][0]
-            sbuf[u][it & 1] = ('P', it)
+            u, w = a[1], a[2]
+            it = sm[u][w][0]
+            sbuf[u][it & 1][w] = ('P', it)
             bar, _ = pbar(u, it)
             bar.arrive()
-            sm[u] = [it + 1, 'wait_s']
+            sm[u][w] = [it + 1, 'wait_s']
         elif kind == 'epilogue':
-            u = a[1]
+            u, w = a[1], a[2]
             if oblocks[u] != n[u]:
                 raise Stale(f"epilogue read O holding {oblocks[u]} of {n[u]} blocks")
-            sm[u][1] = 'done'
+            sm[u][w][1] = 'done'
 
 
 def _case_units(name):
