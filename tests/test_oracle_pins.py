@@ -678,3 +678,58 @@ def test_pins_catch_planted_square_support(monkeypatch):
     monkeypatch.setattr(O, "in_token_support", square)
     with pytest.raises(AssertionError):
         test_token_support_interior_size(2, 13, 25)
+
+
+def test_pins_catch_planted_reversed_routing(monkeypatch):
+    """Routing the least difficult query tiles to dense attention must break the route pin."""
+    real = O.route_dense
+    monkeypatch.setattr(O, "route_dense", lambda d, rho: real(-np.asarray(d), rho))
+    with pytest.raises(AssertionError):
+        test_route_count_and_order(0.25)
+
+
+def test_pins_catch_planted_log2_entropy(monkeypatch):
+    """Entropy in bits instead of nats must break the scipy pin."""
+    real = O.row_entropy
+    monkeypatch.setattr(O, "row_entropy", lambda s: real(s) / math.log(2.0))
+    with pytest.raises(AssertionError):
+        test_entropy_matches_scipy()
+
+
+def test_pins_catch_planted_window_decay_off_by_one(monkeypatch):
+    """A decayed window one tile too wide (max(|dy|,|dx|) <= r - |dt| + 1) must break the
+    golden interior sizes."""
+    real = O.window
+
+    def bad_window(kind, r, T, Hs, Ws):
+        if kind != 1:
+            return real(kind, r, T, Hs, Ws)
+        c = O.tile_coords(T, Hs, Ws)
+        dt = np.abs(c[:, None, 0] - c[None, :, 0])
+        dyx = np.maximum(np.abs(c[:, None, 1] - c[None, :, 1]), np.abs(c[:, None, 2] - c[None, :, 2]))
+        return (dt <= r) & (dyx <= r - dt + 1)
+    monkeypatch.setattr(O, "window", bad_window)
+    with pytest.raises(AssertionError):
+        test_window_interior_size(1, 2, 45)
+
+
+def test_pins_catch_planted_topk_inside_window(monkeypatch):
+    """Taking the top-k over every key tile (window tiles included) must break the row-size
+    invariant |row| = |window| + min(k, outside)."""
+    real = O.top_outside
+    monkeypatch.setattr(O, "top_outside", lambda s, excluded, m: real(s, np.zeros_like(excluded), m))
+    with pytest.raises(AssertionError):
+        test_dense_rows_and_mask_invariants()
+
+
+def test_pins_catch_planted_scale(monkeypatch):
+    """Scaling scores by 1/d instead of 1/sqrt(d) must break the dense SDPA pin."""
+    real = O.attention_tiles
+
+    def bad(qt, kt, vt, mask, rows, **kw):
+        if kw.get("scale") is None:
+            kw["scale"] = 1.0 / qt.shape[-1]
+        return real(qt, kt, vt, mask, rows, **kw)
+    monkeypatch.setattr(O, "attention_tiles", bad)
+    with pytest.raises(AssertionError):
+        test_all_retained_equals_dense_sdpa((4, 8, 8))
