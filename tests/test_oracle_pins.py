@@ -287,6 +287,163 @@ def test_radius_for_budget_brute(grid):
         assert sizes[r + 1] > b or sizes[r] == NT
 
 
+def _decayed_window_by_loops(i, r, T, Hs, Ws):
+    """Decayed window of query tile i (|dt| <= r, max(|dy|, |dx|) <= r - |dt|, clipped at the
+    grid edges), written out with loops over tile coordinates."""
+    nT, nY, nX = O.tile_grid(T, Hs, Ws)
+    ti, yi, xi = i // (nY * nX), (i // nX) % nY, i % nX
+    out = set()
+    for tt in range(nT):
+        for ty in range(nY):
+            for tx in range(nX):
+                dt = abs(tt - ti)
+                if dt <= r and max(abs(ty - yi), abs(tx - xi)) <= r - dt:
+                    out.add((tt * nY + ty) * nX + tx)
+    return out
+
+
+def _budget_row_by_definition(b, i, T, Hs, Ws, order_key):
+    """The budget-mode row of query tile i written from the definition (Token Radius
+    Attention, "Radius construction" and "Entropy-guided budgeting"): the radius grows from
+    0 while the next decayed window still fits the budget b (stopping once the window covers
+    the grid); the window is then topped up to b tiles with the best tiles outside it, in
+    the order given by order_key (best first)."""
+    NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
+    r = 0
+    while len(_decayed_window_by_loops(i, r, T, Hs, Ws)) < NT and \
+            len(_decayed_window_by_loops(i, r + 1, T, Hs, Ws)) <= b:
+        r += 1
+    win = _decayed_window_by_loops(i, r, T, Hs, Ws)
+    outside = sorted((j for j in range(NT) if j not in win), key=order_key)
+    return win | set(outside[:b - len(win)]), r
+
+
+def test_budget_rows_planted_composition():
+    """Entropy-budget rows under planted scores: which tiles a row holds, not only how many.
+
+    qbar_i = a_i * e1 with a_i spread over a decade, kbar_j = c * (j + 1) * e1: every row ranks
+    the key tiles by index (highest first), while its entropy, hence its budget b_i, varies
+    with a_i. Each row must equal the decayed window of the largest radius that fits b_i,
+    topped up with the highest-indexed tiles outside that window."""
+    T, Hs, Ws, d = 12, 16, 20, 4
+    NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
+    e1 = np.zeros(d); e1[0] = 1.0
+    valid = O.slot_valid(T, Hs, Ws)
+    alphas = np.geomspace(0.2, 4.0, NT)[np.random.default_rng(31).permutation(NT)]
+    qt = np.zeros((1, 1, NT, 64, d))
+    kt = np.zeros((1, 1, NT, 64, d))
+    for j in range(NT):
+        qt[0, 0, j, valid[j]] = alphas[j] * e1
+        kt[0, 0, j, valid[j]] = 0.05 * (j + 1) * e1
+    res = O.build_mask(qt, kt, np.zeros((1, NT), np.float32), T=T, Hs=Hs, Ws=Ws,
+                       window_kind=1, radius=0, topk=0, dense_fraction=0.0,
+                       budget_mode=1, budget_target=0.19)
+    budgets = res["budget"][0, 0]
+    radii, extras = set(), 0
+    for i in range(NT):
+        expect, r = _budget_row_by_definition(int(budgets[i]), i, T, Hs, Ws, lambda j: -j)
+        assert set(np.nonzero(res["mask"][0, 0, i])[0]) == expect, i
+        assert res["count"][0, 0, i] == budgets[i]
+        radii.add(r)
+        extras += int(budgets[i]) - len(_decayed_window_by_loops(i, r, T, Hs, Ws))
+    # the case is not degenerate: several budgets and radii, and rows with top-up tiles
+    assert len(set(budgets.tolist())) >= 5 and len(radii) >= 2 and extras > 0
+
+
+def test_budget_rows_dominant_tile_outside_window():
+    """Uniform kbar except one dominant key tile: every row holds its decayed window, that
+    tile, and then the lowest-indexed tiles outside the window (ties to the lower index)."""
+    T, Hs, Ws, d = 12, 16, 20, 4
+    NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
+    e1 = np.zeros(d); e1[0] = 1.0
+    star = 37
+    kvals = [e1 * (6.0 if j == star else 1.0) for j in range(NT)]
+    qt, kt = _planted(T, Hs, Ws, 1, d, kvals, e1)
+    res = O.build_mask(qt, kt, np.zeros((1, NT), np.float32), T=T, Hs=Hs, Ws=Ws,
+                       window_kind=1, radius=0, topk=0, dense_fraction=0.0,
+                       budget_mode=1, budget_target=0.3)
+    b = int(res["budget"][0, 0, 0])
+    assert np.all(res["budget"][0, 0] == b) and b == 18        # equal entropies: round(0.3 * 60)
+    n_star_outside = 0
+    for i in range(NT):
+        expect, r = _budget_row_by_definition(b, i, T, Hs, Ws, lambda j: (j != star, j))
+        got = set(np.nonzero(res["mask"][0, 0, i])[0])
+        assert got == expect, i
+        n_star_outside += star not in _decayed_window_by_loops(i, r, T, Hs, Ws)
+    assert n_star_outside > NT // 2
+
+
+# ------------------------------------------------------------------------------ near-tie band
+# Mask disagreements are allowed only where score gaps are below 1e-4 relative (the
+# benchmark's tolerance statement); the pins use that number, not the oracle's constant.
+BAND = 1e-4
+
+
+def test_near_tie_flag_both_sides_of_band():
+    """The boundary gap is judged against 1e-4 of the row's largest |score|: a gap of half
+    that band is flagged, a gap of twice the band is not."""
+    scale = 10.0
+    base = np.array([scale, 9.0, 8.0, 0.0, 1.0, -3.0, 0.5, 2.0])
+    excluded = np.zeros(base.size, dtype=bool)
+    for frac, flagged in ((0.5, True), (0.99, True), (1.01, False), (2.0, False)):
+        s = base.copy()
+        s[3] = 8.0 - frac * BAND * scale        # the 4th best, just below the 3rd
+        assert O.boundary_near_tie(s, excluded, 3) == flagged, frac
+    # the band is relative to the row's scale, not to the scores at the boundary
+    s = base.copy() * 1e3
+    s[3] = s[2] - 0.5e-4 * np.abs(s).max()
+    assert O.boundary_near_tie(s, excluded, 3)
+    s[3] = s[2] - 2e-4 * np.abs(s).max()
+    assert not O.boundary_near_tie(s, excluded, 3)
+    # an excluded (window) tile never takes part in the boundary
+    s = base.copy()
+    s[3] = 8.0 - 0.5 * BAND * scale
+    ex = excluded.copy(); ex[3] = True
+    assert not O.boundary_near_tie(s, ex, 3)
+
+
+@pytest.mark.parametrize("gap_in_bands,flagged", [(0.5, True), (2.0, False)])
+def test_near_tie_flag_through_build_mask(gap_in_bands, flagged):
+    """Fixed top-k rows under planted scores: the k-th and (k+1)-th best tiles outside the
+    window differ by gap_in_bands times the band; rows are flagged exactly when that gap is
+    inside the band."""
+    T, Hs, Ws, d, k = 8, 16, 16, 4, 2
+    NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
+    e1 = np.zeros(d); e1[0] = 1.0
+    top, second, third = NT - 1, NT - 2, NT - 3       # the graded order puts these first
+    vals = [0.01 * (j + 1) for j in range(NT)]
+    smax = vals[top]
+    vals[third] = vals[second] - gap_in_bands * BAND * smax
+    qt, kt = _planted(T, Hs, Ws, 1, d, [v * e1 for v in vals], e1)
+    res = O.build_mask(qt, kt, np.zeros((1, NT), np.float32), T=T, Hs=Hs, Ws=Ws,
+                       window_kind=0, radius=0, topk=k, dense_fraction=0.0)
+    for i in range(NT):
+        if i in (top, second, third):
+            continue                                   # the window removes one of the three
+        assert set(np.nonzero(res["mask"][0, 0, i])[0]) == {i, top, second}
+        assert res["near_tie"][0, 0, i] == flagged, i
+
+
+@pytest.mark.parametrize("offset_in_bands,flagged", [(0.5, True), (2.0, False)])
+def test_budget_half_integer_flag_both_sides(offset_in_bands, flagged):
+    """Budget mode: a pre-rounding budget within 1e-4*max(x, 1) of a half-integer is flagged,
+    one twice that band away is not. Equal rows (the same qbar for every query tile) make
+    every pre-rounding budget tau*NKT; the graded kbar keeps the score gaps far from their
+    own band."""
+    T, Hs, Ws, d = 8, 16, 16, 4
+    NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
+    e1 = np.zeros(d); e1[0] = 1.0
+    qt, kt = _planted(T, Hs, Ws, 1, d, [0.02 * (j + 1) * e1 for j in range(NT)], e1)
+    x0 = 6.5
+    tau = (x0 + offset_in_bands * BAND * x0) / NT
+    res = O.build_mask(qt, kt, np.zeros((1, NT), np.float32), T=T, Hs=Hs, Ws=Ws,
+                       window_kind=1, radius=0, topk=0, dense_fraction=0.0,
+                       budget_mode=1, budget_target=tau)
+    np.testing.assert_allclose(res["budget_x"][0, 0], float(np.float32(tau)) * NT, rtol=1e-12)
+    assert np.all(res["budget"][0, 0] == 7)
+    assert np.all(res["near_tie"][0, 0] == flagged)
+
+
 # ------------------------------------------------------------------------------ bitmask
 def test_bitmask_layout():
     m = np.zeros((2, 70), dtype=bool)
@@ -733,3 +890,35 @@ def test_pins_catch_planted_scale(monkeypatch):
     monkeypatch.setattr(O, "attention_tiles", bad)
     with pytest.raises(AssertionError):
         test_all_retained_equals_dense_sdpa((4, 8, 8))
+
+
+def test_pins_catch_planted_budget_topk_over_whole_row(monkeypatch):
+    """Budget mode taking the top b_i tiles over the whole row (window tiles competing with
+    the rest) instead of topping the window up from outside it must break the composition
+    pin."""
+    real = O.top_outside
+    monkeypatch.setattr(O, "top_outside",
+                        lambda s, excluded, m: real(s, np.zeros_like(excluded), m + int(excluded.sum())))
+    with pytest.raises(AssertionError):
+        test_budget_rows_planted_composition()
+
+
+def test_pins_catch_planted_budget_radius_one_short(monkeypatch):
+    """A radius one below the largest that fits the budget (more tiles by score, fewer by
+    distance) must break the composition pin."""
+    real = O.radius_for_budget
+    monkeypatch.setattr(O, "radius_for_budget", lambda b, i, T, Hs, Ws: max(real(b, i, T, Hs, Ws) - 1, 0))
+    with pytest.raises(AssertionError):
+        test_budget_rows_planted_composition()
+
+
+@pytest.mark.parametrize("band,case", [(1e-3, (2.0, False)), (1e-5, (0.5, True))])
+def test_pins_catch_planted_near_tie_band(monkeypatch, band, case):
+    """A near-tie band ten times too wide (it would excuse real mask disagreements) or ten
+    times too narrow (it would fail rows that float32 may decide either way) must break the
+    two-sided band pins."""
+    monkeypatch.setattr(O, "NEAR_TIE_REL", band)
+    with pytest.raises(AssertionError):
+        test_near_tie_flag_through_build_mask(*case)
+    with pytest.raises(AssertionError):
+        test_budget_half_integer_flag_both_sides(*case)
