@@ -15,6 +15,13 @@ from oracle import bsa_oracle as O
 O_REL_L2 = 5e-3
 O_MAX_ABS = 2e-2
 LSE_ABS = 1e-3
+# The output is bf16, so where half a bf16 ulp of |O| reaches the max-abs bound (|O| >= 8)
+# no bf16 result can meet it literally. Per element the bound is therefore
+#   max(O_MAX_ABS, half_ulp_bf16(O) + O_PRE_ROUNDING)
+# with O_PRE_ROUNDING = 2e-2 - 2^-6: the computation error that the literal bound leaves
+# at the top of its attainable range (|O| just below 8, half an ulp 2^-6). Every element
+# with |O| < 8 is held to the literal 2e-2.
+O_PRE_ROUNDING = O_MAX_ABS - 2.0 ** -6
 
 SMALL_D128 = {
     "small128": Workload("small128", B=1, H=2, d=128, T=8, Hs=16, Ws=16, seed=1010,
@@ -96,21 +103,34 @@ def compare_masks(gpu: np.ndarray, ref: dict) -> dict:
                 diff_rows=diff_rows)
 
 
-def compare_attention(w: Workload, out: torch.Tensor, lse: torch.Tensor | None, ref: dict,
-                      skip_rows: np.ndarray | None = None) -> dict:
-    """GPU out [B,N,H,d] / lse [B,H,N] against oracle per-tile results {(b,h,i): entry}."""
+def max_abs_bound(want: np.ndarray) -> np.ndarray:
+    """Per-element max-abs bound (see O_PRE_ROUNDING)."""
+    return np.maximum(O_MAX_ABS, bf16_half_ulp(want) + O_PRE_ROUNDING)
+
+
+def mask_for_reference(oracle_mask: np.ndarray, gpu_mask: np.ndarray, diff_rows: np.ndarray) -> np.ndarray:
+    """The mask the oracle attends through: its own rows, except rows where the GPU's mask
+    differs (allowed only at flagged near-ties), which take the GPU's row so that those rows
+    are still checked, against the oracle run under the GPU's own mask."""
+    return np.where(diff_rows[..., None], gpu_mask, oracle_mask)
+
+
+def compare_attention(w: Workload, out: torch.Tensor, lse: torch.Tensor | None, ref: dict) -> dict:
+    """GPU out [B,N,H,d] / lse [B,H,N] against oracle per-tile results {(b,h,i): entry}.
+
+    Reports the raw max abs error, the |O| where it occurs, and the largest ratio of an
+    element's error to its bound (max_abs_bound); the assertion is on that ratio."""
     src = O.slot_tokens(w.T, w.Hs, w.Ws)
     out64 = out.float().cpu().numpy().astype(np.float64)
     lse64 = lse.cpu().numpy().astype(np.float64) if lse is not None else None
     num = den = 0.0
     max_abs = 0.0
-    max_excess = 0.0
+    at_abs = 0.0
+    worst_ratio = 0.0
     max_lse = 0.0
     worst_tile = 0.0
     compared = 0
     for (b, h, i), e in ref.items():
-        if skip_rows is not None and skip_rows[b, h, i]:
-            continue
         toks = src[i][e["valid"]]
         got = out64[b, toks, h, :]
         want = e["o"][e["valid"]]
@@ -119,19 +139,22 @@ def compare_attention(w: Workload, out: torch.Tensor, lse: torch.Tensor | None, 
         num += dn
         den += dd
         worst_tile = max(worst_tile, math.sqrt(dn / max(dd, 1e-300)))
-        max_abs = max(max_abs, float(np.abs(got - want).max()))
-        max_excess = max(max_excess, float((np.abs(got - want) - bf16_half_ulp(want)).max()))
+        err = np.abs(got - want)
+        k = np.unravel_index(int(np.argmax(err)), err.shape)
+        if err[k] > max_abs:
+            max_abs, at_abs = float(err[k]), float(abs(want[k]))
+        worst_ratio = max(worst_ratio, float((err / max_abs_bound(want)).max()))
         if lse64 is not None:
             max_lse = max(max_lse, float(np.abs(lse64[b, h, toks] - e["lse"][e["valid"]]).max()))
         compared += 1
     return dict(rel_l2=math.sqrt(num / max(den, 1e-300)), worst_tile_rel_l2=worst_tile,
-                max_abs=max_abs, max_abs_beyond_output_rounding=max_excess, max_lse=max_lse,
-                tiles=compared)
+                max_abs=max_abs, max_abs_at_abs_o=at_abs, max_abs_over_bound=worst_ratio,
+                max_lse=max_lse, tiles=compared)
 
 
 def assert_attention_close(stats: dict) -> None:
     assert stats["tiles"] > 0
     assert stats["rel_l2"] <= O_REL_L2, stats
     assert stats["worst_tile_rel_l2"] <= O_REL_L2, stats
-    assert stats["max_abs_beyond_output_rounding"] <= O_MAX_ABS, stats
+    assert stats["max_abs_over_bound"] <= 1.0, stats
     assert stats["max_lse"] <= LSE_ABS, stats

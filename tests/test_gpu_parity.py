@@ -89,12 +89,14 @@ def test_mask_wan5b_rho_sweep(rho):
     w, g, gm, ref, cmp, _, _ = _mask_case("wan5b", heads=[0, 11, 23],
                                           overrides=(("dense_fraction", rho),))
     assert cmp["n_unflagged"] == 0, cmp
+    assert cmp["n_diff"] <= max(1, cmp["n_rows"] // 200), cmp
     assert ref["dense"].sum() == O.n_dense(rho, g.NT)
 
 
 def test_mask_wan14b_heads():
     w, g, gm, ref, cmp, _, _ = _mask_case("wan14b", heads=[0, 39])
     assert cmp["n_unflagged"] == 0, cmp
+    assert cmp["n_diff"] <= max(1, cmp["n_rows"] // 200), cmp
 
 
 @pytest.mark.parametrize("theta", [0.3, 0.7])
@@ -112,6 +114,7 @@ def test_mask_hunyuan_budget_heads(tau):
     w, g, gm, ref, cmp, _, _ = _mask_case("hunyuan", heads=[0, 23],
                                           overrides=(("budget_target", tau),))
     assert cmp["n_unflagged"] == 0, cmp
+    assert cmp["n_diff"] <= max(1, cmp["n_rows"] // 200), cmp
     retained = gm.mean()
     assert abs(retained - tau) < 0.05, retained
 
@@ -194,8 +197,8 @@ def test_attention_all_retained_equals_dense():
     ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv).permute(0, 2, 1, 3)
     got = out.double().cpu()
     rel = ((got - ref).norm() / ref.norm()).item()
-    excess = (got - ref).abs().numpy() - C.bf16_half_ulp(ref.numpy())
-    assert rel <= C.O_REL_L2 and excess.max() <= C.O_MAX_ABS
+    ratio = (got - ref).abs().numpy() / C.max_abs_bound(ref.numpy())
+    assert rel <= C.O_REL_L2 and ratio.max() <= 1.0, (rel, ratio.max())
     s = torch.einsum("bhnd,bhmd->bhnm", tq, tk) / np.sqrt(w.d)
     assert (lse.double().cpu() - torch.logsumexp(s, -1)).abs().max().item() <= C.LSE_ABS
 
@@ -280,15 +283,18 @@ def test_forward_path(name):
     assert bsa.read_error(b.ws) == 0
     qt64, kt64, vt64 = (O.reorder(O.to_f64(x), w.T, w.Hs, w.Ws) for x in (q, k, v))
     mref = C.oracle_mask(w, qt64, kt64, diff.numpy())
-    cmp = C.compare_masks(C.gpu_mask_bool(b.mask, g.NT), mref)
+    gm = C.gpu_mask_bool(b.mask, g.NT)
+    cmp = C.compare_masks(gm, mref)
     assert cmp["n_unflagged"] == 0, cmp
     if name == "wan13b":
         rng = np.random.default_rng(11)
         rows = [(0, int(rng.integers(w.H)), int(rng.integers(g.NT))) for _ in range(20)]
     else:
         rows = [(bb, h, i) for bb in range(w.B) for h in range(w.H) for i in range(g.NT)]
-    ref = O.attention_tiles(qt64, kt64, vt64, mref["mask"], rows, T=w.T, Hs=w.Hs, Ws=w.Ws)
-    st = C.compare_attention(w, b.out, b.lse, ref, skip_rows=cmp["diff_rows"])
+    rows += [tuple(int(x) for x in r) for r in np.argwhere(cmp["diff_rows"])][:8]
+    used = C.mask_for_reference(mref["mask"], gm, cmp["diff_rows"])
+    ref = O.attention_tiles(qt64, kt64, vt64, used, rows, T=w.T, Hs=w.Hs, Ws=w.Ws)
+    st = C.compare_attention(w, b.out, b.lse, ref)
     print(name, st, cmp["n_diff"])
     C.assert_attention_close(st)
 
@@ -324,13 +330,17 @@ def test_forward_path_max_tiles():
     assert bsa.read_error(b.ws) == 0
     qt64, kt64, vt64 = (O.reorder(O.to_f64(x), w.T, w.Hs, w.Ws) for x in (q, k, v))
     mref = C.oracle_mask(w, qt64, kt64, diff.numpy())
-    cmp = C.compare_masks(C.gpu_mask_bool(b.mask, g.NT), mref)
+    gm = C.gpu_mask_bool(b.mask, g.NT)
+    cmp = C.compare_masks(gm, mref)
     assert cmp["n_unflagged"] == 0, cmp
+    assert cmp["n_diff"] <= max(1, cmp["n_rows"] // 200), cmp
     rng = np.random.default_rng(17)
     dense_rows = np.nonzero(mref["dense"][0])[0]
     rows = [(0, 0, int(i)) for i in rng.integers(g.NT, size=12)] + [(0, 0, int(dense_rows[0]))]
-    ref = O.attention_tiles(qt64, kt64, vt64, mref["mask"], rows, T=w.T, Hs=w.Hs, Ws=w.Ws)
-    st = C.compare_attention(w, b.out, b.lse, ref, skip_rows=cmp["diff_rows"])
+    rows += [tuple(int(x) for x in r) for r in np.argwhere(cmp["diff_rows"])][:4]
+    used = C.mask_for_reference(mref["mask"], gm, cmp["diff_rows"])
+    ref = O.attention_tiles(qt64, kt64, vt64, used, rows, T=w.T, Hs=w.Hs, Ws=w.Ws)
+    st = C.compare_attention(w, b.out, b.lse, ref)
     C.assert_attention_close(st)
 
 
@@ -349,14 +359,15 @@ def test_forward_path_full_size(name, overrides):
     gm = C.gpu_mask_bool(b.mask, g.NT)[:, heads]
     cmp = C.compare_masks(gm, mref)
     assert cmp["n_unflagged"] == 0, cmp
+    assert cmp["n_diff"] <= max(1, cmp["n_rows"] // 200), cmp
     rng = np.random.default_rng(23)
     rows = [(0, int(rng.integers(2)), int(rng.integers(g.NT))) for _ in range(10)]
-    ref = O.attention_tiles(qt64, kt64, vt64, mref["mask"], rows, T=w.T, Hs=w.Hs, Ws=w.Ws)
+    rows += [tuple(int(x) for x in r) for r in np.argwhere(cmp["diff_rows"])][:4]
+    used = C.mask_for_reference(mref["mask"], gm, cmp["diff_rows"])
+    ref = O.attention_tiles(qt64, kt64, vt64, used, rows, T=w.T, Hs=w.Hs, Ws=w.Ws)
     # map the oracle's head slots back to the call's heads
     ref = {(bb, heads[h], i): e for (bb, h, i), e in ref.items()}
-    skip = np.zeros((w.B, w.H, g.NT), dtype=bool)
-    skip[:, heads] = cmp["diff_rows"]
-    st = C.compare_attention(w, b.out, b.lse, ref, skip_rows=skip)
+    st = C.compare_attention(w, b.out, b.lse, ref)
     print(name, st, cmp["n_diff"], "retained", float(gm.mean()))
     C.assert_attention_close(st)
 
@@ -398,11 +409,13 @@ def test_forward_mask_reuse():
     assert bsa.read_error(b.ws) == 0
     qa64, ka64 = (O.reorder(O.to_f64(x), wa.T, wa.Hs, wa.Ws) for x in (qa, ka))
     mref = C.oracle_mask(wa, qa64, ka64, da.numpy())
-    cmp = C.compare_masks(C.gpu_mask_bool(mask_a, g.NT), mref)
+    gm = C.gpu_mask_bool(mask_a, g.NT)
+    cmp = C.compare_masks(gm, mref)
     assert cmp["n_unflagged"] == 0, cmp
     qb64, kb64, vb64 = (O.reorder(O.to_f64(x), wb.T, wb.Hs, wb.Ws) for x in (qb, kb, vb))
     rows = [(bb, h, i) for bb in range(wb.B) for h in range(wb.H) for i in range(g.NT)]
-    ref = O.attention_tiles(qb64, kb64, vb64, mref["mask"], rows, T=wb.T, Hs=wb.Hs, Ws=wb.Ws)
-    st = C.compare_attention(wb, b.out, b.lse, ref, skip_rows=cmp["diff_rows"])
+    used = C.mask_for_reference(mref["mask"], gm, cmp["diff_rows"])
+    ref = O.attention_tiles(qb64, kb64, vb64, used, rows, T=wb.T, Hs=wb.Hs, Ws=wb.Ws)
+    st = C.compare_attention(wb, b.out, b.lse, ref)
     print(st)
     C.assert_attention_close(st)
