@@ -1,13 +1,17 @@
 """Benchmark of the block-sparse video attention path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload hunyuan|wan13b|wan14b|...] [--report [--only PREFIX]]
 
-One step = one pass of the whole path over one attention call of the Wan-1.3B-480p-shaped
-workload (B=1, 12 heads, d=128, 21x30x52 latent grid = 32,760 tokens, 20% of query tiles
-dense, the rest a decayed window of radius 2 plus the top-8 key tiles): reorder Q, K, V
-to tile-major, build the block mask, block-sparse attention with the output and LSE
-written back in raster order. Inputs are synthetic (seeded generator) and resident in HBM
-(302 MB of raster Q/K/V, larger than the 126 MB L2) when the timed region starts.
+One step = one pass of the whole path over one attention call of the HunyuanVideo-720p-
+shaped workload (B=1, 24 heads, d=128, 33x45x80 latent grid = 118,800 tokens in 2160 tiles;
+every (head, query tile) keeps a budget of key tiles proportional to exp(entropy) of its
+pooled-score softmax, normalised to 19% of all tile pairs, as the decayed window of the
+largest radius that fits the budget topped up by pooled score): reorder Q, K, V to
+tile-major, build the block mask, block-sparse attention with the output and LSE written
+back in raster order. It is the largest of the benchmark's single-GPU calls at about 20%
+retained tiles. Inputs are synthetic (seeded generator) and resident in HBM (2.2 GB of
+raster Q/K/V, larger than the 126 MB L2) when the timed region starts.
 
 The metric is effective TFLOP/s: 4*64*64*d FLOPs per retained (query tile, key tile) pair,
 divided by the device time of the step; `ms_per_step` gives the time per call.
@@ -32,7 +36,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-WORKLOAD = "wan13b"
+WORKLOAD = "hunyuan"          # default; --workload picks another benchmark call
 METRIC = "sparse-attn ms/call & effective TFLOP/s at ~20% tiles; % of B200 BF16 peak"
 NOMINAL_BF16_TFLOPS = 2250.0
 
@@ -43,6 +47,8 @@ def _args():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="benchmark call of the step (hunyuan: tau = 0.19; wan13b, wan14b, wan5b, tiny)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--report", action="store_true",
@@ -109,16 +115,33 @@ def _mask_bytes(g):
     return 2 * g.B * g.N * g.H * g.d * 2 + g.B * g.H * g.NT * (g.NW + 1) * 4
 
 
+def _workload_text(w):
+    grid = (f"B={w.B} heads={w.H} d={w.d} grid {w.T}x{w.Hs}x{w.Ws} ({w.N} tokens, "
+            f"{w.NT} tiles of 4x4x4)")
+    names = {"hunyuan": "HunyuanVideo-720p-shaped", "wan13b": "Wan-1.3B-480p-shaped",
+             "wan14b": "Wan-14B-720p-shaped", "wan5b": "Wan2.2-5B-shaped", "tiny": "Tiny"}
+    kinds = {0: "cube window", 1: "decayed window", 2: "token-level circular window"}
+    if w.budget_mode == 1:
+        rule = (f"entropy budget tau={w.budget_target} of key tiles per (head, query tile): "
+                "decayed window of the largest radius that fits the budget, topped up by "
+                "pooled score")
+    elif w.budget_mode == 2:
+        rule = (f"rho={w.dense_fraction} dense query tiles, {kinds[w.window_kind]} "
+                f"r={w.radius} + tiles up to pooled mass theta={w.budget_target}")
+    else:
+        rule = (f"rho={w.dense_fraction} dense query tiles, {kinds[w.window_kind]} "
+                f"r={w.radius} + top-{w.topk}")
+    return f"{names.get(w.name, w.name)} attention call: {grid}, {rule}"
+
+
 def _workload_desc(w, retention):
+    raster_mb = 3 * w.B * w.N * w.H * w.d * 2 / 1e6
     return {
-        "workload": (f"Wan-1.3B-480p-shaped attention call: B={w.B} heads={w.H} d={w.d} "
-                     f"grid {w.T}x{w.Hs}x{w.Ws} ({w.N} tokens, {w.NT} tiles of 4x4x4), "
-                     f"rho={w.dense_fraction} dense query tiles, decayed window r={w.radius} "
-                     f"+ top-{w.topk}"),
+        "workload": _workload_text(w),
         "global_batch": w.B,
         "seq_len": w.N,
         "retained_tile_fraction": round(retention, 4),
-        "l2": "inputs larger than L2 (raster Q/K/V 302 MB > 126 MB)",
+        "l2": f"inputs larger than L2 (raster Q/K/V {raster_mb:.0f} MB > 126 MB)",
         "parallelism": "independent call per rank (weak scaling)",
     }
 
@@ -186,11 +209,12 @@ def _attn_source_hash():
     return h.hexdigest()[:16]
 
 
-def _traffic():
-    """DRAM bytes per attention launch from the committed ncu summary, if it is current."""
-    p = os.path.join(ROOT, "profiles", "attn_kernel_wan13b_traffic.json")
+def _traffic(workload):
+    """DRAM bytes per attention launch from the committed ncu summary of this workload, if
+    it is current."""
+    p = os.path.join(ROOT, "profiles", f"attn_kernel_{workload}_traffic.json")
     if not os.path.exists(p):
-        return None, None
+        return None, "no ncu capture of this workload's attention launch"
     with open(p) as f:
         d = json.load(f)
     if d.get("attn_source_sha256_16") != _attn_source_hash():
@@ -199,10 +223,14 @@ def _traffic():
 
 
 # ------------------------------------------------------------------------------ CPU oracle
-def _oracle_sample(w, q, k, v, diff, head, rows):
-    """Oracle path for one head: reorder, mask, attention of the listed query tiles.
+def _oracle_sample(w, q, k, v, diff, head, n_rows, seconds):
+    """Oracle path for one head, bounded in time: reorder and mask of the head (all its query
+    tiles), then attention of seeded-shuffled query tiles of the head until `seconds` of
+    attention have been spent (at least n_rows tiles).
 
-    Returns (seconds, retained tile pairs attended)."""
+    Returns (seconds charged, retained tile pairs attended, rows attended, setup seconds):
+    the attention time plus the setup time in proportion to the head's retained pairs that
+    were attended, so that attending every row would charge the whole setup."""
     import numpy as np
     from oracle import bsa_oracle as O
     t0 = time.perf_counter()
@@ -211,10 +239,18 @@ def _oracle_sample(w, q, k, v, diff, head, rows):
     m = O.build_mask(qt, kt, diff.numpy(), T=w.T, Hs=w.Hs, Ws=w.Ws, window_kind=w.window_kind,
                      radius=w.radius, topk=w.topk, dense_fraction=w.dense_fraction,
                      budget_mode=w.budget_mode, budget_target=w.budget_target)
-    O.attention_tiles(qt, kt, vt, m["mask"], [(0, 0, i) for i in rows], T=w.T, Hs=w.Hs, Ws=w.Ws)
-    dt = time.perf_counter() - t0
-    pairs = int(sum(int(m["mask"][0, 0, i].sum()) for i in rows))
-    return dt, pairs
+    t_setup = time.perf_counter() - t0
+    counts = m["mask"][0, 0].sum(-1)
+    order = np.random.default_rng(7).permutation(w.NT)
+    t_attn, pairs, n = 0.0, 0, 0
+    while n < w.NT and (n < n_rows or t_attn < seconds):
+        i = int(order[n])
+        t1 = time.perf_counter()
+        O.attention_tiles(qt, kt, vt, m["mask"], [(0, 0, i)], T=w.T, Hs=w.Hs, Ws=w.Ws)
+        t_attn += time.perf_counter() - t1
+        pairs += int(counts[i])
+        n += 1
+    return t_attn + t_setup * pairs / int(counts.sum()), pairs, n, t_setup
 
 
 def _blas_threads():
@@ -229,11 +265,12 @@ def _blas_threads():
 def run_reference(args):
     """Oracle timed on the host cores, rank 0 only.
 
-    Setup (timed once): reorder of Q, K, V and the mask of the whole call. Each step then
-    attends a chunk of query tiles (a seeded shuffle of every (head, tile) row), taking rows
-    until the step's time budget of about 120 s / (steps + warmup) is used. A step is
-    charged its attention time plus the setup time in proportion to the retained tile
-    pairs it attended, so that the sum over all rows of the call would be the full call.
+    Setup (timed once): reorder of Q, K, V and the mask of head 0 of the call (the oracle's
+    mask construction loops over every row in Python; one head keeps the run to minutes).
+    Each step then attends a chunk of head 0's query tiles (a seeded shuffle), taking rows
+    until the step's time budget of about 120 s / (steps + warmup) is used. A step is charged
+    its attention time plus the setup time in proportion to the retained tile pairs it
+    attended, so that attending every row of the head would charge the whole setup.
     """
     rank, world, _ = _dist_env()
     if rank != 0:
@@ -241,19 +278,19 @@ def run_reference(args):
     import numpy as np
     from bsa_synth import WORKLOADS, generate_difficulty, generate_qkv
     from oracle import bsa_oracle as O
-    w = WORKLOADS[WORKLOAD]
+    w = WORKLOADS[args.workload]
     q, k, v = generate_qkv(w)
     diff = generate_difficulty(w)
     t0 = time.perf_counter()
-    qt, kt, vt = (O.reorder(O.to_f64(x), w.T, w.Hs, w.Ws) for x in (q, k, v))
+    qt, kt, vt = (O.reorder(O.to_f64(x[:, :, :1]), w.T, w.Hs, w.Ws) for x in (q, k, v))
     m = O.build_mask(qt, kt, diff.numpy(), T=w.T, Hs=w.Hs, Ws=w.Ws, window_kind=w.window_kind,
                      radius=w.radius, topk=w.topk, dense_fraction=w.dense_fraction,
                      budget_mode=w.budget_mode, budget_target=w.budget_target)
     t_setup = time.perf_counter() - t0
     counts = m["mask"].sum(-1)
-    pairs_call = int(counts.sum())
+    pairs_head = int(counts.sum())
     flop_pair = 4 * 64 * 64 * w.d
-    rows = [(0, h, i) for h in range(w.H) for i in range(w.NT)]
+    rows = [(0, 0, i) for i in range(w.NT)]
     order = np.random.default_rng(7).permutation(len(rows))
     budget = min(5.0, max(0.05, 120.0 / (args.steps + args.warmup)))
     cursor = 0
@@ -268,20 +305,20 @@ def run_reference(args):
             t_attn += time.perf_counter() - t1
             pairs += int(counts[b, h, i])
         if s >= args.warmup:
-            times.append(t_attn + t_setup * pairs / pairs_call)
+            times.append(t_attn + t_setup * pairs / pairs_head)
             flops.append(pairs * flop_pair)
     total_t = sum(times)
     value = sum(flops) / total_t / 1e12
     ms = 1e3 * total_t / len(times)
-    sample = (f"oracle on the whole call's reorder + mask ({t_setup:.1f} s, charged to the steps "
-              f"by retained pairs) and, per step, attention of seeded-shuffled (head, query "
-              f"tile) rows for about {budget:.2f} s; value = FLOPs of the attended retained "
-              "tile pairs / charged time")
+    sample = (f"oracle on head 0 of {w.H}: reorder + mask ({t_setup:.1f} s, charged to the steps "
+              f"by retained pairs) and, per step, attention of seeded-shuffled query tiles of "
+              f"head 0 for about {budget:.2f} s; value = FLOPs of the attended retained tile "
+              "pairs / charged time")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": _workload_desc(w, pairs_call / counts.size / w.NT),
+        "data": "synthetic", "config": _workload_desc(w, pairs_head / counts.size / w.NT),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _blas_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -320,7 +357,7 @@ def run_ours(args):
     def sum_over_ranks(x: float) -> float:
         return reduce_scalar(x, "sum", world, dev)
 
-    w = WORKLOADS[WORKLOAD]
+    w = WORKLOADS[args.workload]
     q_h, k_h, v_h = generate_qkv(w)
     diff_h = generate_difficulty(w)
     g = bsa.Geometry(w.B, w.H, w.d, w.T, w.Hs, w.Ws)
@@ -484,7 +521,7 @@ def run_ours(args):
     other = peaks["bf16"] if capped else peaks["bf16_sustained"]
     attn_tflops = flops_call / (attn_ms * 1e-3) / 1e12
     valid_flops = _valid_token_flops(g, mask_snapshot)
-    traffic, traffic_src = _traffic()
+    traffic, traffic_src = _traffic(args.workload)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -509,17 +546,14 @@ def run_ours(args):
         "e2e": e2e,
     }
     if not args.no_cpu_baseline and world == 1:
-        heads = [0]
-        t_cpu, pairs = 0.0, 0
-        for hh in heads:
-            dt, pr = _oracle_sample(w, q_h, k_h, v_h, diff_h, hh, list(range(w.NT)))
-            t_cpu += dt
-            pairs += pr
+        t_cpu, pairs, n_rows, t_setup = _oracle_sample(w, q_h, k_h, v_h, diff_h, 0, 64, 8.0)
         line["cpu_baseline"] = {
             "value": pairs * 4.0 * 64 * 64 * w.d / t_cpu / 1e12, "unit": "TFLOP/s",
             "cores": _blas_threads(), "kind": "oracle",
-            "sample": (f"oracle path (reorder, mask, attention of all {w.NT} query tiles) for "
-                       f"head 0 of {w.H}: {pairs} retained tile pairs in {t_cpu:.1f} s")}
+            "sample": (f"oracle path for head 0 of {w.H}: reorder and mask of all {w.NT} query "
+                       f"tiles ({t_setup:.1f} s, charged by the share of retained pairs "
+                       f"attended), attention of {n_rows} seeded-shuffled query tiles: "
+                       f"{pairs} retained tile pairs in {t_cpu:.1f} s charged")}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -55,7 +55,7 @@ def test_mask_bytes():
 
 def test_reference_arm_prints_a_contract_line():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                          "--steps", "3", "--warmup", "3"], capture_output=True, text=True,
+                          "--workload", "tiny", "--steps", "3", "--warmup", "3"], capture_output=True, text=True,
                          timeout=600, cwd=ROOT)
     assert out.returncode == 0, out.stderr[-2000:]
     line = json.loads([ln for ln in out.stdout.splitlines() if ln.startswith("{")][-1])
