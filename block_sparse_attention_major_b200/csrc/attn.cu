@@ -1,4 +1,4 @@
-// Block-sparse attention forward for sm_100a (tcgen05 + TMEM + TMA).
+// Block-sparse attention forward for sm_100a (tcgen05 + TMEM + TMA), persistent.
 //
 // Execution of a block-sparse tile mask (Token Radius Attention summary, "Efficient
 // execution"), FlashAttention-style: for every query row, an online softmax over the
@@ -6,92 +6,144 @@
 // product, fp32 accumulation, output and natural-log LSE written in raster order.
 //
 // Work unit: up to four query tiles of one (b, h) and of the same route class (all
-// dense, or all local), consecutive in tile order. They form two sub-units of two tiles,
-// A and B, each one M=128 tcgen05 tile. The CTA streams the union of the four rows'
-// retained key tiles, in ascending order, through a K ring and a V ring of one key tile
-// (64 keys) per stage. A sub-unit's blocks are the union tiles one of its two query tiles
-// retains; for each it computes S = Q K^T (N=64) and O += P V, so no tensor work is spent
-// on tiles that neither of its query tiles retains; a tile retained by only one of them
-// gets zero probabilities in the other half of the rows.
+// dense, or all local), consecutive in tile order. They form two query blocks of two
+// tiles, A and B, each one M=128 tcgen05 tile. The unit's key stream is the union of the
+// four rows' retained key tiles, ascending, taken two tiles (128 keys) per stream block.
+// For each stream block a query block uses one or both of its tiles (a tile is used when
+// either of the block's two query tiles retains it) or none; it then computes
+// S = Q K^T with N = 128 (both tiles) or N = 64 (one tile) and O += P V over the used keys.
+// A key tile retained by only one of the block's two query tiles gets zero probabilities
+// in the other query tile's rows.
 //
-// Each sub-unit has two S buffers in TMEM. S of block c+1 is computed while the softmax
-// warpgroup turns S of block c into P (written as bf16 over S), so the softmax warpgroups
-// run back to back while the tensor pipe runs the other products. Each sub-unit has its
-// own issuing thread, which sends each product out as soon as its inputs and buffers are
-// ready; the two issuers cover each other's barrier tests, during which a single issuer
-// would leave the tensor pipe idle.
+// Persistent grid: one CTA per SM takes units from a device work list through an atomic
+// counter. The list (built by the scheduler kernels below) is ordered head by head, and
+// within a head by decreasing cost (longest processing time first), so that the heads'
+// K/V tiles stay in L2 while their units run and the last units of the launch are the
+// cheapest. Units flow through the CTA without a barrier between them: the K/V ring, the
+// Q buffers and the TMEM accumulators pass from one unit to the next through the same
+// mbarriers that order the work inside a unit.
 //
-// Schedule (one launch each, on the caller's stream):
-//   sched_count  per (b, h): number of dense rows (kv_count == NKT) and local rows
-//   sched_scan   offsets: every dense unit of every (b, h) first, then the local units
-//   sched_write  per (b, h): the units, four consecutive rows of a class each
-//   attn         one CTA per unit, in list order: heavy (dense) units first, and units of
-//                the same head next to each other so that their K/V tiles stay in L2.
-//
-// CTA roles (352 threads):
-//   warps 0-3  softmax of sub-unit A: thread t owns query row t = TMEM lane t
-//   warps 4-7  softmax of sub-unit B
+// CTA roles (384 threads, three warpgroups):
+//   warps 0-3  softmax of query block A: thread t owns query row t = TMEM lane t
+//   warps 4-7  softmax of query block B
 //              (each reads S from TMEM, writes P as bf16 pairs over S, rescales its O in
-//              TMEM when the running max grows, and runs the epilogue)
-//   warp 8     builds the key-tile lists in shared memory, then lane 0 issues the TMA
-//              loads of Q and of the K/V rings
-//   warp 9     allocates TMEM; lane 0 issues S_A = Q_A K^T (SS) and O_A += P_A V (TS)
-//   warp 10    lane 0 issues the products of sub-unit B
-// TMEM columns: S buffers A0, A1, B0, B1 at 0, 64, 128, 192 (64 each); O_A at 256, O_B at
-// 256 + D. Shared memory (1024-byte aligned): Q_A, Q_B as [D/64][128 rows][128 B], four
-// K and four V stages as [D/64][64 rows][128 B], each with the 128-byte swizzle that TMA
-// and tcgen05 share; barriers; the key-tile list; the per-sub-unit block lists.
+//              TMEM when a row maximum grows by more than 2^8, and runs the epilogue)
+//   warp 8     lane 0 issues the TMA loads of Q and of the K/V ring
+//   warp 9     allocates TMEM; lane 0 issues every tcgen05.mma of both query blocks
+//   warp 10    takes the next unit from the work list and builds its key stream in shared
+//              memory (double buffered, one unit ahead)
+//   warp 11    idle (it completes the third warpgroup)
+// The softmax warpgroups raise their register budget to 208 and the third lowers its own to
+// 88 (setmaxnreg), which keeps a whole 128-column score block of a row in registers.
+// TMEM columns: S_A at 0, S_B at 128 (128 each; P is written over S as bf16 pairs, key k of
+// the block at column k/2), O_A at 256, O_B at 256 + D. Shared memory (1024-byte aligned):
+// Q_A, Q_B, two K and two V stages, each a 128-row operand laid out as [D/64 column
+// blocks][128 rows][128 B] with the 128-byte swizzle that TMA and tcgen05 share (a K or V
+// stage holds the stream block's first tile in rows 0-63, its second in rows 64-127); two
+// key-stream buffers; barriers.
+//
+// Softmax numerics. Scores are scaled by softmax_scale * log2(e) with one FFMA and
+// exponentiated with ex2.approx. A row keeps a reference maximum m and is rescaled only
+// when a block's maximum exceeds m by more than 8 (then O and the row sums are multiplied
+// by 2^(m - m_new); the previous P.V has completed by then, since the pipe ran it before
+// this block's Q K^T); otherwise probabilities up to
+// 2^8 enter P. O is normalised by the sum of the bf16-rounded probabilities that entered
+// P.V (so a row dominated by one key returns that key's value exactly); the LSE uses the
+// fp32 sum of the unrounded probabilities.
+//
+// Token-level support (window kind 2, Token Radius Attention summary: query-centred
+// circular neighbourhoods): when a radius in tokens is given, the key-stream builder marks,
+// per query tile of a local row, the window tiles that the support of some of the tile's
+// tokens does not cover whole; the softmax masks those tiles' slots token by token (the
+// support of this row's token), and treats every other retained tile as a whole tile.
 #include "common.cuh"
 #include "sm100_ptx.cuh"
 #include "tmem_ops.cuh"
+#include "window.cuh"
 
 #include <math.h>
 
 namespace bsa {
 namespace {
 
-constexpr int kAttnThreads = 352;
-constexpr int kNS = 4;                             // K and V ring stages, one key tile each
+constexpr int kAttnThreads = 384;
+constexpr int kRegsLaunch = 168;                   // 65536 / (3 warps per SM sub-partition x 32 x 4), rounded to 8
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsControl = 88;
+static_assert(128 * (2 * kRegsSoftmax + kRegsControl) <= kAttnThreads * kRegsLaunch,
+              "register split above the launch's pool");
+constexpr int kNS = 2;                             // K and V ring stages, two key tiles each
 constexpr long long kWaitLimit = 4000000000LL;     // SM cycles, about 2 s
 constexpr int kTmemCols = 512;
-constexpr int kUnitInts = 8;                       // {bh, q0, q1, q2, q3, 0, 0, 0}
+constexpr int kUnitInts = 8;                       // {bh, q0, q1, q2, q3, cost, 0, 0}
+constexpr float kRescaleLog2 = 8.0f;               // O is rescaled only past 2^8 of growth
 
 template <int D>
 struct Cfg {
   static constexpr int kTileBytes = 64 * D * 2;         // one 64-token tile
-  static constexpr int kQBytes = 2 * kTileBytes;        // one sub-unit's Q (128 rows)
-  static constexpr int kQDB = 128 * 128;                // Q: bytes between 64-column blocks
-  static constexpr int kKDB = 64 * 128;                 // K/V stage: bytes between 64-column blocks
+  static constexpr int kOpBytes = 2 * kTileBytes;       // one 128-row operand
+  static constexpr int kCB = 128 * 128;                 // bytes between 64-column blocks
+  static constexpr int kHalf = 64 * 128;                // rows 64-127 start here in a block
   static constexpr int kQOff = 0;                       // Q_A, then Q_B
-  static constexpr int kKOff = 2 * kQBytes;
-  static constexpr int kVOff = kKOff + kNS * kTileBytes;
-  static constexpr int kBarOff = kVOff + kNS * kTileBytes;
-  // barriers: q, kfull[NS], kempty[NS], vfull[NS], vempty[NS], sfull[4] (sub-unit u,
-  // S buffer b at 2u + b), pfull[2], odone[2], drain[2] (one per issuer)
-  static constexpr int kNumBars = 1 + 4 * kNS + 4 + 2 + 2 + 2;
-  static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base, counts, abort, stage counters
-  static constexpr int kListOff = kMiscOff + 128;
-  static constexpr int kBlkOff = kListOff + kMaxTiles * 4;  // uint16 block lists of A and B
-  static constexpr int kSmemBytes = 1024 + kBlkOff + 2 * kMaxTiles * 2;
-  // TMEM columns: S buffer b of sub-unit u at 64 (2u + b); O of sub-unit u at 256 + u D.
-  static constexpr uint32_t s_col(int u, int b) { return 64u * (2u * u + b); }
-  static constexpr uint32_t o_col(int u) { return 256u + (uint32_t)(u * D); }
+  static constexpr int kKOff = 2 * kOpBytes;
+  static constexpr int kVOff = kKOff + kNS * kOpBytes;
+  static constexpr int kListOff = kVOff + kNS * kOpBytes;
+  // key-stream buffer: meta (8 ints: bh or -1, q0..q3, L), tile ids (u16), flags (u16:
+  // bit t = query tile t retains the tile, bit 4 = the tile has no padding slot, bit 5 + t
+  // = query tile t sees the tile through its tokens' support)
+  static constexpr int kListMeta = 32;
+  static constexpr int kListBytes = kListMeta + kMaxTiles * 2 + kMaxTiles * 2;
+  static constexpr int kBarOff = kListOff + 2 * kListBytes;
+  // kfull, kempty, vfull, vempty [kNS each]; qfull, qempty, sfull, pfull, odone [2 each];
+  // lfull, lempty [2 each]; drain
+  static constexpr int kNumBars = 4 * kNS + 5 * 2 + 2 * 2 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base, abort
+  static constexpr int kSmemBytes = 1024 + kMiscOff + 64;
+  static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
 struct AttnArgs {
   Geom g;
   const uint32_t* mask;
   const int* units;          // kUnitInts per unit
-  const int* header;         // header[1] = number of units
+  int* header;               // header[1] = number of units, header[2] = next unit counter
   __nv_bfloat16* out;
   float* lse;
   uint32_t* err;
   float scale_log2;          // softmax scale * log2(e)
+  // Token-level support: radius in tokens, or -1 for none; local rows (dense[b * NT + i]
+  // == 0) see the tiles of their token window token by token.
+  const uint8_t* dense;
+  int token_rho;
 };
+
+struct Bars {
+  uint32_t b0;
+  __device__ uint32_t kfull(int s) const { return b0 + 8 * s; }
+  __device__ uint32_t kempty(int s) const { return b0 + 8 * (kNS + s); }
+  __device__ uint32_t vfull(int s) const { return b0 + 8 * (2 * kNS + s); }
+  __device__ uint32_t vempty(int s) const { return b0 + 8 * (3 * kNS + s); }
+  __device__ uint32_t qfull(int x) const { return b0 + 8 * (4 * kNS + x); }
+  __device__ uint32_t qempty(int x) const { return b0 + 8 * (4 * kNS + 2 + x); }
+  __device__ uint32_t sfull(int x) const { return b0 + 8 * (4 * kNS + 4 + x); }
+  __device__ uint32_t pfull(int x) const { return b0 + 8 * (4 * kNS + 6 + x); }
+  __device__ uint32_t odone(int x) const { return b0 + 8 * (4 * kNS + 8 + x); }
+  __device__ uint32_t lfull(int b) const { return b0 + 8 * (4 * kNS + 10 + b); }
+  __device__ uint32_t lempty(int b) const { return b0 + 8 * (4 * kNS + 12 + b); }
+  __device__ uint32_t drain() const { return b0 + 8 * (4 * kNS + 14); }
+};
+
+// lempty arrivals per key-stream buffer: the TMA producer, the two issuer cursors and the
+// eight softmax warps.
+constexpr int kListConsumers = 1 + 2 + 8;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+// The two bf16 values of a packed pair, widened exactly to fp32, summed.
+__device__ __forceinline__ float pair_sum(uint32_t w) {
+  return __uint_as_float(w << 16) + __uint_as_float(w & 0xffff0000u);
 }
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -112,73 +164,82 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 // How one key tile's 64 score columns enter this thread's row (warp-uniform): all of them
-// (the row's query tile retains the tile and the tile has no padding), only the valid
-// slots (a retained edge tile), or none (the tile is not retained by this row's query
-// tile: its probabilities are zero). The scores themselves are never rewritten, so the
-// three paths share the registers the TMEM load filled.
+// (the row's query tile retains the tile and the tile has no padding), only some slots (a
+// retained edge tile: its valid slots; a tile seen through the token support: its valid
+// slots in this row's support), or none (this row's query tile does not retain the tile:
+// its probabilities are zero).
 enum TileUse { kUseFull = 0, kUsePartial = 1, kUseSkip = 2 };
 
-// 64 score columns as two 32-column TMEM loads (32-register destination ranges are easier
-// for the register allocator to place than one 64-register range).
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
-  tmem_ld_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-  tmem_ld_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+__device__ __forceinline__ int tile_use(uint32_t flags, int t) {
+  if (!((flags >> t) & 1u)) return kUseSkip;
+  return (((flags >> 4) & 1u) && !((flags >> (5 + t)) & 1u)) ? kUseFull : kUsePartial;
 }
 
-__device__ __forceinline__ int tile_use(uint32_t e, int mshift) {
-  if (!((e >> mshift) & 1u)) return kUseSkip;
-  return ((e >> 20) & 1u) ? kUseFull : kUsePartial;
-}
-
-__device__ __forceinline__ uint64_t entry_valid_mask(uint32_t e, const Geom& g) {
+// Slots of key tile j that this row's scores may use: the valid slots, and under the token
+// support (flag bit 5 + t) only those in the support of the row's token (tq, yq, xq).
+__device__ __forceinline__ uint64_t tile_slots(int j, uint32_t flags, int t, const Geom& g, int tq, int yq,
+                                               int xq, int rho) {
   int tt, ty, tx;
-  tile_xyz(g, (int)(e & 0xffffu), tt, ty, tx);
-  return tile_valid_mask(g, tt, ty, tx);
+  tile_xyz(g, j, tt, ty, tx);
+  uint64_t m = tile_valid_mask(g, tt, ty, tx);
+  if ((flags >> (5 + t)) & 1u) m &= token_support_slots(tq, yq, xq, tt, ty, tx, rho);
+  return m;
 }
 
-// Row maximum with four independent chains (short dependency chains for the scheduler).
-__device__ __forceinline__ float row_max64(const uint32_t (&r)[64], float m) {
+// Row maximum over the 64 columns at offset OFF of r (four short chains).
+template <int OFF>
+__device__ __forceinline__ float half_max_full(const uint32_t (&r)[128], float m) {
   float a0 = m, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
   for (int c = 0; c < 64; c += 8) {
-    a0 = max3(a0, __uint_as_float(r[c + 0]), __uint_as_float(r[c + 1]));
-    a1 = max3(a1, __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
-    a2 = max3(a2, __uint_as_float(r[c + 4]), __uint_as_float(r[c + 5]));
-    a3 = max3(a3, __uint_as_float(r[c + 6]), __uint_as_float(r[c + 7]));
+    a0 = max3(a0, __uint_as_float(r[OFF + c + 0]), __uint_as_float(r[OFF + c + 1]));
+    a1 = max3(a1, __uint_as_float(r[OFF + c + 2]), __uint_as_float(r[OFF + c + 3]));
+    a2 = max3(a2, __uint_as_float(r[OFF + c + 4]), __uint_as_float(r[OFF + c + 5]));
+    a3 = max3(a3, __uint_as_float(r[OFF + c + 6]), __uint_as_float(r[OFF + c + 7]));
   }
   return fmaxf(max3(a0, a1, a2), a3);
 }
 
 // Same over the valid slots only (bit c of `valid` set).
-__device__ __forceinline__ float row_max64_valid(const uint32_t (&r)[64], uint64_t valid, float m) {
+template <int OFF>
+__device__ __forceinline__ float half_max_valid(const uint32_t (&r)[128], uint64_t valid, float m) {
   const uint32_t lo = (uint32_t)valid, hi = (uint32_t)(valid >> 32);
   float a0 = m, a1 = -INFINITY;
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
-    a0 = fmaxf(a0, ((lo >> c) & 1u) ? __uint_as_float(r[c]) : -INFINITY);
-    a1 = fmaxf(a1, ((hi >> c) & 1u) ? __uint_as_float(r[32 + c]) : -INFINITY);
+    a0 = fmaxf(a0, ((lo >> c) & 1u) ? __uint_as_float(r[OFF + c]) : -INFINITY);
+    a1 = fmaxf(a1, ((hi >> c) & 1u) ? __uint_as_float(r[OFF + 32 + c]) : -INFINITY);
   }
   return fmaxf(a0, a1);
 }
 
-// p = 2^(s*c - m) for 64 columns (zero on slots whose bit in `valid` is clear), added to
-// the fp32 row sum and stored to TMEM as bf16 pairs (column 2i in the low half of 32-bit
-// column i), 16 columns per store.
-template <bool kMasked>
-__device__ __forceinline__ void exp_store64(const uint32_t (&r)[64], uint64_t valid, float c, float m,
-                                            float& sum, uint32_t taddr) {
+template <int OFF>
+__device__ __forceinline__ float half_max(const uint32_t (&r)[128], int use, uint64_t valid, float m) {
+  if (use == kUseFull) return half_max_full<OFF>(r, m);
+  if (use == kUsePartial) return half_max_valid<OFF>(r, valid, m);
+  return m;
+}
+
+// p = 2^(s*c - m) for the 64 columns at offset OFF of r (zero on slots whose bit in
+// `valid` is clear), stored to TMEM as bf16 pairs (column 2i in the low half of 32-bit
+// column i), 16 columns per store. `sum` gets the fp32 probabilities, `sum_bf` the
+// bf16-rounded ones that P.V uses.
+template <bool kMasked, int OFF>
+__device__ __forceinline__ void exp_half(const uint32_t (&r)[128], uint64_t valid, float c, float m,
+                                         float& sum, float& sum_bf, uint32_t taddr) {
   const uint32_t lo = (uint32_t)valid, hi = (uint32_t)(valid >> 32);
-  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;       // four short chains
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+  float b0 = 0.f, b1 = 0.f;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     uint32_t pk[8];
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
       const int b = 16 * k + 2 * i;
-      float p0 = ex2(fmaf(__uint_as_float(r[b + 0]), c, -m));
-      float p1 = ex2(fmaf(__uint_as_float(r[b + 1]), c, -m));
-      float p2 = ex2(fmaf(__uint_as_float(r[b + 2]), c, -m));
-      float p3 = ex2(fmaf(__uint_as_float(r[b + 3]), c, -m));
+      float p0 = ex2(fmaf(__uint_as_float(r[OFF + b + 0]), c, -m));
+      float p1 = ex2(fmaf(__uint_as_float(r[OFF + b + 1]), c, -m));
+      float p2 = ex2(fmaf(__uint_as_float(r[OFF + b + 2]), c, -m));
+      float p3 = ex2(fmaf(__uint_as_float(r[OFF + b + 3]), c, -m));
       if (kMasked) {
         const uint32_t w = b < 32 ? lo : hi;
         const int sh = b & 31;
@@ -193,10 +254,13 @@ __device__ __forceinline__ void exp_store64(const uint32_t (&r)[64], uint64_t va
       s1 += p1;
       s2 += p2;
       s3 += p3;
+      b0 += pair_sum(pk[i]);
+      b1 += pair_sum(pk[i + 1]);
     }
     tmem_st_x8(taddr + 8 * k, pk);
   }
   sum += (s0 + s1) + (s2 + s3);
+  sum_bf += b0 + b1;
 }
 
 // Zero probabilities for a tile the row does not retain (32 TMEM columns of bf16 pairs).
@@ -208,18 +272,11 @@ __device__ __forceinline__ void store_zero_p(uint32_t taddr) {
   for (int k = 0; k < 4; ++k) tmem_st_x8(taddr + 8 * k, z);
 }
 
-// Max over one key tile's columns for this row, by its use.
-__device__ __forceinline__ float tile_max(const uint32_t (&r)[64], int use, uint64_t valid, float m) {
-  if (use == kUseFull) return row_max64(r, m);
-  if (use == kUsePartial) return row_max64_valid(r, valid, m);
-  return m;
-}
-
-// Probabilities of one key tile into TMEM, by its use.
-__device__ __forceinline__ void tile_exp(const uint32_t (&r)[64], int use, uint64_t valid, float c, float m,
-                                         float& sum, uint32_t taddr) {
-  if (use == kUseFull) exp_store64<false>(r, 0ull, c, m, sum, taddr);
-  else if (use == kUsePartial) exp_store64<true>(r, valid, c, m, sum, taddr);
+template <int OFF>
+__device__ __forceinline__ void half_exp(const uint32_t (&r)[128], int use, uint64_t valid, float c, float m,
+                                         float& sum, float& sum_bf, uint32_t taddr) {
+  if (use == kUseFull) exp_half<false, OFF>(r, 0ull, c, m, sum, sum_bf, taddr);
+  else if (use == kUsePartial) exp_half<true, OFF>(r, valid, c, m, sum, sum_bf, taddr);
   else store_zero_p(taddr);
 }
 
@@ -238,6 +295,13 @@ __device__ __forceinline__ void rescale_o(uint32_t o_tmem, float alpha) {
   }
 }
 
+// Which tiles of stream block c query block x uses: bit 0 the first tile, bit 1 the second.
+__device__ __forceinline__ int block_use(const uint16_t* flags, int L, int c, int x) {
+  const uint32_t f0 = flags[2 * c];
+  const uint32_t f1 = 2 * c + 1 < L ? flags[2 * c + 1] : 0u;
+  return (((f0 >> (2 * x)) & 3u) ? 1 : 0) | (((f1 >> (2 * x)) & 3u) ? 2 : 0);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -250,45 +314,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   const Geom& g = a.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if ((int)blockIdx.x >= a.header[1]) return;
-  const int* up = a.units + (size_t)blockIdx.x * kUnitInts;
-  const int bh = up[0];
-  const int q0 = up[1], q1 = up[2], q2 = up[3], q3 = up[4];
-  const bool bad = bh < 0 || bh >= g.B * g.H || q0 < 0 || q0 >= g.NT || q1 >= g.NT || q2 >= g.NT ||
-                   q3 >= g.NT || q1 < -1 || q2 < -1 || q3 < -1;
-  if (bad) {
-    if (threadIdx.x == 0) report_error(a.err, BSA_KERR_BAD_UNIT);
-    return;
-  }
-  const bool hasB = q2 >= 0;
-
-  const uint32_t bar0 = sbase + C::kBarOff;
-  const uint32_t bar_q = bar0;
-  const uint32_t kfull0 = bar0 + 8, kempty0 = kfull0 + 8 * kNS, vfull0 = kempty0 + 8 * kNS,
-                 vempty0 = vfull0 + 8 * kNS;
-  const uint32_t sfull0 = vempty0 + 8 * kNS, pfull0 = sfull0 + 32, odone0 = pfull0 + 16,
-                 bar_drain = odone0 + 16;
+  const Bars bar{sbase + C::kBarOff};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
-  int* counts = reinterpret_cast<int*>(smem + C::kMiscOff + 4);        // L, nA, nB
-  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 16);
-  uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::kListOff);
-  uint16_t* blk = reinterpret_cast<uint16_t*>(smem + C::kBlkOff);      // [2][kMaxTiles]
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(bar_q, 1);
     for (int s = 0; s < kNS; ++s) {
-      ptx::mbar_init(kfull0 + 8 * s, 1);
-      ptx::mbar_init(kempty0 + 8 * s, hasB ? 2 : 1);     // one arrival per issuer
-      ptx::mbar_init(vfull0 + 8 * s, 1);
-      ptx::mbar_init(vempty0 + 8 * s, hasB ? 2 : 1);
+      ptx::mbar_init(bar.kfull(s), 1);
+      ptx::mbar_init(bar.kempty(s), 1);
+      ptx::mbar_init(bar.vfull(s), 1);
+      ptx::mbar_init(bar.vempty(s), 1);
     }
-    for (int s = 0; s < 4; ++s) ptx::mbar_init(sfull0 + 8 * s, 1);
-    for (int u = 0; u < 2; ++u) {
-      ptx::mbar_init(pfull0 + 8 * u, 128);
-      ptx::mbar_init(odone0 + 8 * u, 1);
+    for (int x = 0; x < 2; ++x) {
+      ptx::mbar_init(bar.qfull(x), 1);
+      ptx::mbar_init(bar.qempty(x), 1);
+      ptx::mbar_init(bar.sfull(x), 1);
+      ptx::mbar_init(bar.pfull(x), 4);        // one arrival per softmax warp
+      ptx::mbar_init(bar.odone(x), 1);
+      ptx::mbar_init(bar.lfull(x), 1);
+      ptx::mbar_init(bar.lempty(x), kListConsumers);
     }
-    ptx::mbar_init(bar_drain, 1);
-    ptx::mbar_init(bar_drain + 8, 1);
+    ptx::mbar_init(bar.drain(), 1);
     *abort = 0;
     ptx::fence_mbar_init();
   }
@@ -296,213 +342,364 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
     ptx::tmem_relinquish();
   }
-  if (warp == 8) {
-    // Union of the four rows' key tiles, ascending; bit 16+t: retained by query tile q_t;
-    // bit 20: the tile has no padding slot.
-    if (lane == 0) {
-      ptx::prefetch_tensormap(&tmQ);
-      ptx::prefetch_tensormap(&tmK);
-      ptx::prefetch_tensormap(&tmV);
-    }
-    const long long rbase = (long long)bh * g.NT;
-    const uint32_t* m0 = a.mask + (rbase + q0) * g.NW;
-    const uint32_t* m1 = a.mask + (rbase + (q1 >= 0 ? q1 : q0)) * g.NW;
-    const uint32_t* m2 = a.mask + (rbase + (q2 >= 0 ? q2 : q0)) * g.NW;
-    const uint32_t* m3 = a.mask + (rbase + (q3 >= 0 ? q3 : q0)) * g.NW;
-    int running = 0;
-    for (int w0 = 0; w0 < g.NW; w0 += 32) {
-      const int w = w0 + lane;
-      uint32_t b0 = 0u, b1 = 0u, b2 = 0u, b3 = 0u;
-      if (w < g.NW) {
-        const int rem = g.NT - 32 * w;
-        const uint32_t keep = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
-        b0 = __ldg(&m0[w]) & keep;
-        b1 = q1 >= 0 ? (__ldg(&m1[w]) & keep) : 0u;
-        b2 = q2 >= 0 ? (__ldg(&m2[w]) & keep) : 0u;
-        b3 = q3 >= 0 ? (__ldg(&m3[w]) & keep) : 0u;
-      }
-      uint32_t u = b0 | b1 | b2 | b3;
-      const int cnt = __popc(u);
-      int incl = cnt;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
-      }
-      int pos = running + incl - cnt;
-      while (u) {
-        const int bit = __ffs(u) - 1;
-        u &= u - 1;
-        const int j = 32 * w + bit;
-        int tt, ty, tx;
-        tile_xyz(g, j, tt, ty, tx);
-        const uint32_t full = tile_valid_count(g, tt, ty, tx) == 64 ? 1u : 0u;
-        list[pos++] = (uint32_t)j | (((b0 >> bit) & 1u) << 16) | (((b1 >> bit) & 1u) << 17) |
-                      (((b2 >> bit) & 1u) << 18) | (((b3 >> bit) & 1u) << 19) | (full << 20);
-      }
-      running += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    __syncwarp();
-    // Per-sub-unit block lists: the union entries one of the sub-unit's two query tiles
-    // retains, in union order (one key tile per block), each with the number of sub-units
-    // that use it (bits 13-14).
-    const int L = running;
-    int ca = 0, cb = 0;
-    for (int i0 = 0; i0 < L; i0 += 32) {
-      const int i = i0 + lane;
-      const uint32_t e = i < L ? list[i] : 0u;
-      const bool na = ((e >> 16) & 3u) != 0u, nb = ((e >> 18) & 3u) != 0u;
-      const uint32_t ba = __ballot_sync(0xffffffffu, na), bb = __ballot_sync(0xffffffffu, nb);
-      const uint32_t lt = (1u << lane) - 1u;
-      const uint16_t ent = (uint16_t)(i | ((na && nb ? 2 : 1) << 13));   // entry | users << 13
-      if (na) blk[ca + __popc(ba & lt)] = ent;
-      if (nb) blk[kMaxTiles + cb + __popc(bb & lt)] = ent;
-      ca += __popc(ba);
-      cb += __popc(bb);
-    }
-    if (lane == 0) {
-      counts[0] = L;
-      counts[1] = ca;
-      counts[2] = cb;
-    }
-  }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int L = counts[0];
-  if (L == 0 && threadIdx.x == 0) report_error(a.err, BSA_KERR_BAD_MASK);
-  const long long tile_row0 = (long long)bh * g.NT;   // tile index base of this (b, h)
-
-  if (warp == 8) {
+  if (warp >= 8) {
+  ptx::setmaxnreg_dec<kRegsControl>();
+  if (warp == 11) {
+    // idle
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ key-stream builder
+    const int nunits = a.header[1];
+    for (int it = 0;; ++it) {
+      const int buf = it & 1;
+      uint8_t* lb = smem + C::kListOff + buf * C::kListBytes;
+      int* meta = reinterpret_cast<int*>(lb);
+      uint16_t* tiles = reinterpret_cast<uint16_t*>(lb + C::kListMeta);
+      uint16_t* flags = reinterpret_cast<uint16_t*>(lb + C::kListMeta + kMaxTiles * 2);
+      if (it >= 2 && !warp_wait(bar.lempty(buf), ((it >> 1) - 1) & 1, abort, a.err)) break;
+      int bh = -1, q0 = -1, q1 = -1, q2 = -1, q3 = -1;
+      while (true) {
+        int idx = 0;
+        if (lane == 0) idx = atomicAdd(&a.header[2], 1);
+        idx = __shfl_sync(0xffffffffu, idx, 0);
+        if (idx >= nunits) {
+          bh = -1;
+          break;
+        }
+        const int* up = a.units + (size_t)idx * kUnitInts;
+        bh = up[0];
+        q0 = up[1], q1 = up[2], q2 = up[3], q3 = up[4];
+        const bool bad = bh < 0 || bh >= g.B * g.H || q0 < 0 || q0 >= g.NT || q1 >= g.NT || q2 >= g.NT ||
+                         q3 >= g.NT || q1 < -1 || q2 < -1 || q3 < -1;
+        if (!bad) break;
+        if (lane == 0) report_error(a.err, BSA_KERR_BAD_UNIT);
+      }
+      if (bh < 0) {
+        if (lane == 0) {
+          meta[0] = -1;
+          ptx::mbar_arrive(bar.lfull(buf));
+        }
+        break;
+      }
+      // Union of the four rows' key tiles, ascending, with the retaining query tiles.
+      const long long rbase = (long long)bh * g.NT;
+      const uint32_t* m0 = a.mask + (rbase + q0) * g.NW;
+      const uint32_t* m1 = a.mask + (rbase + (q1 >= 0 ? q1 : q0)) * g.NW;
+      const uint32_t* m2 = a.mask + (rbase + (q2 >= 0 ? q2 : q0)) * g.NW;
+      const uint32_t* m3 = a.mask + (rbase + (q3 >= 0 ? q3 : q0)) * g.NW;
+      // token support: coordinates of the query tiles, and which of them are local rows
+      const int rho = a.token_rho;
+      uint32_t cq[4];
+      bool loc[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int qtile = t == 0 ? q0 : t == 1 ? q1 : t == 2 ? q2 : q3;
+        int tt, ty, tx;
+        tile_xyz(g, qtile >= 0 ? qtile : q0, tt, ty, tx);
+        cq[t] = pack_coord(tt, ty, tx);
+        loc[t] = rho >= 0 && qtile >= 0 && a.dense[(long long)(bh / g.H) * g.NT + qtile] == 0;
+      }
+      int running = 0;
+      for (int w0 = 0; w0 < g.NW; w0 += 32) {
+        const int w = w0 + lane;
+        uint32_t b0 = 0u, b1 = 0u, b2 = 0u, b3 = 0u;
+        if (w < g.NW) {
+          const int rem = g.NT - 32 * w;
+          const uint32_t keep = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+          b0 = __ldg(&m0[w]) & keep;
+          b1 = q1 >= 0 ? (__ldg(&m1[w]) & keep) : 0u;
+          b2 = q2 >= 0 ? (__ldg(&m2[w]) & keep) : 0u;
+          b3 = q3 >= 0 ? (__ldg(&m3[w]) & keep) : 0u;
+        }
+        uint32_t u = b0 | b1 | b2 | b3;
+        const int cnt = __popc(u);
+        int incl = cnt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += v;
+        }
+        int pos = running + incl - cnt;
+        while (u) {
+          const int bit = __ffs(u) - 1;
+          u &= u - 1;
+          const int j = 32 * w + bit;
+          int tt, ty, tx;
+          tile_xyz(g, j, tt, ty, tx);
+          const uint32_t full = tile_valid_count(g, tt, ty, tx) == 64 ? 1u : 0u;
+          const uint32_t kept = ((b0 >> bit) & 1u) | (((b1 >> bit) & 1u) << 1) | (((b2 >> bit) & 1u) << 2) |
+                                (((b3 >> bit) & 1u) << 3);
+          uint32_t tok = 0u;
+          if (rho >= 0) {
+            const uint32_t cj = pack_coord(tt, ty, tx);
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+              if (loc[t] && ((kept >> t) & 1u) && in_token_window(cq[t], cj, rho) &&
+                  !token_tiles_all_inside(cq[t], cj, g.T, g.Hs, g.Ws, rho))
+                tok |= 1u << t;
+          }
+          tiles[pos] = (uint16_t)j;
+          flags[pos] = (uint16_t)(kept | (full << 4) | (tok << 5));
+          ++pos;
+        }
+        running += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) {
+        meta[0] = bh;
+        meta[1] = q0;
+        meta[2] = q1;
+        meta[3] = q2;
+        meta[4] = q3;
+        meta[5] = running;
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar.lfull(buf));
+    }
+  } else if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0 && L > 0) {
-      const int nsub = hasB ? 2 : 1;
-      ptx::mbar_arrive_expect_tx(bar_q, nsub * C::kQBytes);
-      for (int t = 0; t < 2 * nsub; ++t) {
-        const int qt = t == 0 ? q0 : t == 1 ? q1 : t == 2 ? q2 : q3;
-        const int tile = qt >= 0 ? qt : (t < 2 ? q0 : q2);
-        const int row = (int)((tile_row0 + tile) * 64);
-        const uint32_t dst = sbase + C::kQOff + (t >> 1) * C::kQBytes + (t & 1) * 8192;
+    if (lane == 0) {
+      ptx::prefetch_tensormap(&tmQ);
+      ptx::prefetch_tensormap(&tmK);
+      ptx::prefetch_tensormap(&tmV);
+      int qn[2] = {0, 0};       // Q loads issued per query block
+      long long nk = 0, nv = 0; // stream blocks whose K / V load was issued
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        const int buf = it & 1;
+        const uint8_t* lb = smem + C::kListOff + buf * C::kListBytes;
+        const int* meta = reinterpret_cast<const int*>(lb);
+        const uint16_t* tiles = reinterpret_cast<const uint16_t*>(lb + C::kListMeta);
+        if (!ptx::mbar_wait(bar.lfull(buf), (it >> 1) & 1, abort, a.err, kWaitLimit)) break;
+        const int bh = meta[0];
+        if (bh < 0) break;
+        const int q[4] = {meta[1], meta[2], meta[3], meta[4]};
+        const int L = meta[5];
+        const long long tile_row0 = (long long)bh * g.NT;
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (q[2 * x] < 0) continue;
+          if (qn[x] > 0 && !ptx::mbar_wait(bar.qempty(x), (qn[x] - 1) & 1, abort, a.err, kWaitLimit)) {
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(bar.qfull(x), C::kOpBytes);
+          for (int rh = 0; rh < 2; ++rh) {
+            const int tile = q[2 * x + rh] >= 0 ? q[2 * x + rh] : q[2 * x];   // a missing tile repeats the first
+            const int row = (int)((tile_row0 + tile) * 64);
+            const uint32_t dst = sbase + C::kQOff + x * C::kOpBytes + rh * C::kHalf;
 #pragma unroll
-        for (int db = 0; db < D / 64; ++db) ptx::tma_load_2d(dst + db * C::kQDB, &tmQ, bar_q, db * 64, row);
+            for (int cb = 0; cb < D / 64; ++cb) ptx::tma_load_2d(dst + cb * C::kCB, &tmQ, bar.qfull(x), cb * 64, row);
+          }
+          ++qn[x];
+        }
+        const int nb = (L + 1) / 2;
+        for (int c = 0; c < nb && ok; ++c) {
+          const int nh = 2 * c + 1 < L ? 2 : 1;
+          {
+            const int s = (int)(nk % kNS);
+            const uint32_t ph = ((nk / kNS) & 1) ^ 1;
+            if (!ptx::mbar_wait(bar.kempty(s), ph, abort, a.err, kWaitLimit)) { ok = false; break; }
+            ptx::mbar_arrive_expect_tx(bar.kfull(s), nh * C::kTileBytes);
+            for (int h = 0; h < nh; ++h) {
+              const int row = (int)((tile_row0 + tiles[2 * c + h]) * 64);
+              const uint32_t dst = sbase + C::kKOff + s * C::kOpBytes + h * C::kHalf;
+#pragma unroll
+              for (int cb = 0; cb < D / 64; ++cb) ptx::tma_load_2d(dst + cb * C::kCB, &tmK, bar.kfull(s), cb * 64, row);
+            }
+            ++nk;
+          }
+          {
+            const int s = (int)(nv % kNS);
+            const uint32_t ph = ((nv / kNS) & 1) ^ 1;
+            if (!ptx::mbar_wait(bar.vempty(s), ph, abort, a.err, kWaitLimit)) { ok = false; break; }
+            ptx::mbar_arrive_expect_tx(bar.vfull(s), nh * C::kTileBytes);
+            for (int h = 0; h < nh; ++h) {
+              const int row = (int)((tile_row0 + tiles[2 * c + h]) * 64);
+              const uint32_t dst = sbase + C::kVOff + s * C::kOpBytes + h * C::kHalf;
+#pragma unroll
+              for (int cb = 0; cb < D / 64; ++cb) ptx::tma_load_2d(dst + cb * C::kCB, &tmV, bar.vfull(s), cb * 64, row);
+            }
+            ++nv;
+          }
+        }
+        if (ok) ptx::mbar_arrive(bar.lempty(buf));
       }
-      int nk = 0, nv = 0;       // tiles whose K / V load was issued
-      for (int i = 0; i < L; ++i) {
-        const int s = i % kNS;
-        const uint32_t ph = ((i / kNS) & 1) ^ 1;
-        const int row = (int)((tile_row0 + (int)(list[i] & 0xffffu)) * 64);
-        if (!ptx::mbar_wait(kempty0 + 8 * s, ph, abort, a.err, kWaitLimit)) break;
-        ptx::mbar_arrive_expect_tx(kfull0 + 8 * s, C::kTileBytes);
-#pragma unroll
-        for (int db = 0; db < D / 64; ++db)
-          ptx::tma_load_2d(sbase + C::kKOff + s * C::kTileBytes + db * C::kKDB, &tmK, kfull0 + 8 * s, db * 64, row);
-        ++nk;
-        if (!ptx::mbar_wait(vempty0 + 8 * s, ph, abort, a.err, kWaitLimit)) break;
-        ptx::mbar_arrive_expect_tx(vfull0 + 8 * s, C::kTileBytes);
-#pragma unroll
-        for (int db = 0; db < D / 64; ++db)
-          ptx::tma_load_2d(sbase + C::kVOff + s * C::kTileBytes + db * C::kKDB, &tmV, vfull0 + 8 * s, db * 64, row);
-        ++nv;
-      }
-      // Never leave with copies in flight: wait for the last load issued into each stage.
+      // Never leave with copies in flight: wait for the last load issued into each buffer.
       int zero = 0;
       for (int s = 0; s < kNS; ++s) {
         if (nk > s) {
-          const int last = s + kNS * ((nk - 1 - s) / kNS);
-          ptx::mbar_wait(kfull0 + 8 * s, (last / kNS) & 1, &zero, a.err, kWaitLimit);
+          const long long last = s + kNS * ((nk - 1 - s) / kNS);
+          ptx::mbar_wait(bar.kfull(s), (uint32_t)((last / kNS) & 1), &zero, a.err, kWaitLimit);
         }
         if (nv > s) {
-          const int last = s + kNS * ((nv - 1 - s) / kNS);
-          ptx::mbar_wait(vfull0 + 8 * s, (last / kNS) & 1, &zero, a.err, kWaitLimit);
+          const long long last = s + kNS * ((nv - 1 - s) / kNS);
+          ptx::mbar_wait(bar.vfull(s), (uint32_t)((last / kNS) & 1), &zero, a.err, kWaitLimit);
         }
       }
-      ptx::mbar_wait(bar_q, 0, &zero, a.err, kWaitLimit);
+      for (int x = 0; x < 2; ++x)
+        if (qn[x] > 0) ptx::mbar_wait(bar.qfull(x), (qn[x] - 1) & 1, &zero, a.err, kWaitLimit);
     }
-  } else if (warp == 9 || warp == 10) {
-    // ------------------------------------------------------------------ MMA issuers
-    // One issuing thread per sub-unit (lane 0 of warp 9 for A, of warp 10 for B). Issue is
-    // throttled to the tensor pipe's pace, so a single thread leaves the pipe idle while it
-    // tests barriers between products; two threads cover each other's tests.
-    //
-    // Each issuer walks the whole union list in order with two cursors. K cursor: for an
-    // entry its sub-unit uses, S = Q K^T into the next S buffer once the K tile is in and
-    // the buffer is free (the P.V two blocks back has been issued: the tensor pipe runs a
-    // thread's products in issue order, so S of block c can overwrite the P of block c - 2
-    // issued before it), then a commit on the stage's empty barrier; for any other entry, a
-    // plain arrive there once the entry's K tile was seen loaded. V cursor: for an entry it
-    // uses, O += P V once its softmax has written P and the V tile is in, then a commit on
-    // the stage's empty barrier; for any other entry, a plain arrive once its V tile was
-    // seen loaded. The empty barriers count one arrival per issuer, so a stage is reloaded
-    // only after both issuers' products on it have completed (a commit tracks its own
-    // thread's products). Because each cursor sees every load of its ring in order, the
-    // full barrier is never more than one phase behind the entry tested and the parity
-    // tests are exact. Nothing blocks: a wait on one cursor could hold up the other.
-    static_assert(kNS == 4, "stage arithmetic below assumes four stages");
-    const int u = warp - 9;
-    if (lane == 0 && L > 0 && (u == 0 || hasB)) {
-      constexpr uint32_t kIdQK = ptx::idesc_bf16_f32(128, 64, 0, 0);
+  } else if (warp == 9) {
+    // ------------------------------------------------------------------ MMA issuer
+    // Lane 0 issues every product of both query blocks. Two cursors (A and B) walk the
+    // units' stream blocks in order, each with a K position and a V position. At its K
+    // position a cursor issues S = Q K^T for a block its query block uses, once the K
+    // stage is in and its single S buffer is free (the P.V of its previous block has been
+    // issued: the tensor pipe runs one thread's products in issue order, so S may
+    // overwrite that P); at its V position it issues O += P V once its softmax has written
+    // P and the V stage is in. A block the query block does not use is passed once its
+    // stage is seen loaded. A stage is released (one commit on its empty barrier) when the
+    // second cursor passes it, so both cursors' products on it are tracked by the commit.
+    // Each cursor sees every load of the ring in order, so a full barrier is never more
+    // than one phase behind the block tested and the parity tests are exact. Nothing
+    // blocks: one cursor waiting must not hold up the other.
+    if (lane == 0) {
+      constexpr uint32_t kIdQK128 = ptx::idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t kIdQK64 = ptx::idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t kIdPV = ptx::idesc_bf16_f32(128, D, 0, 1);
-      constexpr int kNoEntry = 1 << 20;
-      const uint64_t qd = ptx::smem_desc_sw128(sbase + C::kQOff + u * C::kQBytes, 16, 1024);
-      const uint64_t dK0 = ptx::smem_desc_sw128(sbase + C::kKOff, 16, 1024);
-      const uint64_t dV0 = ptx::smem_desc_sw128(sbase + C::kVOff, C::kKDB, 1024);
-      const uint32_t o_tmem = tmem + C::o_col(u);
-      const uint32_t pfull_u = pfull0 + 8 * u, odone_u = odone0 + 8 * u;
-      const int n = counts[1 + u];
-      const uint16_t* my_blk = blk + u * kMaxTiles;
-      int qc = 0, pc = 0, ki = 0, vi = 0;
-      int qnext = n > 0 ? (int)(my_blk[0] & 0x1fffu) : kNoEntry;   // union index of the next QK block
-      int pnext = qnext;                                            // and of the next P.V block
-      bool ok = ptx::mbar_wait(bar_q, 0, abort, a.err, kWaitLimit);
+      struct Cursor {
+        int it;            // key-stream buffer iteration
+        bool have, done;
+        int L, nb, kc, vc, pend;
+        bool hasq, qready, qreleased, first_pv;
+        long long gbase;   // global index of the unit's first stream block
+        int qn;            // Q loads consumed (units with this query block)
+        uint32_t pn;       // P.V products issued (= pfull phases consumed)
+        const uint16_t* flags;
+      };
+      Cursor cur[2];
+      for (int x = 0; x < 2; ++x) {
+        cur[x].it = 0;
+        cur[x].have = cur[x].done = false;
+        cur[x].L = cur[x].nb = cur[x].kc = cur[x].vc = 0;
+        cur[x].pend = -1;
+        cur[x].hasq = cur[x].qready = cur[x].qreleased = cur[x].first_pv = false;
+        cur[x].gbase = 0;
+        cur[x].qn = 0;
+        cur[x].pn = 0;
+        cur[x].flags = nullptr;
+      }
+      long long kpass[2] = {0, 0}, vpass[2] = {0, 0};
+      bool ok = true;
       long long idle_since = clock64();
-      while (ok && vi < L) {
+      while (ok && !(cur[0].done && cur[1].done)) {
         bool progress = false;
-        if (ki < L) {
-          const uint32_t s = ki & 3;
-          if (ki == qnext) {
-            if (qc - pc < 2 && ptx::mbar_test_wait(kfull0 + 8 * s, (ki >> 2) & 1)) {
-              // No tcgen05 fence: K arrived through the TMA barrier, and the S buffer is
-              // reused behind this thread's own P.V (ordered by the fence on that path).
-              const uint32_t s_tmem = tmem + C::s_col(u, qc & 1);
-              const uint64_t kd = dK0 + s * (C::kTileBytes >> 4);
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk)
-                ptx::mma_ss(s_tmem, qd + (((kk >> 2) * C::kQDB + (kk & 3) * 32) >> 4),
-                            kd + (((kk >> 2) * C::kKDB + (kk & 3) * 32) >> 4), kIdQK, kk > 0 ? 1u : 0u);
-              ptx::mma_commit(sfull0 + 8 * (2 * u + (qc & 1)));
-              ptx::mma_commit(kempty0 + 8 * s);
-              ++qc;
-              qnext = qc < n ? (int)(my_blk[qc] & 0x1fffu) : kNoEntry;
-              ++ki;
-              progress = true;
-            }
-          } else if (ptx::mbar_test_wait(kfull0 + 8 * s, (ki >> 2) & 1)) {
-            ptx::mbar_arrive(kempty0 + 8 * s);
-            ++ki;
+        for (int x = 0; x < 2; ++x) {
+          Cursor& cu = cur[x];
+          if (cu.done) continue;
+          if (!cu.have) {
+            const int buf = cu.it & 1;
+            if (!ptx::mbar_test_wait(bar.lfull(buf), (cu.it >> 1) & 1)) continue;
+            const uint8_t* lb = smem + C::kListOff + buf * C::kListBytes;
+            const int* meta = reinterpret_cast<const int*>(lb);
             progress = true;
+            if (meta[0] < 0) {
+              cu.done = true;
+              continue;
+            }
+            cu.have = true;
+            cu.L = meta[5];
+            cu.nb = (cu.L + 1) / 2;
+            cu.kc = cu.vc = 0;
+            cu.pend = -1;
+            cu.hasq = meta[1 + 2 * x] >= 0;
+            cu.qready = false;
+            cu.qreleased = false;
+            cu.first_pv = true;
+            cu.flags = reinterpret_cast<const uint16_t*>(lb + C::kListMeta + kMaxTiles * 2);
           }
-        }
-        if (vi < ki) {
-          const uint32_t s = vi & 3;
-          if (vi == pnext) {
-            if (ptx::mbar_test_wait(pfull_u, pc & 1) && ptx::mbar_test_wait(vfull0 + 8 * s, (vi >> 2) & 1)) {
-              ptx::tc_fence_after();
-              const uint32_t p_tmem = tmem + C::s_col(u, pc & 1);
-              const uint64_t vd = dV0 + s * (C::kTileBytes >> 4);
+          // ---- K position
+          if (cu.kc < cu.nb) {
+            const int u = cu.hasq ? block_use(cu.flags, cu.L, cu.kc, x) : 0;
+            const long long gi = cu.gbase + cu.kc;
+            const int s = (int)(gi % kNS);
+            const uint32_t fph = (uint32_t)((gi / kNS) & 1);
+            bool passed = false;
+            if (u == 0) {
+              passed = ptx::mbar_test_wait(bar.kfull(s), fph);
+            } else if (cu.pend < 0) {
+              if (!cu.qready) cu.qready = ptx::mbar_test_wait(bar.qfull(x), cu.qn & 1);
+              if (cu.qready && ptx::mbar_test_wait(bar.kfull(s), fph)) {
+                // S = Q K^T over the used tiles: N = 128 for both, N = 64 for one (its
+                // columns at 64 * tile in S).
+                const int h0 = u == 2 ? 1 : 0;
+                const uint32_t s_tmem = tmem + (uint32_t)(x * 128 + h0 * 64);
+                const uint64_t qd = ptx::smem_desc_sw128(sbase + C::kQOff + x * C::kOpBytes, 16, 1024);
+                const uint64_t kd =
+                    ptx::smem_desc_sw128(sbase + C::kKOff + s * C::kOpBytes + h0 * C::kHalf, 16, 1024);
+                const uint32_t id = u == 3 ? kIdQK128 : kIdQK64;
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + kk * (2048 >> 4), kIdPV, (pc > 0 || kk > 0) ? 1u : 0u);
-              ptx::mma_commit(odone_u);
-              ptx::mma_commit(vempty0 + 8 * s);
-              ++pc;
-              pnext = pc < n ? (int)(my_blk[pc] & 0x1fffu) : kNoEntry;
-              ++vi;
+                for (int kk = 0; kk < D / 16; ++kk) {
+                  const uint32_t off = (uint32_t)(((kk >> 2) * C::kCB + (kk & 3) * 32) >> 4);
+                  ptx::mma_ss(s_tmem, qd + off, kd + off, id, kk > 0 ? 1u : 0u);
+                }
+                ptx::mma_commit(bar.sfull(x));
+                cu.pend = cu.kc;
+                passed = true;
+              }
+            }
+            if (passed) {
+              kpass[x] = gi + 1;
+              if (kpass[x ^ 1] >= gi + 1) ptx::mma_commit(bar.kempty(s));
+              ++cu.kc;
+              progress = true;
+              if (cu.kc == cu.nb && cu.hasq && cu.qready && !cu.qreleased) {
+                ptx::mma_commit(bar.qempty(x));      // the unit's last Q K^T has been issued
+                cu.qreleased = true;
+              }
+            }
+          }
+          // ---- V position
+          if (cu.vc < cu.kc) {
+            const long long gi = cu.gbase + cu.vc;
+            const int s = (int)(gi % kNS);
+            const uint32_t fph = (uint32_t)((gi / kNS) & 1);
+            bool passed = false;
+            if (cu.vc == cu.pend) {
+              if (ptx::mbar_test_wait(bar.pfull(x), cu.pn & 1) && ptx::mbar_test_wait(bar.vfull(s), fph)) {
+                ptx::tc_fence_after();
+                const int u = block_use(cu.flags, cu.L, cu.vc, x);
+                const uint32_t o_tmem = tmem + 256u + (uint32_t)(x * D);
+                const uint32_t p_tmem = tmem + (uint32_t)(x * 128);
+                const uint64_t vd = ptx::smem_desc_sw128(sbase + C::kVOff + s * C::kOpBytes, C::kCB, 1024);
+                const int k0 = (u & 1) ? 0 : 4, k1 = (u & 2) ? 8 : 4;
+                for (int kk = k0; kk < k1; ++kk) {
+                  ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + (uint64_t)(kk * (2048 >> 4)), kIdPV,
+                              (cu.first_pv && kk == k0) ? 0u : 1u);
+                }
+                ptx::mma_commit(bar.odone(x));
+                cu.first_pv = false;
+                ++cu.pn;
+                cu.pend = -1;
+                passed = true;
+              }
+            } else {
+              passed = ptx::mbar_test_wait(bar.vfull(s), fph);
+            }
+            if (passed) {
+              vpass[x] = gi + 1;
+              if (vpass[x ^ 1] >= gi + 1) ptx::mma_commit(bar.vempty(s));
+              ++cu.vc;
               progress = true;
             }
-          } else if (ptx::mbar_test_wait(vfull0 + 8 * s, (vi >> 2) & 1)) {
-            ptx::mbar_arrive(vempty0 + 8 * s);
-            ++vi;
+          }
+          // ---- end of the unit
+          if (cu.kc == cu.nb && cu.vc == cu.nb) {
+            if (cu.hasq && !cu.qreleased) {
+              // No product used Q (its rows retain nothing here): release it once loaded.
+              if (!cu.qready) cu.qready = ptx::mbar_test_wait(bar.qfull(x), cu.qn & 1);
+              if (!cu.qready) continue;
+              ptx::mma_commit(bar.qempty(x));
+              cu.qreleased = true;
+            }
+            if (cu.hasq) ++cu.qn;
+            ptx::mbar_arrive(bar.lempty(cu.it & 1));
+            ++cu.it;
+            cu.have = false;
+            cu.gbase += cu.nb;
             progress = true;
           }
         }
@@ -518,80 +715,126 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       // Never free TMEM under a running MMA: wait until everything issued has completed.
       int zero = 0;
-      ptx::mma_commit(bar_drain + 8 * u);
-      ptx::mbar_wait(bar_drain + 8 * u, 0, &zero, a.err, kWaitLimit);
+      ptx::mma_commit(bar.drain());
+      ptx::mbar_wait(bar.drain(), 0, &zero, a.err, kWaitLimit);
     }
+  }
   } else {
+    ptx::setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------------------------------------------ softmax + epilogue
-    const int u = warp >> 2;                 // sub-unit of this warpgroup
+    const int x = warp >> 2;                 // query block of this warpgroup
     const int row = threadIdx.x & 127;       // TMEM lane
-    const int half = row >> 6;
-    const int qt = u ? (half ? q3 : q2) : (half ? q1 : q0);   // this row's query tile (-1: none)
+    const int rh = row >> 6;                 // which of the block's two query tiles
+    const int t = 2 * x + rh;                // query tile slot in the unit
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t o_tmem = tmem + C::o_col(u) + lane_base;
-    const uint32_t pfull_u = pfull0 + 8 * u, odone_u = odone0 + 8 * u;
-    const int n = counts[1 + u];
-    const uint16_t* my_blk = blk + u * kMaxTiles;
-    const int mshift = 16 + 2 * u + half;
+    const uint32_t s_tmem = tmem + (uint32_t)(x * 128) + lane_base;
+    const uint32_t o_tmem = tmem + 256u + (uint32_t)(x * D) + lane_base;
     const float c = a.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
-    bool ok = n > 0;
-    for (int it = 0; it < n; ++it) {
-      const int b = it & 1;
-      if (!warp_wait(sfull0 + 8 * (2 * u + b), (it >> 1) & 1, abort, a.err)) { ok = false; break; }
-      ptx::tc_fence_after();
-      const uint32_t e = list[my_blk[it] & 0x1fffu];
-      const uint32_t s_tmem = tmem + C::s_col(u, b) + lane_base;
-      const int use = tile_use(e, mshift);
-      const uint64_t valid = use == kUsePartial ? entry_valid_mask(e, g) : ~0ull;
-      uint32_t r[64];
-      float mx = -INFINITY;
-      if (use != kUseSkip) {
-        tmem_ld64(s_tmem, r);
-        ptx::tmem_wait_ld();
-        mx = tile_max(r, use, valid, mx);
+    uint32_t sidx = 0;                       // blocks processed (sfull / pfull phases)
+    for (int it = 0;; ++it) {
+      const int buf = it & 1;
+      const uint8_t* lb = smem + C::kListOff + buf * C::kListBytes;
+      const int* meta = reinterpret_cast<const int*>(lb);
+      const uint16_t* tiles = reinterpret_cast<const uint16_t*>(lb + C::kListMeta);
+      const uint16_t* flags = reinterpret_cast<const uint16_t*>(lb + C::kListMeta + kMaxTiles * 2);
+      if (!warp_wait(bar.lfull(buf), (it >> 1) & 1, abort, a.err)) break;
+      const int bh = meta[0];
+      if (bh < 0) break;
+      const int qt = meta[1 + t];
+      const int L = meta[5];
+      const int nb = (L + 1) / 2;
+      int tq = 0, yq = 0, xq = 0;            // this row's token (the token support's centre)
+      {
+        int tt, ty, tx;
+        tile_xyz(g, qt >= 0 ? qt : 0, tt, ty, tx);
+        const int rr = row & 63;
+        tq = 4 * tt + (rr >> 4);
+        yq = 4 * ty + ((rr >> 2) & 3);
+        xq = 4 * tx + (rr & 3);
       }
-      // The reference follows the running max exactly, so the row's largest probability
-      // is 2^0 = 1, which bf16 holds exactly: rows dominated by one key lose nothing to
-      // the bf16 rounding of P. O is rescaled in TMEM whenever the max grows.
-      const float m_new = fmaxf(m_run, mx * c);
-      const bool grow = m_new > m_run;
-      const float alpha = grow ? ex2(m_run - m_new) : 1.0f;
-      const float m_use = (m_new == -INFINITY) ? 0.0f : m_new;
-      float sum = 0.f;
-      tile_exp(r, use, valid, c, m_use, sum, s_tmem);
-      l_run = l_run * alpha + sum;
-      if (it > 0) {
-        // The previous block's P.V must be complete: O is rescaled only over exactly the
-        // previous blocks, and P of this block is released only after it, so that the
-        // issuing thread never sees P phases two ahead of the products it has issued.
-        if (!warp_wait(odone_u, (it - 1) & 1, abort, a.err)) { ok = false; break; }
+      float m_run = -INFINITY, l_ex = 0.f, l_bf = 0.f;
+      int nused = 0;
+      bool ok = true;
+      for (int cb = 0; cb < nb; ++cb) {
+        const int u = meta[1 + 2 * x] >= 0 ? block_use(flags, L, cb, x) : 0;
+        if (!u) continue;
+        const uint32_t f0 = flags[2 * cb];
+        const uint32_t f1 = 2 * cb + 1 < L ? flags[2 * cb + 1] : 0u;
+        const int use0 = (u & 1) ? tile_use(f0, t) : kUseSkip;
+        const int use1 = (u & 2) ? tile_use(f1, t) : kUseSkip;
+        const uint64_t valid0 =
+            use0 == kUsePartial ? tile_slots(tiles[2 * cb], f0, t, g, tq, yq, xq, a.token_rho) : ~0ull;
+        const uint64_t valid1 =
+            use1 == kUsePartial ? tile_slots(tiles[2 * cb + 1], f1, t, g, tq, yq, xq, a.token_rho) : ~0ull;
+        if (!warp_wait(bar.sfull(x), sidx & 1, abort, a.err)) { ok = false; break; }
         ptx::tc_fence_after();
-        if (__any_sync(0xffffffffu, grow)) rescale_o<D>(o_tmem, alpha);
+        uint32_t r[128];
+        if (u & 1) {
+          tmem_ld_x32(s_tmem + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld_x32(s_tmem + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        }
+        if (u & 2) {
+          tmem_ld_x32(s_tmem + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
+          tmem_ld_x32(s_tmem + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+        }
+        ptx::tmem_wait_ld();
+        float mx = -INFINITY;
+        mx = half_max<0>(r, use0, valid0, mx);
+        mx = half_max<64>(r, use1, valid1, mx);
+        const float mb = mx * c;                       // block maximum, log2 domain
+        bool resc = false;
+        if (m_run == -INFINITY) m_run = mb;            // O of this row is still zero
+        else if (mb > m_run + kRescaleLog2) resc = true;
+        if (__any_sync(0xffffffffu, resc)) {
+          // O holds exactly the unit's earlier blocks here: the issuer sent this block's
+          // Q K^T after the previous block's P.V, the pipe ran them in that order, and S of
+          // this block is complete.
+          const float alpha = resc ? ex2(m_run - mb) : 1.0f;
+          rescale_o<D>(o_tmem, alpha);
+          l_ex *= alpha;
+          l_bf *= alpha;
+          if (resc) m_run = mb;
+        }
+        const float m_use = m_run == -INFINITY ? 0.0f : m_run;
+        if (u & 1) half_exp<0>(r, use0, valid0, c, m_use, l_ex, l_bf, s_tmem + 0);
+        if (u & 2) half_exp<64>(r, use1, valid1, c, m_use, l_ex, l_bf, s_tmem + 32);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar.pfull(x));
+        ++sidx;
+        ++nused;
       }
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(pfull_u);
-      m_run = m_new;
-    }
-    if (ok && warp_wait(odone_u, (n - 1) & 1, abort, a.err)) {
-      ptx::tc_fence_after();
-      const int r = row & 63;
+      const int bq = bh / g.H, hq = bh - (bh / g.H) * g.H;
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar.lempty(buf));
+      if (!ok) break;
+      // ---- epilogue: O / l (bf16) and the LSE, in raster order
+      const int rr = row & 63;
       int n_tok = -1;
       if (qt >= 0) {
         int tt, ty, tx;
         tile_xyz(g, qt, tt, ty, tx);
-        const int t = tt * 4 + (r >> 4), y = ty * 4 + ((r >> 2) & 3), xx = tx * 4 + (r & 3);
-        if (t < g.T && y < g.Hs && xx < g.Ws) n_tok = (t * g.Hs + y) * g.Ws + xx;
+        const int tk = tt * 4 + (rr >> 4), y = ty * 4 + ((rr >> 2) & 3), xx = tx * 4 + (rr & 3);
+        if (tk < g.T && y < g.Hs && xx < g.Ws) n_tok = (tk * g.Hs + y) * g.Ws + xx;
       }
-      const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
-      const int bb = bh / g.H, h = bh - bb * g.H;
-      uint4* dst = n_tok >= 0 ? reinterpret_cast<uint4*>(a.out + (((long long)bb * g.N + n_tok) * g.H + h) * D) : nullptr;
+      if (nused > 0) {
+        if (!warp_wait(bar.odone(x), (sidx - 1) & 1, abort, a.err)) break;
+        ptx::tc_fence_after();
+      }
+      const float inv_l = l_bf > 0.f ? 1.0f / l_bf : 0.f;
+      uint4* dst = n_tok >= 0 ? reinterpret_cast<uint4*>(a.out + (((long long)bq * g.N + n_tok) * g.H + hq) * D)
+                              : nullptr;
 #pragma unroll 1
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t ov[32];
-        tmem_ld_x32(o_tmem + ch * 32, ov);
-        ptx::tmem_wait_ld();
+        if (nused > 0) {
+          tmem_ld_x32(o_tmem + ch * 32, ov);
+          ptx::tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) ov[k] = 0u;
+        }
         if (dst) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -605,13 +848,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       if (n_tok >= 0) {
-        if (!(l_run > 0.f)) report_error(a.err, BSA_KERR_BAD_MASK);
+        if (!(l_ex > 0.f)) report_error(a.err, BSA_KERR_BAD_MASK);
         if (a.lse) {
-          const float m_fin = (m_run == -INFINITY) ? 0.0f : m_run;
+          const float m_fin = m_run == -INFINITY ? 0.0f : m_run;
           a.lse[(long long)bh * g.N + n_tok] =
-              l_run > 0.f ? (m_fin + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+              l_ex > 0.f ? (m_fin + __log2f(l_ex)) * 0.69314718055994531f : -INFINITY;
         }
       }
+      // The next unit's first P.V overwrites O: every TMEM read above must be complete
+      // before this warp releases that unit's first P (ordered by the fence before it).
     }
   }
 
@@ -625,6 +870,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 }
 
 // ------------------------------------------------------------------------ scheduler
+// Units of a (b, h): the dense rows (kv_count == NKT) four at a time in tile order, then
+// the local rows four at a time. Unit cost = the key tiles query block A uses plus those B
+// uses (popcounts of the OR of each block's two mask rows), the tensor work of the unit.
+
 __global__ void __launch_bounds__(256) sched_count_kernel(Geom g, const int32_t* __restrict__ kv_count,
                                                           int4* __restrict__ bhcnt) {
   __shared__ int s_nd;
@@ -642,55 +891,122 @@ __global__ void __launch_bounds__(256) sched_count_kernel(Geom g, const int32_t*
   }
 }
 
-// Single thread: exclusive offsets, dense units of every (b, h) before any local unit.
-// bhcnt[i] = (nd, nl, ud, ul) on entry, (dense offset, local offset, ud, ul) on exit.
+// Single thread: exclusive offsets of each (b, h)'s units, head by head; the unit count
+// and a zeroed unit counter for the persistent attention kernel.
+// bhcnt[i] = (nd, nl, ud, ul) on entry, (offset, nd, ud, ul) on exit.
 __global__ void sched_scan_kernel(int BH, int4* __restrict__ bhcnt, int* __restrict__ header) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  int td = 0;
-  for (int i = 0; i < BH; ++i) td += bhcnt[i].z;
-  int od = 0, ol = td;
+  int off = 0;
   for (int i = 0; i < BH; ++i) {
     const int4 c = bhcnt[i];
-    bhcnt[i] = make_int4(od, ol, c.z, c.w);
-    od += c.z;
-    ol += c.w;
+    bhcnt[i] = make_int4(off, c.x, c.z, c.w);
+    off += c.z + c.w;
   }
-  header[1] = ol;
+  header[1] = off;
+  header[2] = 0;
 }
 
-// One warp per (b, h): ordered compaction of each class with ballots. The k-th row of a
-// class becomes query tile k % 4 of unit k / 4 of that class; the last unit of a class
-// may be short (missing tiles -1).
-__global__ void __launch_bounds__(32) sched_write_kernel(Geom g, const int32_t* __restrict__ kv_count,
-                                                         const int4* __restrict__ bhcnt,
-                                                         int* __restrict__ units) {
-  const int bh = blockIdx.x, lane = threadIdx.x;
+constexpr int kSchedThreads = 512;
+constexpr int kSortCap = 2048;      // power of two >= NT/4 + 2 for NT <= 4096
+
+// One block per (b, h): form the units, cost them, sort by decreasing cost (ties by
+// position), write them at the (b, h)'s offset.
+__global__ void __launch_bounds__(kSchedThreads) sched_write_kernel(Geom g, const uint32_t* __restrict__ mask,
+                                                                    const int32_t* __restrict__ kv_count,
+                                                                    const int4* __restrict__ bhcnt,
+                                                                    int* __restrict__ units) {
+  __shared__ int rows[kMaxTiles];            // dense rows, then local rows, each in tile order
+  __shared__ uint32_t key[kSortCap];
+  const int bh = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long base = (long long)bh * g.NT;
-  const int od = bhcnt[bh].x, ol = bhcnt[bh].y;
-  int cd = 0, cl = 0;
-  for (int i0 = 0; i0 < g.NT; i0 += 32) {
-    const int i = i0 + lane;
-    const bool valid = i < g.NT;
-    const bool isd = valid && kv_count[base + i] == g.NT;
-    const bool isl = valid && !isd;
-    const uint32_t bd = __ballot_sync(0xffffffffu, isd), bl = __ballot_sync(0xffffffffu, isl);
-    const uint32_t lt = (1u << lane) - 1u;
-    if (isd || isl) {
-      const int k = (isd ? cd : cl) + __popc((isd ? bd : bl) & lt);
-      int* up = units + (size_t)((isd ? od : ol) + (k >> 2)) * kUnitInts;
-      up[1 + (k & 3)] = i;
-      if ((k & 3) == 0) {
-        up[0] = bh;
-        up[5] = up[6] = up[7] = 0;
-      }
+  const int4 bc = bhcnt[bh];
+  const int off = bc.x, nd = bc.y, ud = bc.z, ul = bc.w, nu = ud + ul;
+  if (warp == 0) {
+    int cd = 0, cl = 0;
+    for (int i0 = 0; i0 < g.NT; i0 += 32) {
+      const int i = i0 + lane;
+      const bool valid = i < g.NT;
+      const bool isd = valid && kv_count[base + i] == g.NT;
+      const bool isl = valid && !isd;
+      const uint32_t bd = __ballot_sync(0xffffffffu, isd), bl = __ballot_sync(0xffffffffu, isl);
+      const uint32_t lt = (1u << lane) - 1u;
+      if (isd) rows[cd + __popc(bd & lt)] = i;
+      if (isl) rows[nd + cl + __popc(bl & lt)] = i;
+      cd += __popc(bd);
+      cl += __popc(bl);
     }
-    cd += __popc(bd);
-    cl += __popc(bl);
   }
-  if (lane == 0) {
-    for (int t = cd & 3; t != 0 && t < 4; ++t) units[(size_t)(od + (cd >> 2)) * kUnitInts + 1 + t] = -1;
-    for (int t = cl & 3; t != 0 && t < 4; ++t) units[(size_t)(ol + (cl >> 2)) * kUnitInts + 1 + t] = -1;
+  __syncthreads();
+  // unit k: rows of its class, four at a time; q_t = -1 past the end of the class
+  auto unit_row = [&](int k, int t) -> int {
+    if (k < ud) {
+      const int r = 4 * k + t;
+      return r < nd ? rows[r] : -1;
+    }
+    const int r = 4 * (k - ud) + t;
+    return r < g.NT - nd ? rows[nd + r] : -1;
+  };
+  const int nwarps = kSchedThreads / 32;
+  for (int k = warp; k < kSortCap; k += nwarps) {
+    if (k >= nu) {
+      if (lane == 0) key[k] = 0xffffffffu;
+      continue;
+    }
+    const int q0 = unit_row(k, 0), q1 = unit_row(k, 1), q2 = unit_row(k, 2), q3 = unit_row(k, 3);
+    int cnt = 0;
+    for (int w = lane; w < g.NW; w += 32) {
+      const uint32_t a0 = mask[(base + q0) * g.NW + w] | (q1 >= 0 ? mask[(base + q1) * g.NW + w] : 0u);
+      const uint32_t b0 = q2 >= 0 ? (mask[(base + q2) * g.NW + w] | (q3 >= 0 ? mask[(base + q3) * g.NW + w] : 0u)) : 0u;
+      cnt += __popc(a0) + __popc(b0);
+    }
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    if (lane == 0) key[k] = ((uint32_t)(16383 - min(cnt, 16383)) << 11) | (uint32_t)k;
   }
+  __syncthreads();
+  // bitonic sort of key[0, kSortCap) ascending: decreasing cost, then position
+  for (int size = 2; size <= kSortCap; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < kSortCap / 2; i += kSchedThreads) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const uint32_t a = key[lo], b = key[hi];
+        if ((a > b) == up) {
+          key[lo] = b;
+          key[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int p = tid; p < nu; p += kSchedThreads) {
+    const int k = (int)(key[p] & 2047u);
+    int* up = units + (size_t)(off + p) * kUnitInts;
+    up[0] = bh;
+    up[1] = unit_row(k, 0);
+    up[2] = unit_row(k, 1);
+    up[3] = unit_row(k, 2);
+    up[4] = unit_row(k, 3);
+    up[5] = 16383 - (int)(key[p] >> 11);
+    up[6] = up[7] = 0;
+  }
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+cudaError_t run_sched(const Geom& g, const uint32_t* mask, const int32_t* kv_count, int* header, int4* bhcnt,
+                      int* units, cudaStream_t s) {
+  const int BH = g.B * g.H;
+  sched_count_kernel<<<BH, 256, 0, s>>>(g, kv_count, bhcnt);
+  sched_scan_kernel<<<1, 32, 0, s>>>(BH, bhcnt, header);
+  sched_write_kernel<<<BH, kSchedThreads, 0, s>>>(g, mask, kv_count, bhcnt, units);
+  count_launches(3);
+  return cudaGetLastError();
 }
 
 template <int D>
@@ -699,7 +1015,14 @@ cudaError_t run_attn(const Geom& g, const CUtensorMap& mq, const CUtensorMap& mk
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int grid = g.B * g.H * units_per_bh(g.NT);
+  // The register split must not ask for more than the launch provides (a larger split
+  // would wait forever in setmaxnreg): refuse a build that was allocated fewer registers.
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, attn_kernel<D>);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs * kAttnThreads < 128 * (2 * kRegsSoftmax + kRegsControl)) return cudaErrorInvalidConfiguration;
+  const long long max_units = (long long)g.B * g.H * units_per_bh(g.NT);
+  const int grid = (int)(max_units < sm_count() ? max_units : sm_count());
   attn_kernel<D><<<grid, kAttnThreads, Cfg<D>::kSmemBytes, s>>>(mq, mk, mv, a);
   count_launches(1);
   return cudaGetLastError();
@@ -735,24 +1058,10 @@ bool make_map(CUtensorMap* m, const void* base, long long rows, int D) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
-cudaError_t launch_sparse_attn(const Geom& g, const __nv_bfloat16* qt, const __nv_bfloat16* kt,
-                               const __nv_bfloat16* vt, const uint32_t* mask, const int32_t* kv_count,
-                               float scale, __nv_bfloat16* out, float* lse, uint8_t* ws, cudaStream_t s) {
-  const WsLayout L = ws_layout(g);
-  int* header = reinterpret_cast<int*>(ws);
-  int4* bhcnt = reinterpret_cast<int4*>(ws + L.bhcnt);
-  int* units = reinterpret_cast<int*>(ws + L.units);
-  const int BH = g.B * g.H;
-
-  sched_count_kernel<<<BH, 256, 0, s>>>(g, kv_count, bhcnt);
-  sched_scan_kernel<<<1, 32, 0, s>>>(BH, bhcnt, header);
-  sched_write_kernel<<<BH, 32, 0, s>>>(g, kv_count, bhcnt, units);
-  count_launches(3);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-
+cudaError_t attn_after_sched(const Geom& g, const __nv_bfloat16* qt, const __nv_bfloat16* kt,
+                             const __nv_bfloat16* vt, const uint32_t* mask, float scale, __nv_bfloat16* out,
+                             float* lse, int* header, const int* units, uint32_t* err, const uint8_t* dense,
+                             int token_rho, cudaStream_t s) {
   const long long rows = (long long)g.B * g.H * g.NT * 64;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, qt, rows, g.d) || !make_map(&mk, kt, rows, g.d) || !make_map(&mv, vt, rows, g.d))
@@ -764,10 +1073,28 @@ cudaError_t launch_sparse_attn(const Geom& g, const __nv_bfloat16* qt, const __n
   a.header = header;
   a.out = out;
   a.lse = lse;
-  a.err = reinterpret_cast<uint32_t*>(ws);
+  a.err = err;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.dense = dense;
+  a.token_rho = token_rho;
   if (g.d == 128) return run_attn<128>(g, mq, mk, mv, a, s);
   return run_attn<64>(g, mq, mk, mv, a, s);
+}
+
+}  // namespace
+
+cudaError_t launch_sparse_attn(const Geom& g, const __nv_bfloat16* qt, const __nv_bfloat16* kt,
+                               const __nv_bfloat16* vt, const uint32_t* mask, const int32_t* kv_count,
+                               float scale, __nv_bfloat16* out, float* lse, uint8_t* ws, cudaStream_t s,
+                               const uint8_t* dense, int token_rho) {
+  const WsLayout L = ws_layout(g);
+  int* header = reinterpret_cast<int*>(ws);
+  int4* bhcnt = reinterpret_cast<int4*>(ws + L.bhcnt);
+  int* units = reinterpret_cast<int*>(ws + L.units);
+  cudaError_t e = run_sched(g, mask, kv_count, header, bhcnt, units, s);
+  if (e != cudaSuccess) return e;
+  return attn_after_sched(g, qt, kt, vt, mask, scale, out, lse, header, units,
+                          reinterpret_cast<uint32_t*>(ws), dense, token_rho, s);
 }
 
 }  // namespace bsa
@@ -796,15 +1123,20 @@ std::mutex g_fixed_mu;
 uint8_t* g_fixed_addr[kMaxDevices] = {};   // device address of g_fixed_scratch, per device
 
 // The array's device address on the current device. In host code the array's name is a
-// host-side stand-in, not a device address, so the first call on each device looks the
-// address up (with that device current) and keeps it.
-cudaError_t fixed_scratch_addr(uint8_t** out) {
+// host-side stand-in, not a device address, so the address is looked up with the device
+// current. It is looked up again on every call made outside a stream capture, so that a
+// context torn down and created again (cudaDeviceReset) never leaves a stale address; a
+// call under capture uses the address its device had at its last call outside capture.
+cudaError_t fixed_scratch_addr(cudaStream_t s, uint8_t** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(s, &cap);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_fixed_mu);
-  if (!g_fixed_addr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone || !g_fixed_addr[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_fixed_scratch);
     if (e != cudaSuccess) return e;
@@ -818,7 +1150,8 @@ cudaError_t fixed_scratch_addr(uint8_t** out) {
 
 size_t fixed_scratch_capacity() { return kFixedScratchBytes; }
 
-// Scratch of one call: 256-byte header (error word, unit count), per-(b, h) counts, units.
+// Scratch of one call: 256-byte header (error word, unit count, unit counter), per-(b, h)
+// counts, units.
 size_t fixed_scratch_need(const Geom& g) {
   const size_t bh = (size_t)g.B * g.H;
   return 256 + align256(bh * sizeof(int4)) + bh * units_per_bh(g.NT) * kUnitInts * sizeof(int);
@@ -830,7 +1163,7 @@ cudaError_t launch_sparse_attn_fixed_scratch(const Geom& g, const __nv_bfloat16*
                                              float* lse, uint32_t* errors, cudaStream_t s) {
   if (fixed_scratch_need(g) > kFixedScratchBytes) return cudaErrorInvalidValue;
   uint8_t* base = nullptr;
-  cudaError_t e = fixed_scratch_addr(&base);
+  cudaError_t e = fixed_scratch_addr(s, &base);
   if (e != cudaSuccess) return e;
   const int BH = g.B * g.H;
   int* header = reinterpret_cast<int*>(base);
@@ -841,27 +1174,10 @@ cudaError_t launch_sparse_attn_fixed_scratch(const Geom& g, const __nv_bfloat16*
   // start at zero; counts and units are fully rewritten by the scheduler before use.
   e = cudaMemsetAsync(base, 0, 256, s);
   if (e != cudaSuccess) return e;
-  sched_count_kernel<<<BH, 256, 0, s>>>(g, kv_count, bhcnt);
-  sched_scan_kernel<<<1, 32, 0, s>>>(BH, bhcnt, header);
-  sched_write_kernel<<<BH, 32, 0, s>>>(g, kv_count, bhcnt, units);
-  count_launches(3);
-  e = cudaGetLastError();
+  e = run_sched(g, mask, kv_count, header, bhcnt, units, s);
   if (e != cudaSuccess) return e;
-
-  const long long rows = (long long)g.B * g.H * g.NT * 64;
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, qt, rows, g.d) || !make_map(&mk, kt, rows, g.d) || !make_map(&mv, vt, rows, g.d))
-    return cudaErrorInvalidValue;
-  AttnArgs a;
-  a.g = g;
-  a.mask = mask;
-  a.units = units;
-  a.header = header;
-  a.out = out;
-  a.lse = lse;
-  a.err = reinterpret_cast<uint32_t*>(base);
-  a.scale_log2 = scale * 1.4426950408889634f;
-  e = (g.d == 128) ? run_attn<128>(g, mq, mk, mv, a, s) : run_attn<64>(g, mq, mk, mv, a, s);
+  e = attn_after_sched(g, qt, kt, vt, mask, scale, out, lse, header, units, reinterpret_cast<uint32_t*>(base),
+                       nullptr, -1, s);
   if (e != cudaSuccess) return e;
   if (errors) e = cudaMemcpyAsync(errors, base, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s);
   return e;

@@ -1,27 +1,33 @@
-"""Discrete-event model of the attention kernel's pipeline protocol (CPU only).
+"""Discrete-event model of the persistent attention kernel's pipeline protocol (CPU only).
 
-The attention kernel hands work between a TMA producer, one MMA-issuing thread per
-sub-unit and two softmax warpgroups through mbarriers that are tested by phase parity.
-This model replays that protocol on the unit lists of real masks under random
-interleavings and checks that it always finishes (no deadlock) and that every read sees
-what it should: each product the key/value tile of its entry (no stale ring stage), the
-softmax S of its own block, each P.V the P of its own block, O holding exactly the blocks
-before it at each P.V and rescale, and every block at the epilogue.
+The attention kernel hands work between a key-stream builder, a TMA producer, one
+MMA-issuing thread with two cursors (query blocks A and B) and two softmax warpgroups of
+four warps, through mbarriers that are tested by phase parity. Units follow one another
+inside a CTA without a barrier between them. This model replays that protocol on
+sequences of units taken from real masks (and on edge cases: a missing query block, query
+tiles that retain nothing, odd stream lengths) under random interleavings, and checks that
+it always finishes (no deadlock) and that every read sees what it should:
+
+  * each Q K^T product the Q of its own unit and the K tiles of its own stream block;
+  * each softmax warp the S of its own block;
+  * each P.V the P of its own block, the V tiles of its block, and O holding exactly the
+    unit's earlier blocks (the unit's first P.V overwrites O);
+  * each rescale O holding exactly the unit's earlier blocks (the softmax rescales right
+    after S of its block is complete, with no wait of its own: the issuer sends Q K^T of a
+    block only after the previous block's P.V, and the pipe runs them in that order);
+  * each epilogue O holding every block of the unit;
+  * the next unit's first P.V only after every warp has read O in the epilogue.
 
 mbarrier semantics modelled: a phase completes when its expected arrival count is
 reached; a parity test for parity P succeeds when the current phase's parity differs from
-P, so a barrier two phases behind the awaited one looks complete. Each issuing thread's
-products run in its issue order, and its commit arrives once the products it issued
-before the commit are done; nothing orders the two issuers' products against each other.
+P (a barrier two phases behind the awaited one looks complete). The issuing thread's
+products run in its issue order, and a commit arrives once the products issued before it
+are done. TMA loads land at a random later time and write their stage when they land.
 
-The protocol: S-full barriers per (sub-unit, S buffer), one P-ready and one P.V-done
-barrier per sub-unit, and a softmax that waits for the previous block's P.V before it
-releases P (and rescales O, when the row max grew). Each sub-unit's softmax runs as four
-independent warps, each with its own rows, so warps of one sub-unit may be at different
-blocks. Deliberately broken variants must be
-caught, which shows the checker can see the hazards: issuers that test only their own next
-entries (ring stages), a softmax that releases P without that wait, an epilogue that waits
-one block early, and QK products three blocks ahead of P.V.
+Deliberately broken variants must be caught, which shows the checker can see the
+hazards: a stage released when the first cursor passes it, a Q K^T issued before the
+previous P.V (overwriting P), a P.V issued before its softmax released P, Q released at
+the unit's first product, and an epilogue that does not wait for the last P.V.
 """
 import random
 
@@ -31,8 +37,8 @@ import pytest
 import _cases as C
 from oracle import bsa_oracle as O
 
-NS = 4          # ring stages, one key tile each
-WARPS = 4       # softmax warps per sub-unit; each warp's 32 threads arrive on P-ready
+NS = 2          # ring stages (two key tiles each)
+WARPS = 4       # softmax warps per query block
 
 
 class Bar:
@@ -54,8 +60,8 @@ class Stale(Exception):
 
 
 def units_from_mask(mask):
-    """Work units of one (b, h): the kernel's grouping of four consecutive rows per class
-    (rows retaining every key tile first), as (union list, used by A, used by B)."""
+    """The kernel's units of one (b, h) (dense rows four at a time, then local rows), as
+    (q tuple, per-stream-entry retention flags [4 bools]) sorted by decreasing cost."""
     nt = mask.shape[0]
     cnt = mask.sum(-1)
     dense = [i for i in range(nt) if cnt[i] == nt]
@@ -64,299 +70,451 @@ def units_from_mask(mask):
     for rows in (dense, local):
         for u0 in range(0, len(rows), 4):
             qs = rows[u0:u0 + 4] + [-1] * (4 - len(rows[u0:u0 + 4]))
-            mk = [mask[q] if q >= 0 else np.zeros(nt, bool) for q in qs]
-            union = np.nonzero(mk[0] | mk[1] | mk[2] | mk[3])[0]
-            out.append((len(union), [bool(mk[0][j] or mk[1][j]) for j in union],
-                        [bool(mk[2][j] or mk[3][j]) for j in union]))
+            out.append(unit_from_rows(qs, [mask[q] if q >= 0 else np.zeros(nt, bool) for q in qs]))
+    out.sort(key=lambda u: -cost(u))
     return out
 
 
-def run_protocol(L, need_a, need_b, seed, careless=False, no_wait=False):
-    """True if the unit finishes; False on deadlock; raises Stale on a wrong read.
+def unit_from_rows(qs, rows):
+    union = np.nonzero(rows[0] | rows[1] | rows[2] | rows[3])[0]
+    return (tuple(qs), [[bool(rows[t][j]) for t in range(4)] for j in union])
 
-    Besides the ring stages, the model tracks what each S buffer holds (S of block it after
-    its QK product, P of block it after the softmax released it) and how many P.V
-    products O has absorbed, and checks every read against them: the softmax reads S of
-    its own block, a P.V reads P of its own block and adds to O holding exactly the
-    blocks before it, a rescale sees O holding exactly the blocks before it, and the
-    epilogue sees every block. From its second block on, a softmax waits for the previous
-    P.V (then may rescale O) before it releases P.
 
-    careless: one issuer per sub-unit that tests only its own next entries (ring hazard).
-    no_wait: the softmax releases P without that wait (it can then run two P-ready phases
-    ahead of the issuer).
-    """
+def cost(unit):
+    qs, ent = unit
+    return sum(e[0] or e[1] for e in ent) + sum(e[2] or e[3] for e in ent)
+
+
+def block_use(ent, c, x):
+    u = 0
+    for h in range(2):
+        i = 2 * c + h
+        if i < len(ent) and (ent[i][2 * x] or ent[i][2 * x + 1]):
+            u |= 1 << h
+    return u
+
+
+def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=False,
+                 no_pfull_wait=False, no_epilogue_wait=False):
+    """True if every unit finishes; False on deadlock; raises Stale on a wrong read."""
     rng = random.Random(seed)
-    need = [need_a, need_b]
-    has = [any(need_a), any(need_b)]
-    users = sum(has)
-    blk = [[i for i in range(L) if need[u][i]] for u in range(2)]
-    n = [len(b) for b in blk]
-    kfull, vfull = [Bar(1) for _ in range(NS)], [Bar(1) for _ in range(NS)]
-    kempty = [Bar(1 if careless else users) for _ in range(NS)]
-    vempty = [Bar(1 if careless else users) for _ in range(NS)]
-    sfull = [Bar(1) for _ in range(4)]          # 2u + b
-    pfull = [Bar(WARPS) for _ in range(2)]      # u (one arrival per warp stands for its 32)
-    odone = [Bar(1) for _ in range(2)]          # u
-    pipe, kload, vload = [[], []], [], []     # one product queue per issuing thread
-    kdata, vdata = [None] * NS, [None] * NS
-    sbuf = [[[None] * WARPS for _ in range(2)] for _ in range(2)]   # per warp's rows: ('S', it) / ('P', it)
-    oblocks = [0, 0]                            # P.V products absorbed by O
-    prod = [0, 'k']
-    ki, vi, qc, pc = [0, 0], [0, 0], [0, 0], [0, 0]
-    # one agent per softmax warp: [block, state]; each warp owns a quarter of the rows
-    sm = [[[0, 'wait_s'] for _ in range(WARPS)] for _ in range(2)]
+    nunits = len(units)
+    # ------------------------------------------------------------------ barriers
+    kfull, kempty = [Bar(1) for _ in range(NS)], [Bar(1) for _ in range(NS)]
+    vfull, vempty = [Bar(1) for _ in range(NS)], [Bar(1) for _ in range(NS)]
+    qfull, qempty = [Bar(1), Bar(1)], [Bar(1), Bar(1)]
+    sfull, pfull, odone = [Bar(1), Bar(1)], [Bar(WARPS), Bar(WARPS)], [Bar(1), Bar(1)]
+    lfull, lempty = [Bar(1), Bar(1)], [Bar(1 + 2 + 2 * WARPS), Bar(1 + 2 + 2 * WARPS)]
+    # ------------------------------------------------------------------ state
+    lists = [None, None]                      # key-stream buffers: unit index or 'end'
+    kdata, vdata, qdata = [None] * NS, [None] * NS, [None, None]
+    sbuf = [[None] * WARPS for _ in range(2)]  # per warp's rows: ('S'|'P', unit, block)
+    obuf = [[None, 0], [None, 0]]             # (unit, blocks absorbed)
+    epi_done = [[-1] * WARPS for _ in range(2)]   # last unit whose epilogue each warp finished
+    inflight = []                             # TMA loads: (barrier, apply)
+    pipe = []                                 # products / commits in issue order
 
-    def pbar(u, it):
-        return pfull[u], it & 1
+    bld = {"it": 0, "next": 0, "done": False}
+    prod = {"it": 0, "state": "list", "unit": None, "c": 0, "qn": [0, 0], "nk": 0, "nv": 0, "x": 0,
+            "done": False}
 
-    def obar(u, it):
-        return odone[u], it & 1
+    def new_cursor():
+        return {"it": 0, "have": False, "done": False, "unit": None, "kc": 0, "vc": 0, "pend": -1,
+                "hasq": False, "qready": False, "qrel": False, "first": True, "gbase": 0, "qn": 0,
+                "pn": 0, "nb": 0}
+    cur = [new_cursor(), new_cursor()]
+    kpass, vpass = [0, 0], [0, 0]
+    sm = [[{"it": 0, "state": "list", "unit": None, "c": 0, "sidx": 0, "nused": 0, "blocks": 0,
+            "done": False} for _ in range(WARPS)] for _ in range(2)]
 
-    def actions():
-        acts = []
-        i = prod[0]
-        if i < L:
-            s, ph = i % NS, ((i // NS) & 1) ^ 1
-            if prod[1] == 'k' and kempty[s].test(ph):
-                acts.append(('load_k',))
-            if prod[1] == 'v' and vempty[s].test(ph):
-                acts.append(('load_v',))
-        if kload:
-            acts.append(('tma_k',))
-        if vload:
-            acts.append(('tma_v',))
-        for u in range(2):
-            if pipe[u]:
-                acts.append(('pipe', u))
-        for u in range(2):
-            if not has[u]:
-                continue
-            if careless:
-                if qc[u] < n[u] and qc[u] - pc[u] < 2:
-                    e = blk[u][qc[u]]
-                    if kfull[e % NS].test((e // NS) & 1):
-                        acts.append(('qk', u))
-                bar, par = pbar(u, pc[u])
-                if pc[u] < qc[u] and bar.test(par):
-                    e = blk[u][pc[u]]
-                    if vfull[e % NS].test((e // NS) & 1):
-                        acts.append(('pv', u))
+    def enqueue(kind, **kw):
+        pipe.append(dict(kind=kind, **kw))
+
+    def unit_of(buf):
+        return lists[buf]
+
+    def nblocks(ui):
+        return (len(units[ui][1]) + 1) // 2
+
+    # ------------------------------------------------------------------ agents
+    def builder_actions():
+        if bld["done"]:
+            return []
+        it = bld["it"]
+        buf = it & 1
+        if it >= 2 and not lempty[buf].test(((it >> 1) - 1) & 1):
+            return []
+
+        def act():
+            if bld["next"] >= nunits:
+                lists[buf] = "end"
+                bld["done"] = True
             else:
-                k = ki[u]
-                if k < L and kfull[k % NS].test((k // NS) & 1):
-                    if not need[u][k]:
-                        acts.append(('k_arrive', u))
-                    elif qc[u] - pc[u] < 2:
-                        acts.append(('qk', u))
-                v = vi[u]
-                if v < ki[u] and vfull[v % NS].test((v // NS) & 1):
-                    if not need[u][v]:
-                        acts.append(('v_arrive', u))
-                    else:
-                        bar, par = pbar(u, pc[u])
-                        if bar.test(par):
-                            acts.append(('pv', u))
-            for w in range(WARPS):
-                it, st = sm[u][w]
-                if it < n[u]:
-                    if st == 'wait_s' and sfull[2 * u + (it & 1)].test((it >> 1) & 1):
-                        acts.append(('softmax_s', u, w))
-                    if st == 'wait_o':
-                        bar, par = obar(u, it - 1)
-                        if bar.test(par):
-                            acts.append(('softmax_rescale', u, w))
-                    if st == 'release':
-                        acts.append(('softmax_p', u, w))
-                elif st != 'done':
-                    bar, par = obar(u, n[u] - 1)
-                    if n[u] == 0 or bar.test(par):
-                        acts.append(('epilogue', u, w))
+                lists[buf] = bld["next"]
+                bld["next"] += 1
+            lfull[buf].arrive()
+            bld["it"] += 1
+        return [act]
+
+    def producer_actions():
+        p = prod
+        if p["done"]:
+            return []
+        if p["state"] == "list":
+            buf = p["it"] & 1
+            if not lfull[buf].test((p["it"] >> 1) & 1):
+                return []
+
+            def act():
+                ui = unit_of(buf)
+                if ui == "end":
+                    p["done"] = True
+                    return
+                p["unit"], p["state"], p["x"], p["c"] = ui, "q", 0, 0
+            return [act]
+        ui = p["unit"]
+        qs, ent = units[ui]
+        if p["state"] == "q":
+            x = p["x"]
+            if x == 2:
+                def act():
+                    p["state"] = "k"
+                return [act]
+            if qs[2 * x] < 0:
+                def act():
+                    p["x"] += 1
+                return [act]
+            if p["qn"][x] > 0 and not qempty[x].test((p["qn"][x] - 1) & 1):
+                return []
+
+            def act():
+                inflight.append((qfull[x], lambda x=x, ui=ui: qdata.__setitem__(x, ui)))
+                p["qn"][x] += 1
+                p["x"] += 1
+            return [act]
+        nb = nblocks(ui)
+        if p["c"] == nb:
+            def act():
+                lempty[p["it"] & 1].arrive()
+                p["it"] += 1
+                p["state"] = "list"
+            return [act]
+        if p["state"] == "k":
+            s, ph = p["nk"] % NS, ((p["nk"] // NS) & 1) ^ 1
+            if not kempty[s].test(ph):
+                return []
+
+            def act():
+                tag = (ui, p["c"])
+                inflight.append((kfull[s], lambda s=s, tag=tag: kdata.__setitem__(s, tag)))
+                p["nk"] += 1
+                p["state"] = "v"
+            return [act]
+        s, ph = p["nv"] % NS, ((p["nv"] // NS) & 1) ^ 1
+        if not vempty[s].test(ph):
+            return []
+
+        def act():
+            tag = (ui, p["c"])
+            inflight.append((vfull[s], lambda s=s, tag=tag: vdata.__setitem__(s, tag)))
+            p["nv"] += 1
+            p["c"] += 1
+            p["state"] = "k"
+        return [act]
+
+    def release(passes, empty, x, gi):
+        passes[x] = gi + 1
+        if early_release or passes[x ^ 1] >= gi + 1:
+            enqueue("commit", bar=empty[gi % NS])
+
+    def cursor_actions(x):
+        cu = cur[x]
+        if cu["done"]:
+            return []
+        acts = []
+        if not cu["have"]:
+            buf = cu["it"] & 1
+            if lfull[buf].test((cu["it"] >> 1) & 1):
+                def act():
+                    ui = unit_of(buf)
+                    if ui == "end":
+                        cu["done"] = True
+                        return
+                    cu.update(have=True, unit=ui, kc=0, vc=0, pend=-1, hasq=units[ui][0][2 * x] >= 0,
+                              qready=False, qrel=False, first=True, nb=nblocks(ui))
+                acts.append(act)
+            return acts
+        ui = cu["unit"]
+        qs, ent = units[ui]
+        nb = cu["nb"]
+        if cu["kc"] < nb:
+            c = cu["kc"]
+            u = block_use(ent, c, x) if cu["hasq"] else 0
+            gi = cu["gbase"] + c
+            s, fph = gi % NS, (gi // NS) & 1
+            qok = cu["qready"] or qfull[x].test(cu["qn"] & 1)
+            if u == 0:
+                ok = kfull[s].test(fph)
+            else:
+                ok = (cu["pend"] < 0 or qk_before_pv) and qok and kfull[s].test(fph)
+            if ok:
+                def act(u=u, c=c, gi=gi, s=s, qok=qok):
+                    if u:
+                        cu["qready"] = True
+                        enqueue("qk", x=x, unit=ui, block=c, stage=s)
+                        enqueue("commit", bar=sfull[x])
+                        cu["pend"] = c
+                        if early_q and not cu["qrel"]:
+                            enqueue("commit", bar=qempty[x])
+                            cu["qrel"] = True
+                    release(kpass, kempty, x, gi)
+                    cu["kc"] += 1
+                    if cu["kc"] == nb and cu["hasq"] and cu["qready"] and not cu["qrel"]:
+                        enqueue("commit", bar=qempty[x])
+                        cu["qrel"] = True
+                acts.append(act)
+        if cu["vc"] < cu["kc"]:
+            c = cu["vc"]
+            gi = cu["gbase"] + c
+            s, fph = gi % NS, (gi // NS) & 1
+            if c == cu["pend"]:
+                ok = (no_pfull_wait or pfull[x].test(cu["pn"] & 1)) and vfull[s].test(fph)
+            else:
+                ok = vfull[s].test(fph)
+            if ok:
+                def act(c=c, gi=gi, s=s):
+                    if c == cu["pend"]:
+                        enqueue("pv", x=x, unit=ui, block=c, stage=s, first=cu["first"],
+                                ordinal=cu["pn"])
+                        enqueue("commit", bar=odone[x])
+                        cu["first"] = False
+                        cu["pn"] += 1
+                        cu["pend"] = -1
+                    release(vpass, vempty, x, gi)
+                    cu["vc"] += 1
+                acts.append(act)
+        if cu["kc"] == nb and cu["vc"] == nb:
+            if not cu["hasq"] or cu["qrel"] or cu["qready"] or qfull[x].test(cu["qn"] & 1):
+                def act():
+                    if cu["hasq"] and not cu["qrel"]:
+                        enqueue("commit", bar=qempty[x])
+                        cu["qrel"] = True
+                    if cu["hasq"]:
+                        cu["qn"] += 1
+                    lempty[cu["it"] & 1].arrive()
+                    cu["it"] += 1
+                    cu["have"] = False
+                    cu["gbase"] += nb
+                acts.append(act)
         return acts
 
-    def last_user(u, e, cursor):
-        o = 1 - u
-        return not need[o][e] or not has[o] or cursor[o] >= n[o] or blk[o][cursor[o]] > e
+    def pipe_actions():
+        if not pipe:
+            return []
 
-    while True:
-        acts = actions()
-        finished = (prod[0] >= L and all(sm[u][w][1] == 'done' or not has[u] for u in range(2) for w in range(WARPS))
-                    and all(pc[u] >= n[u] for u in range(2)))
-        if finished and not pipe[0] and not pipe[1] and not kload and not vload:
-            return True
+        def act():
+            op = pipe.pop(0)
+            k = op["kind"]
+            if k == "commit":
+                op["bar"].arrive()
+            elif k == "qk":
+                x, ui, c, s = op["x"], op["unit"], op["block"], op["stage"]
+                if qdata[x] != ui:
+                    raise Stale(f"QK of unit {ui} reads Q of {qdata[x]}")
+                if kdata[s] != (ui, c):
+                    raise Stale(f"QK of {(ui, c)} reads K {kdata[s]}")
+                for w in range(WARPS):
+                    if sbuf[x][w] is not None and sbuf[x][w][0] == "S":
+                        raise Stale(f"S of {sbuf[x][w][1:]} overwritten before its softmax read it")
+                    sbuf[x][w] = ("S", ui, c)
+            else:
+                x, ui, c, s = op["x"], op["unit"], op["block"], op["stage"]
+                if vdata[s] != (ui, c):
+                    raise Stale(f"PV of {(ui, c)} reads V {vdata[s]}")
+                for w in range(WARPS):
+                    if sbuf[x][w] != ("P", ui, c):
+                        raise Stale(f"PV of {(ui, c)} reads {sbuf[x][w]} (warp {w})")
+                if op["first"]:
+                    if any(epi_done[x][w] < (obuf[x][0] if obuf[x][0] is not None else -1)
+                           for w in range(WARPS)):
+                        raise Stale("O overwritten before every warp read the previous unit's O")
+                    obuf[x] = [ui, 1]
+                else:
+                    if obuf[x][0] != ui or obuf[x][1] != op["ordinal_in_unit"]:
+                        raise Stale(f"PV of {(ui, c)} adds to O {obuf[x]}")
+                    obuf[x][1] += 1
+        return [act]
+
+    def softmax_actions(x, w):
+        st = sm[x][w]
+        if st["done"]:
+            return []
+        if st["state"] == "list":
+            buf = st["it"] & 1
+            if not lfull[buf].test((st["it"] >> 1) & 1):
+                return []
+
+            def act():
+                ui = unit_of(buf)
+                if ui == "end":
+                    st["done"] = True
+                    return
+                st.update(unit=ui, c=0, nused=0, blocks=0, state="blocks")
+            return [act]
+        ui = st["unit"]
+        qs, ent = units[ui]
+        nb = nblocks(ui)
+        if st["state"] == "blocks":
+            while st["c"] < nb and (qs[2 * x] < 0 or block_use(ent, st["c"], x) == 0):
+                st["c"] += 1
+            if st["c"] == nb:
+                def act():
+                    lempty[st["it"] & 1].arrive()
+                    st["state"] = "epi"
+                return [act]
+            if not sfull[x].test(st["sidx"] & 1):
+                return []
+
+            def act():
+                c = st["c"]
+                if sbuf[x][w] != ("S", ui, c):
+                    raise Stale(f"softmax {(ui, c)} reads {sbuf[x][w]}")
+                st["state"] = "resc" if (st["nused"] > 0 and rng.random() < 0.3) else "release"
+            return [act]
+        if st["state"] == "resc":
+            def act():
+                if obuf[x] != [ui, st["nused"]]:
+                    raise Stale(f"rescale in {(ui, st['c'])} sees O {obuf[x]}")
+                st["state"] = "release"
+            return [act]
+        if st["state"] == "release":
+            def act():
+                sbuf[x][w] = ("P", ui, st["c"])
+                pfull[x].arrive()
+                st["sidx"] += 1
+                st["nused"] += 1
+                st["c"] += 1
+                st["state"] = "blocks"
+            return [act]
+        # epilogue
+        if st["nused"] > 0 and not no_epilogue_wait and not odone[x].test((st["sidx"] - 1) & 1):
+            return []
+
+        def act():
+            if st["nused"] > 0 and obuf[x] != [ui, st["nused"]]:
+                raise Stale(f"epilogue of unit {ui} sees O {obuf[x]}")
+            epi_done[x][w] = ui
+            st["it"] += 1
+            st["state"] = "list"
+        return [act]
+
+    # PV ordinals inside a unit: filled at enqueue time from the cursor's count in the unit
+    unit_pv = {}
+
+    def fix_ordinals():
+        for op in pipe:
+            if op["kind"] == "pv" and "ordinal_in_unit" not in op:
+                key = (op["x"], op["unit"])
+                op["ordinal_in_unit"] = unit_pv.get(key, 0)
+                unit_pv[key] = op["ordinal_in_unit"] + 1
+
+    for _ in range(2_000_000):
+        fix_ordinals()
+        acts = builder_actions() + producer_actions() + cursor_actions(0) + cursor_actions(1) + pipe_actions()
+        for x in range(2):
+            for w in range(WARPS):
+                acts += softmax_actions(x, w)
+        if inflight:
+            def land():
+                i = rng.randrange(len(inflight))
+                b, apply = inflight.pop(i)
+                apply()
+                b.arrive()
+            acts.append(land)
         if not acts:
-            return False
-        a = rng.choice(acts)
-        kind = a[0]
-        if kind == 'load_k':
-            kload.append((prod[0] % NS, prod[0]))
-            prod[1] = 'v'
-        elif kind == 'load_v':
-            vload.append((prod[0] % NS, prod[0]))
-            prod[1] = 'k'
-            prod[0] += 1
-        elif kind == 'tma_k':
-            s, e = kload.pop(0)
-            kdata[s] = e
-            kfull[s].arrive()
-        elif kind == 'tma_v':
-            s, e = vload.pop(0)
-            vdata[s] = e
-            vfull[s].arrive()
-        elif kind == 'pipe':
-            op = pipe[a[1]].pop(0)
-            if op[0] == 'commit':
-                op[1].arrive()
-            elif op[0] == 'qk':
-                _, u, it, s, e = op
-                if kdata[s] != e:
-                    raise Stale(f"QK of entry {e} read K stage {s} holding {kdata[s]}")
-                if it >= 2 and oblocks[u] < it - 1:
-                    raise Stale(f"S of block {it} overwrote P of block {it - 2} before its P.V")
-                sbuf[u][it & 1] = [('S', it)] * WARPS
-            else:
-                _, u, it, s, e = op
-                if vdata[s] != e:
-                    raise Stale(f"P.V of entry {e} read V stage {s} holding {vdata[s]}")
-                if sbuf[u][it & 1] != [('P', it)] * WARPS:
-                    raise Stale(f"P.V of block {it} read {sbuf[u][it & 1]}")
-                if oblocks[u] != it:
-                    raise Stale(f"P.V of block {it} added to O holding {oblocks[u]} blocks")
-                oblocks[u] += 1
-        elif kind == 'qk':
-            u = a[1]
-            e = blk[u][qc[u]]
-            s = e % NS
-            pipe[u] += [('qk', u, qc[u], s, e), ('commit', sfull[2 * u + (qc[u] & 1)])]
-            qc[u] += 1
-            if careless:
-                if last_user(u, e, qc):
-                    pipe[u].append(('commit', kempty[s]))
-            else:
-                pipe[u].append(('commit', kempty[s]))
-                ki[u] += 1
-        elif kind == 'k_arrive':
-            u = a[1]
-            kempty[ki[u] % NS].arrive()
-            ki[u] += 1
-        elif kind == 'pv':
-            u = a[1]
-            e = blk[u][pc[u]]
-            s = e % NS
-            pipe[u] += [('pv', u, pc[u], s, e), ('commit', obar(u, pc[u])[0])]
-            pc[u] += 1
-            if careless:
-                if last_user(u, e, pc):
-                    pipe[u].append(('commit', vempty[s]))
-            else:
-                pipe[u].append(('commit', vempty[s]))
-                vi[u] += 1
-        elif kind == 'v_arrive':
-            u = a[1]
-            vempty[vi[u] % NS].arrive()
-            vi[u] += 1
-        elif kind == 'softmax_s':
-            u, w = a[1], a[2]
-            it = sm[u][w][0]
-            if sbuf[u][it & 1][w] != ('S', it):
-                raise Stale(f"softmax warp {w} of block {it} read {sbuf[u][it & 1][w]}")
-            sm[u][w][1] = 'wait_o' if it > 0 and not no_wait else 'release'
-        elif kind == 'softmax_rescale':
-            u, w = a[1], a[2]
-            if oblocks[u] != sm[u][w][0]:
-                raise Stale(f"rescale at block {sm[u][w][0]} saw O holding {oblocks[u]} blocks")
-            sm[u][w][1] = 'release'
-        elif kind == 'softmax_p':
-            u, w = a[1], a[2]
-            it = sm[u][w][0]
-            sbuf[u][it & 1][w] = ('P', it)
-            bar, _ = pbar(u, it)
-            bar.arrive()
-            sm[u][w] = [it + 1, 'wait_s']
-        elif kind == 'epilogue':
-            u, w = a[1], a[2]
-            if oblocks[u] != n[u]:
-                raise Stale(f"epilogue read O holding {oblocks[u]} of {n[u]} blocks")
-            sm[u][w][1] = 'done'
+            done = bld["done"] and prod["done"] and all(c["done"] for c in cur) and \
+                all(s["done"] for xs in sm for s in xs) and not pipe and not inflight
+            return done
+        rng.choice(acts)()
+    raise AssertionError("model did not terminate")
 
 
-def _case_units(name):
-    w, q, k, v, diff = C.inputs(name)
-    ref = C.oracle_mask(w, O.reorder(O.to_f64(q), w.T, w.Hs, w.Ws),
-                        O.reorder(O.to_f64(k), w.T, w.Hs, w.Ws), diff.numpy())
-    m = ref["mask"]
-    return [u for b in range(m.shape[0]) for h in range(m.shape[1]) for u in units_from_mask(m[b, h])]
+def _mask_units(name, heads=2, **over):
+    w, q, k, v, diff = C.inputs(name, tuple(over.items()))
+    qt64, kt64 = (O.reorder(O.to_f64(x), w.T, w.Hs, w.Ws) for x in (q, k))
+    m = C.oracle_mask(w, qt64[:, :heads], kt64[:, :heads], diff.numpy())["mask"]
+    out = []
+    for h in range(heads):
+        out += units_from_mask(m[0, h])
+    return out
 
 
-@pytest.mark.parametrize("name", ["tiny", "tiny_ragged", "small128", "ragged128", "budget128"])
-def test_two_issuer_protocol_finishes_and_reads_the_right_tiles(name):
-    for L, na, nb in _case_units(name):
-        for seed in range(12):
-            assert run_protocol(L, na, nb, seed), (name, L, seed)
+def _edge_units():
+    nt = 9
+    rng = np.random.default_rng(3)
+    rows = [rng.random(nt) < 0.4 for _ in range(4)]
+    empty = np.zeros(nt, bool)
+    one = np.zeros(nt, bool)
+    one[4] = True
+    return [
+        unit_from_rows((0, 1, 2, 3), rows),                       # random rows
+        unit_from_rows((0, 1, -1, -1), [rows[0], rows[1], empty, empty]),   # no query block B
+        unit_from_rows((0, -1, -1, -1), [one, empty, empty, empty]),        # one tile, one key tile
+        unit_from_rows((0, 1, 2, 3), [empty, empty, rows[2], rows[3]]),     # A retains nothing
+        unit_from_rows((0, 1, 2, 3), [one, empty, empty, one]),             # odd stream, shared tile
+        unit_from_rows((0, 1, 2, -1), [~empty, ~empty, ~empty, empty]),     # dense rows
+    ]
 
 
-def test_random_sparse_unit_lists():
-    rng = np.random.default_rng(7)
-    for trial in range(150):
-        L = int(rng.integers(1, 40))
-        na = list(rng.random(L) < rng.uniform(0.1, 0.9))
-        nb = list(rng.random(L) < rng.uniform(0.1, 0.9))
-        for j in range(L):                       # every union entry has a user
-            if not (na[j] or nb[j]):
-                (na if rng.random() < 0.5 else nb)[j] = True
-        if trial % 5 == 0:                       # units without a second sub-unit
-            na, nb = [True] * L, [False] * L
-        for seed in range(4):
-            assert run_protocol(L, na, nb, seed), (trial, L, seed)
+@pytest.mark.parametrize("seed", range(6))
+def test_protocol_on_real_mask_units(seed):
+    units = _mask_units("small128")
+    rng = random.Random(seed)
+    pick = units[:]
+    rng.shuffle(pick)
+    assert run_protocol(pick[:10], seed)
 
 
-def test_careless_protocol_is_caught():
-    """Testing only a sub-unit's own next entries lets it run two ring phases ahead of
-    the producer: the checker must report a deadlock or a stale-tile read."""
-    caught = 0
-    for L, na, nb in _case_units("budget128"):
-        for seed in range(12):
-            try:
-                caught += not run_protocol(L, na, nb, seed, careless=True)
-            except Stale:
-                caught += 1
-    assert caught > 0
+@pytest.mark.parametrize("seed", range(8))
+def test_protocol_on_edge_units(seed):
+    units = _edge_units()
+    rng = random.Random(100 + seed)
+    seq = [units[rng.randrange(len(units))] for _ in range(8)]
+    assert run_protocol(seq, seed)
 
 
-def test_release_without_waiting_is_caught():
-    """Without the wait for the previous P.V, a softmax can complete two phases of its
-    single P-ready barrier before the issuer tests the first: the parity test aliases, and
-    the checker must report a deadlock or a wrong read."""
-    caught = 0
-    for L, na, nb in _case_units("budget128"):
-        for seed in range(12):
-            try:
-                caught += not run_protocol(L, na, nb, seed, no_wait=True)
-            except Stale:
-                caught += 1
-    assert caught > 0
+@pytest.mark.parametrize("seed", range(3))
+def test_protocol_budget_units(seed):
+    units = _mask_units("budget128", heads=1)
+    assert run_protocol(units[:8], seed)
 
 
-@pytest.mark.parametrize("mutation", ["epilogue_one_block_early", "qk_three_blocks_ahead"])
-def test_broken_waits_are_caught(mutation):
-    """The same checker on two one-line mistakes: an epilogue that waits for the last P.V
-    but one, and QK products allowed three blocks ahead of P.V (S would overwrite P before
-    its product)."""
-    import inspect
-    import textwrap
-    src = inspect.getsource(run_protocol)
-    a, b = {
-        "epilogue_one_block_early": ("bar, par = obar(u, n[u] - 1)", "bar, par = obar(u, max(n[u] - 2, 0))"),
-        "qk_three_blocks_ahead": ("elif qc[u] - pc[u] < 2:", "elif qc[u] - pc[u] < 3:"),
-    }[mutation]
-    assert a in src
-    ns = dict(globals())
-    exec(textwrap.dedent(src.replace(a, b)), ns)
-    caught = 0
-    for L, na, nb in _case_units("budget128"):
-        for seed in range(12):
-            try:
-                caught += not ns["run_protocol"](L, na, nb, seed)
-            except Stale:
-                caught += 1
-    assert caught > 0
+def _catches(**broken):
+    units = _mask_units("small128")[:6] + _edge_units()
+    for seed in range(40):
+        try:
+            if not run_protocol(units, seed, **broken):
+                return True
+        except Stale:
+            return True
+    return False
+
+
+def test_model_catches_early_stage_release():
+    assert _catches(early_release=True)
+
+
+def test_model_catches_qk_before_pv():
+    assert _catches(qk_before_pv=True)
+
+
+def test_model_catches_early_q_release():
+    assert _catches(early_q=True)
+
+
+def test_model_catches_pv_before_p():
+    assert _catches(no_pfull_wait=True)
+
+
+def test_model_catches_epilogue_without_wait():
+    assert _catches(no_epilogue_wait=True)
