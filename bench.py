@@ -110,9 +110,9 @@ def _valid_token_flops(g, mask_i32):
 
 
 def _mask_bytes(g):
-    """Algorithmic bytes of the mask build: the valid Q and K tokens read once (the pooling
-    pass), the bitmask and kv_count written."""
-    return 2 * g.B * g.N * g.H * g.d * 2 + g.B * g.H * g.NT * (g.NW + 1) * 4
+    """Algorithmic bytes of the mask build from pooled means: qbar and kbar read once, the
+    bitmask and kv_count written (the pooling itself rides on the reorder's pass)."""
+    return 2 * g.B * g.H * g.NT * g.d * 4 + g.B * g.H * g.NT * (g.NW + 1) * 4
 
 
 def _workload_text(w):
@@ -394,10 +394,10 @@ def run_ours(args):
     t_start, t_end = ev(), ev()
     t_start.record(stream)
     for s in range(args.steps):
-        bsa.reorder(g, q, bufs.qt)
-        bsa.reorder(g, k, bufs.kt)
+        bsa.reorder_pool(g, q, bufs.qt, bufs.qbar)
+        bsa.reorder_pool(g, k, bufs.kt, bufs.kbar)
         bsa.reorder(g, v, bufs.vt)
-        bsa.build_mask(g, p, bufs.qt, bufs.kt, diff, bufs.mask, bufs.kv_count, bufs.ws)
+        bsa.build_mask_pooled(g, p, bufs.qbar, bufs.kbar, diff, bufs.mask, bufs.kv_count, bufs.ws)
         attn_ev[s][0].record(stream)
         bsa.sparse_attn_fwd(g, bufs.qt, bufs.kt, bufs.vt, bufs.mask, bufs.kv_count, None,
                             bufs.out, bufs.lse, bufs.ws)
@@ -596,8 +596,9 @@ def run_report(args):
         torch.cuda.synchronize()
         retained = int(b.kv_count.sum().item())
         valid_flops = _valid_token_flops(g, b.mask)
-        stages = {"reorder_qkv": lambda: [bsa.reorder(g, x, y) for x, y in ((q, b.qt), (k, b.kt), (v, b.vt))],
-                  "build_mask": lambda: bsa.build_mask(g, p, b.qt, b.kt, diff, b.mask, b.kv_count, b.ws),
+        stages = {"reorder_qkv": lambda: (bsa.reorder_pool(g, q, b.qt, b.qbar), bsa.reorder_pool(g, k, b.kt, b.kbar),
+                                          bsa.reorder(g, v, b.vt)),
+                  "build_mask": lambda: bsa.build_mask_pooled(g, p, b.qbar, b.kbar, diff, b.mask, b.kv_count, b.ws),
                   "sparse_attn": lambda: bsa.sparse_attn_fwd(g, b.qt, b.kt, b.vt, b.mask, b.kv_count, None,
                                                              b.out, b.lse, b.ws)}
         res, pct = {}, {}
@@ -634,7 +635,8 @@ def run_report(args):
         e1.record()
         torch.cuda.synchronize()
         dense_ms = e0.elapsed_time(e1) / nd
-        qkv_bytes = 3 * (g.B * g.N * g.H * g.d * 2 + g.B * g.H * g.NT * 64 * g.d * 2)
+        # raster read + tile-major write of Q, K, V, and the pooled means of Q and K
+        qkv_bytes = 3 * (g.B * g.N * g.H * g.d * 2 + g.B * g.H * g.NT * 64 * g.d * 2) + 2 * g.B * g.H * g.NT * g.d * 4
         print(json.dumps({
             "workload": name, "B": g.B, "H": g.H, "d": g.d, "grid": [g.T, g.Hs, g.Ws], "tiles": g.NT,
             "retained_tile_fraction": retained / dense_pairs, "ms": res,

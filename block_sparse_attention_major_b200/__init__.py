@@ -6,9 +6,13 @@ libbsa.so is missing or the device is not a B200, the calls raise.
 
 Entry points (same names as the C ABI in include/bsa.h):
     reorder(g, x)                   raster [B,N,H,d] -> tile-major [B,H,NT,64,d]
+    reorder_pool(g, x)              the same, plus the per-tile means fp32 [B,H,NT,d]
     unreorder(g, xt)                the inverse
     build_mask(g, p, qt, kt, difficulty)     -> (mask uint32 [B,H,NQT,W], kv_count int32)
+    build_mask_pooled(g, p, qbar, kbar, difficulty)   the same from the per-tile means
     sparse_attn_fwd(g, qt, kt, vt, mask, kv_count)  -> (out bf16 [B,N,H,d], lse fp32 [B,H,N])
+    sparse_attn_fwd_token(g, qt, kt, vt, mask, kv_count, dense, token_radius)
+                                    the same under a token-level circular support
     forward(g, p, q, k, v, difficulty)       the whole path, raster in, raster out
 """
 from __future__ import annotations
@@ -76,10 +80,19 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.bsa_reorder.argtypes = [G, vp, vp, vp]
         lib.bsa_unreorder.restype = ctypes.c_int
         lib.bsa_unreorder.argtypes = [G, vp, vp, vp]
+        lib.bsa_reorder_pool.restype = ctypes.c_int
+        lib.bsa_reorder_pool.argtypes = [G, vp, vp, vp, vp]
+        lib.bsa_build_mask_pooled.restype = ctypes.c_int
+        lib.bsa_build_mask_pooled.argtypes = [G, P, vp, vp, vp, vp, vp, vp, sz, vp]
         lib.bsa_build_mask.restype = ctypes.c_int
         lib.bsa_build_mask.argtypes = [G, P, vp, vp, vp, vp, vp, vp, sz, vp]
         lib.bsa_sparse_attn_fwd.restype = ctypes.c_int
         lib.bsa_sparse_attn_fwd.argtypes = [G, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, sz, vp]
+        lib.bsa_sparse_attn_fwd_token.restype = ctypes.c_int
+        lib.bsa_sparse_attn_fwd_token.argtypes = [G, vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_float, vp,
+                                                  vp, vp, sz, vp]
+        lib.bsa_route_flags_offset.restype = sz
+        lib.bsa_route_flags_offset.argtypes = [G]
         lib.bsa_sparse_attn_fwd_fixed_scratch.restype = ctypes.c_int
         lib.bsa_sparse_attn_fwd_fixed_scratch.argtypes = [G, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp,
                                                           vp, vp]
@@ -232,6 +245,21 @@ def reorder(g: Geometry, x: torch.Tensor, xt: torch.Tensor | None = None, stream
     return xt
 
 
+def reorder_pool(g: Geometry, x: torch.Tensor, xt: torch.Tensor | None = None,
+                 xbar: torch.Tensor | None = None, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Tile-major reorder and the per-tile means of the valid tokens, in one pass."""
+    _need(x, torch.bfloat16, (g.B, g.N, g.H, g.d), "x")
+    if xt is None:
+        xt = torch.empty((g.B, g.H, g.NT, 64, g.d), dtype=torch.bfloat16, device=x.device)
+    if xbar is None:
+        xbar = torch.empty((g.B, g.H, g.NT, g.d), dtype=torch.float32, device=x.device)
+    _need(xt, torch.bfloat16, (g.B, g.H, g.NT, 64, g.d), "xt")
+    _need(xbar, torch.float32, (g.B, g.H, g.NT, g.d), "xbar")
+    _run("bsa_reorder_pool", _device_of(x, xt, xbar), stream,
+         lambda s: load_library().bsa_reorder_pool(ctypes.byref(g.c()), _ptr(x), _ptr(xt), _ptr(xbar), s))
+    return xt, xbar
+
+
 def unreorder(g: Geometry, xt: torch.Tensor, x: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     _need(xt, torch.bfloat16, (g.B, g.H, g.NT, 64, g.d), "xt")
     if x is None:
@@ -267,6 +295,33 @@ def build_mask(g: Geometry, p: MaskParams, qt: torch.Tensor, kt: torch.Tensor,
     return mask, kv_count
 
 
+def build_mask_pooled(g: Geometry, p: MaskParams, qbar: torch.Tensor, kbar: torch.Tensor,
+                      difficulty: torch.Tensor, mask: torch.Tensor | None = None,
+                      kv_count: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                      stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """build_mask from the per-tile means that reorder_pool wrote."""
+    _need(qbar, torch.float32, (g.B, g.H, g.NT, g.d), "qbar")
+    _need(kbar, torch.float32, (g.B, g.H, g.NT, g.d), "kbar")
+    _need(difficulty, torch.float32, (g.B, g.NT), "difficulty")
+    dev = qbar.device
+    if mask is None:
+        mask = torch.empty((g.B, g.H, g.NT, g.NW), dtype=torch.int32, device=dev)
+    if kv_count is None:
+        kv_count = torch.empty((g.B, g.H, g.NT), dtype=torch.int32, device=dev)
+    _need(mask, torch.int32, (g.B, g.H, g.NT, g.NW), "mask")
+    _need(kv_count, torch.int32, (g.B, g.H, g.NT), "kv_count")
+    if ws is None:
+        ws = alloc_workspace(g, dev)
+    _need_ws(ws)
+    pc = p.c()
+    _run("bsa_build_mask_pooled", _device_of(qbar, kbar, difficulty, mask, kv_count, ws), stream,
+         lambda s: load_library().bsa_build_mask_pooled(ctypes.byref(g.c()), ctypes.byref(pc), _ptr(qbar),
+                                                        _ptr(kbar), _ptr(difficulty), _ptr(mask),
+                                                        _ptr(kv_count), _ptr(ws), ctypes.c_size_t(ws.numel()),
+                                                        s))
+    return mask, kv_count
+
+
 def sparse_attn_fwd(g: Geometry, qt: torch.Tensor, kt: torch.Tensor, vt: torch.Tensor,
                     mask: torch.Tensor, kv_count: torch.Tensor, scale: float | None = None,
                     out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
@@ -293,6 +348,49 @@ def sparse_attn_fwd(g: Geometry, qt: torch.Tensor, kt: torch.Tensor, vt: torch.T
                                                       _ptr(mask), _ptr(kv_count), ctypes.c_float(sc),
                                                       _ptr(out), _ptr(lse), _ptr(ws),
                                                       ctypes.c_size_t(ws.numel()), s))
+    return out, lse
+
+
+def route_flags(g: Geometry, ws: torch.Tensor) -> torch.Tensor:
+    """The route flags (uint8 [B, NQT], 1 = dense row) that build_mask left in `ws`: a view
+    into the workspace, valid until the workspace is given to another build_mask."""
+    _need_ws(ws)
+    off = int(load_library().bsa_route_flags_offset(ctypes.byref(g.c())))
+    if off == 0:
+        raise ValueError("invalid geometry")
+    return ws[off:off + g.B * g.NT].view(g.B, g.NT)
+
+
+def sparse_attn_fwd_token(g: Geometry, qt: torch.Tensor, kt: torch.Tensor, vt: torch.Tensor,
+                          mask: torch.Tensor, kv_count: torch.Tensor, dense: torch.Tensor,
+                          token_radius: int, scale: float | None = None, out: torch.Tensor | None = None,
+                          lse: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                          want_lse: bool = True, stream=None) -> tuple[torch.Tensor, torch.Tensor | None]:
+    """Block-sparse attention under a token-level circular support of radius token_radius
+    (tokens): local rows (dense == 0) see their window tiles token by token, as
+    bsa_sparse_attn_fwd_token in include/bsa.h describes."""
+    for name, t in (("qt", qt), ("kt", kt), ("vt", vt)):
+        _need(t, torch.bfloat16, (g.B, g.H, g.NT, 64, g.d), name)
+    _need(mask, torch.int32, (g.B, g.H, g.NT, g.NW), "mask")
+    _need(kv_count, torch.int32, (g.B, g.H, g.NT), "kv_count")
+    _need(dense, torch.uint8, (g.B, g.NT), "dense")
+    dev = qt.device
+    if out is None:
+        out = torch.empty((g.B, g.N, g.H, g.d), dtype=torch.bfloat16, device=dev)
+    _need(out, torch.bfloat16, (g.B, g.N, g.H, g.d), "out")
+    if want_lse and lse is None:
+        lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _need(lse, torch.float32, (g.B, g.H, g.N), "lse")
+    if ws is None:
+        ws = alloc_workspace(g, dev)
+    _need_ws(ws)
+    sc = 1.0 / math.sqrt(g.d) if scale is None else float(scale)
+    _run("bsa_sparse_attn_fwd_token", _device_of(qt, kt, vt, mask, kv_count, dense, out, lse, ws), stream,
+         lambda s: load_library().bsa_sparse_attn_fwd_token(
+             ctypes.byref(g.c()), _ptr(qt), _ptr(kt), _ptr(vt), _ptr(mask), _ptr(kv_count), _ptr(dense),
+             ctypes.c_int(int(token_radius)), ctypes.c_float(sc), _ptr(out), _ptr(lse), _ptr(ws),
+             ctypes.c_size_t(ws.numel()), s))
     return out, lse
 
 
@@ -346,6 +444,8 @@ class Buffers:
         self.qt = torch.empty(tiled, dtype=torch.bfloat16, device=dev)
         self.kt = torch.empty(tiled, dtype=torch.bfloat16, device=dev)
         self.vt = torch.empty(tiled, dtype=torch.bfloat16, device=dev)
+        self.qbar = torch.empty((g.B, g.H, g.NT, g.d), dtype=torch.float32, device=dev)
+        self.kbar = torch.empty((g.B, g.H, g.NT, g.d), dtype=torch.float32, device=dev)
         self.mask = torch.empty((g.B, g.H, g.NT, g.NW), dtype=torch.int32, device=dev)
         self.kv_count = torch.empty((g.B, g.H, g.NT), dtype=torch.int32, device=dev)
         self.out = torch.empty((g.B, g.N, g.H, g.d), dtype=torch.bfloat16, device=dev)
@@ -363,30 +463,34 @@ def forward(g: Geometry, p: MaskParams, q: torch.Tensor, k: torch.Tensor, v: tor
     an earlier call left in `bufs`: the reuse of a previous step's routing and sparsity
     (HetA-DiT reuses the preceding denoising step's estimates; MOD-DiT keeps historical
     sparsity). How often to rebuild is the caller's choice.
-    Window kind 2 (token-level circular support) is refused: its attention masks the tokens
-    outside the support inside window tiles, which the attention kernel does not do yet.
-    build_mask accepts kind 2; sparse_attn_fwd then attends whole retained tiles.
+    With window kind 2 (token-level circular support, radius p.radius in tokens) the
+    attention masks the tokens outside each query token's support inside window tiles,
+    with the route flags the mask build left in the workspace.
     """
-    if p.window_kind == 2:
-        raise ValueError("forward(): window kind 2 needs token-level masking inside window tiles, "
-                         "which the attention kernel does not apply yet; build_mask + "
-                         "sparse_attn_fwd give the tile-granular result")
     if not rebuild_mask and bufs is None:
         raise ValueError("rebuild_mask=False attends through the mask held in bufs: pass the "
                          "Buffers of an earlier call")
     b = bufs or Buffers(g, q.device)
-    reorder(g, q, b.qt, stream)
-    reorder(g, k, b.kt, stream)
+    if rebuild_mask:
+        reorder_pool(g, q, b.qt, b.qbar, stream)
+        reorder_pool(g, k, b.kt, b.kbar, stream)
+    else:
+        reorder(g, q, b.qt, stream)
+        reorder(g, k, b.kt, stream)
     reorder(g, v, b.vt, stream)
     if rebuild_mask:
-        build_mask(g, p, b.qt, b.kt, difficulty, b.mask, b.kv_count, b.ws, stream)
-    sparse_attn_fwd(g, b.qt, b.kt, b.vt, b.mask, b.kv_count, scale, b.out, b.lse, b.ws,
-                    stream=stream)
+        build_mask_pooled(g, p, b.qbar, b.kbar, difficulty, b.mask, b.kv_count, b.ws, stream)
+    if p.window_kind == 2:
+        sparse_attn_fwd_token(g, b.qt, b.kt, b.vt, b.mask, b.kv_count, route_flags(g, b.ws), p.radius,
+                              scale, b.out, b.lse, b.ws, stream=stream)
+    else:
+        sparse_attn_fwd(g, b.qt, b.kt, b.vt, b.mask, b.kv_count, scale, b.out, b.lse, b.ws,
+                        stream=stream)
     return b
 
 
-# kernels launched by forward(): 3 reorders; pool, route, score and select (plus entropy
-# and budget in budget mode) unless the mask is reused; 3 scheduler kernels and the
-# attention kernel
+# kernels launched by forward(): 3 reorders (Q and K fused with their pooling when the
+# mask is rebuilt); route, score and select (plus entropy and budget in budget mode) unless
+# the mask is reused; 3 scheduler kernels and the attention kernel
 def launches_per_forward(p: MaskParams, rebuild_mask: bool = True) -> int:
-    return 3 + ((4 + (2 if p.budget_mode == 1 else 0)) if rebuild_mask else 0) + 4
+    return 3 + ((3 + (2 if p.budget_mode == 1 else 0)) if rebuild_mask else 0) + 4

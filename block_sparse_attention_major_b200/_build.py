@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libbsa.so")
 OBJDIR = os.path.join(HERE, "_objs")
-SOURCES = ["abi.cu", "reorder.cu", "mask.cu", "attn.cu", "selftest.cu"]
+SOURCES = ["abi.cu", "reorder.cu", "mask.cu", "score_tc.cu", "attn.cu", "selftest.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

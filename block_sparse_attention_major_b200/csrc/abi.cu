@@ -139,6 +139,15 @@ int bsa_reorder(const bsa_geom* g, const void* x, void* xt, void* stream) {
                                   static_cast<__nv_bfloat16*>(xt), static_cast<cudaStream_t>(stream)));
 }
 
+int bsa_reorder_pool(const bsa_geom* g, const void* x, void* xt, float* xbar, void* stream) {
+  const CallRange range("bsa_reorder_pool");
+  if (!valid_geom(g) || !aligned16(x) || !aligned16(xt) || !aligned16(xbar)) return BSA_ERR_INVALID_ARG;
+  const int dev = device_ok();
+  if (dev != BSA_OK) return dev;
+  return status_of(launch_reorder_pool(make_geom(*g), static_cast<const __nv_bfloat16*>(x),
+                                       static_cast<__nv_bfloat16*>(xt), xbar, static_cast<cudaStream_t>(stream)));
+}
+
 int bsa_unreorder(const bsa_geom* g, const void* xt, void* x, void* stream) {
   const CallRange range("bsa_unreorder");
   if (!valid_geom(g) || !aligned16(x) || !aligned16(xt)) return BSA_ERR_INVALID_ARG;
@@ -164,10 +173,25 @@ int bsa_build_mask(const bsa_geom* g, const bsa_mask_params* p, const void* qt, 
                                      static_cast<uint8_t*>(ws), static_cast<cudaStream_t>(stream)));
 }
 
-int bsa_sparse_attn_fwd(const bsa_geom* g, const void* qt, const void* kt, const void* vt, const uint32_t* mask,
-                        const int32_t* kv_count, float softmax_scale, void* out, float* lse, void* ws,
-                        size_t ws_bytes, void* stream) {
-  const CallRange range("bsa_sparse_attn_fwd");
+int bsa_build_mask_pooled(const bsa_geom* g, const bsa_mask_params* p, const float* qbar, const float* kbar,
+                          const float* difficulty, uint32_t* mask, int32_t* kv_count, void* ws, size_t ws_bytes,
+                          void* stream) {
+  const CallRange range("bsa_build_mask_pooled");
+  if (!valid_geom(g) || !valid_params(g, p)) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(qbar) || !aligned16(kbar) || !aligned16(difficulty) || !aligned16(mask) || !aligned16(kv_count))
+    return BSA_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return BSA_ERR_WORKSPACE;
+  if (ws_bytes < bsa_workspace_bytes(g, p)) return BSA_ERR_WORKSPACE;
+  const int dev = device_ok();
+  if (dev != BSA_OK) return dev;
+  return status_of(launch_build_mask_pooled(make_geom(*g), *p, qbar, kbar, difficulty, mask, kv_count,
+                                            static_cast<uint8_t*>(ws), static_cast<cudaStream_t>(stream)));
+}
+
+// The checks shared by both workspace attention entry points; BSA_OK when the call may run.
+static int check_attn_args(const bsa_geom* g, const void* qt, const void* kt, const void* vt,
+                           const uint32_t* mask, const int32_t* kv_count, float softmax_scale, const void* out,
+                           const float* lse, const void* ws, size_t ws_bytes) {
   if (!valid_geom(g)) return BSA_ERR_INVALID_ARG;
   if (!aligned16(qt) || !aligned16(kt) || !aligned16(vt) || !aligned16(mask) || !aligned16(kv_count) ||
       !aligned16(out))
@@ -176,12 +200,39 @@ int bsa_sparse_attn_fwd(const bsa_geom* g, const void* qt, const void* kt, const
   if (!(softmax_scale > 0.0f) || isinf(softmax_scale)) return BSA_ERR_INVALID_ARG;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return BSA_ERR_WORKSPACE;
   if (ws_bytes < bsa_workspace_bytes(g, nullptr)) return BSA_ERR_WORKSPACE;
-  const int dev = device_ok();
-  if (dev != BSA_OK) return dev;
+  return device_ok();
+}
+
+int bsa_sparse_attn_fwd(const bsa_geom* g, const void* qt, const void* kt, const void* vt, const uint32_t* mask,
+                        const int32_t* kv_count, float softmax_scale, void* out, float* lse, void* ws,
+                        size_t ws_bytes, void* stream) {
+  const CallRange range("bsa_sparse_attn_fwd");
+  const int st = check_attn_args(g, qt, kt, vt, mask, kv_count, softmax_scale, out, lse, ws, ws_bytes);
+  if (st != BSA_OK) return st;
   return status_of(launch_sparse_attn(make_geom(*g), static_cast<const __nv_bfloat16*>(qt),
                                       static_cast<const __nv_bfloat16*>(kt), static_cast<const __nv_bfloat16*>(vt),
                                       mask, kv_count, softmax_scale, static_cast<__nv_bfloat16*>(out), lse,
                                       static_cast<uint8_t*>(ws), static_cast<cudaStream_t>(stream)));
+}
+
+int bsa_sparse_attn_fwd_token(const bsa_geom* g, const void* qt, const void* kt, const void* vt,
+                              const uint32_t* mask, const int32_t* kv_count, const uint8_t* dense,
+                              int token_radius, float softmax_scale, void* out, float* lse, void* ws,
+                              size_t ws_bytes, void* stream) {
+  const CallRange range("bsa_sparse_attn_fwd_token");
+  if (!dense || token_radius < 0 || token_radius > kMaxTokenRadius) return BSA_ERR_INVALID_ARG;
+  const int st = check_attn_args(g, qt, kt, vt, mask, kv_count, softmax_scale, out, lse, ws, ws_bytes);
+  if (st != BSA_OK) return st;
+  return status_of(launch_sparse_attn(make_geom(*g), static_cast<const __nv_bfloat16*>(qt),
+                                      static_cast<const __nv_bfloat16*>(kt), static_cast<const __nv_bfloat16*>(vt),
+                                      mask, kv_count, softmax_scale, static_cast<__nv_bfloat16*>(out), lse,
+                                      static_cast<uint8_t*>(ws), static_cast<cudaStream_t>(stream), dense,
+                                      token_radius));
+}
+
+size_t bsa_route_flags_offset(const bsa_geom* g) {
+  if (!valid_geom(g)) return 0;
+  return ws_layout(make_geom(*g)).dense;
 }
 
 int bsa_sparse_attn_fwd_fixed_scratch(const bsa_geom* g, const void* qt, const void* kt, const void* vt,

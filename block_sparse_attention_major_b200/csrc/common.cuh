@@ -126,12 +126,18 @@ __device__ __forceinline__ void report_error(uint32_t* err, uint32_t bits) {
 namespace bsa {
 cudaError_t launch_reorder(const Geom& g, const __nv_bfloat16* x, __nv_bfloat16* xt, cudaStream_t s);
 cudaError_t launch_unreorder(const Geom& g, const __nv_bfloat16* xt, __nv_bfloat16* x, cudaStream_t s);
+cudaError_t launch_reorder_pool(const Geom& g, const __nv_bfloat16* x, __nv_bfloat16* xt, float* xbar,
+                                cudaStream_t s);
+cudaError_t launch_build_mask_pooled(const Geom& g, const bsa_mask_params& p, const float* qbar,
+                                     const float* kbar, const float* difficulty, uint32_t* mask,
+                                     int32_t* kv_count, uint8_t* ws, cudaStream_t s);
 cudaError_t launch_build_mask(const Geom& g, const bsa_mask_params& p, const __nv_bfloat16* qt,
                               const __nv_bfloat16* kt, const float* difficulty, uint32_t* mask,
                               int32_t* kv_count, uint8_t* ws, cudaStream_t s);
 cudaError_t launch_sparse_attn(const Geom& g, const __nv_bfloat16* qt, const __nv_bfloat16* kt,
                                const __nv_bfloat16* vt, const uint32_t* mask, const int32_t* kv_count,
-                               float scale, __nv_bfloat16* out, float* lse, uint8_t* ws, cudaStream_t s);
+                               float scale, __nv_bfloat16* out, float* lse, uint8_t* ws, cudaStream_t s,
+                               const uint8_t* dense = nullptr, int token_rho = -1);
 // Attention with its scratch in the library's fixed device array (no workspace argument).
 size_t fixed_scratch_capacity();
 size_t fixed_scratch_need(const Geom& g);

@@ -4,8 +4,8 @@
 //            pooling" of tiles) -> qbar, kbar fp32 [B, H, NT, d]
 //  route     HetA-DiT routing (Abstract): the floor(rho*NQT + 1/2) query tiles of highest
 //            difficulty of each batch item take dense attention, ties to the lower index
-//  score     pooled scores qbar_i . kbar_j of every (b, h, query tile, key tile), fp32,
-//            into the workspace (a register-blocked SIMT SGEMM per head)
+//  score     pooled scores qbar_i . kbar_j of every (b, h, query tile, key tile), fp32-level
+//            accuracy on the tensor cores (3xTF32, score_tc.cu), into the workspace
 //  entropy   (budget mode) entropy of each row's softmax of the scaled scores
 //  budget    (budget mode) per row: the tile budget, the window radius it affords and the
 //            number of extra tiles
@@ -30,6 +30,11 @@
 #include <math.h>
 
 namespace bsa {
+
+// score_tc.cu
+cudaError_t launch_score_tc(const Geom& g, const float* qbar, const float* kbar, float* S, int NKTP,
+                            uint32_t* err, cudaStream_t s);
+
 namespace {
 
 constexpr int kSelThreads = 256;
@@ -142,75 +147,8 @@ __device__ int decayed_window_size(const Geom& g, int tt, int ty, int tx, int r)
   return s;
 }
 
-// ---- pooled scores: one 128 x 128 tile of S = qbar kbar^T (unscaled) per block, for one
-// (b, h). Register-blocked SIMT SGEMM: each of the 256 threads owns an 8 x 8 sub-tile, split
-// as rows {4 ty + r, 64 + 4 ty + r} and columns {4 tx + c, 64 + 4 tx + c} so that its four
-// float4 shared loads per d step are broadcast or conflict-free (4 loads per 64 FMAs). The d
-// dimension is staged through shared memory 32 at a time, transposed. Each output is
-// summed over d in increasing order, so the scores are deterministic.
-constexpr int kScoreTile = 128;
-constexpr int kScoreK = 32;
-constexpr int kScorePad = kScoreTile + 4;
-
-template <int D>
-__global__ void __launch_bounds__(256, 2) score_kernel(Geom g, const float* __restrict__ qbar,
-                                                    const float* __restrict__ kbar, float* __restrict__ S,
-                                                    int NKTP) {
-  __shared__ __align__(16) float sA[kScoreK][kScorePad];   // sA[c][r] = qbar[i0 + r][k0 + c]
-  __shared__ __align__(16) float sB[kScoreK][kScorePad];   // sB[c][r] = kbar[j0 + r][k0 + c]
-  const int i0 = blockIdx.x * kScoreTile, j0 = blockIdx.y * kScoreTile;
-  const long long bh = blockIdx.z;
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  const float4* q4 = reinterpret_cast<const float4*>(qbar + (bh * g.NT) * D);
-  const float4* k4 = reinterpret_cast<const float4*>(kbar + (bh * g.NT) * D);
-  float acc[8][8];
-#pragma unroll
-  for (int r = 0; r < 8; ++r)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
-  for (int k0 = 0; k0 < D; k0 += kScoreK) {
-#pragma unroll
-    for (int t = 0; t < kScoreTile * kScoreK / 4 / 256; ++t) {
-      const int e = tid + 256 * t;
-      const int r = e / (kScoreK / 4), c4 = e % (kScoreK / 4);
-      float4 va = make_float4(0.f, 0.f, 0.f, 0.f), vb = va;
-      if (i0 + r < g.NT) va = q4[(long long)(i0 + r) * (D / 4) + k0 / 4 + c4];
-      if (j0 + r < g.NT) vb = k4[(long long)(j0 + r) * (D / 4) + k0 / 4 + c4];
-      sA[4 * c4 + 0][r] = va.x;
-      sA[4 * c4 + 1][r] = va.y;
-      sA[4 * c4 + 2][r] = va.z;
-      sA[4 * c4 + 3][r] = va.w;
-      sB[4 * c4 + 0][r] = vb.x;
-      sB[4 * c4 + 1][r] = vb.y;
-      sB[4 * c4 + 2][r] = vb.z;
-      sB[4 * c4 + 3][r] = vb.w;
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int c = 0; c < kScoreK; ++c) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&sA[c][4 * ty]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&sA[c][64 + 4 * ty]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&sB[c][4 * tx]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&sB[c][64 + 4 * tx]);
-      const float qv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float kv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) acc[r][cc] = fmaf(qv[r], kv[cc], acc[r][cc]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const int i = i0 + (r < 4 ? 4 * ty + r : 64 + 4 * ty + (r - 4));
-    if (i >= g.NT) continue;
-    float* row = S + (bh * g.NT + i) * (long long)NKTP;
-    const int j_lo = j0 + 4 * tx, j_hi = j0 + 64 + 4 * tx;
-    if (j_lo < NKTP) *reinterpret_cast<float4*>(row + j_lo) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-    if (j_hi < NKTP) *reinterpret_cast<float4*>(row + j_hi) = make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
-  }
-}
+// ---- pooled scores: S = qbar kbar^T (unscaled) per (b, h), on the tensor cores in
+// score_tc.cu (3xTF32 products, fp32-level accuracy).
 
 // ---- row entropy (budget mode): H = log Z - sum(e (s - m)) / Z with s = scale * score,
 // e = exp(s - m); one warp per row.
@@ -572,6 +510,153 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
   if (q == 0 && lane == 0) a.kv_count[rowid] = count;
 }
 
+// ---- selection by radix (fixed top-k and budget modes): one row per warp, kRsWarps rows
+// per block. The row's order keys live in shared memory (0 for window tiles and for slots
+// past NKT). The key of the extra-th best candidate is found four bits at a time from the
+// top: each pass counts, in per-lane private shared-memory bins (no atomics), the keys
+// that carry the digits found so far, sums the 16 bins across lanes and keeps the largest
+// digit under which at least the still-needed number of keys lie. A pass that finds a
+// digit holding exactly that number ends the search (every key from that prefix up is
+// taken); otherwise the search ends at the exact key, and of the keys equal to it the
+// first in tile order are taken. The result is "highest score, ties to the lower index",
+// as the argmax and threshold search of select_kernel give it.
+constexpr int kRsWarps = 8;
+constexpr int kRsBinStride = 17;                 // per-lane bins, padded so lanes hit distinct banks
+
+template <int MODE, bool TOK>
+__global__ void __launch_bounds__(kRsWarps * 32) select_radix_kernel(SelArgs a, const float* __restrict__ S,
+                                                                     int NKTP) {
+  extern __shared__ __align__(16) uint32_t sm_u32[];
+  const Geom& g = a.g;
+  const int NKT = g.NT, NQT = g.NT;
+  const int NKW = g.NW * 32;                                   // key slots per row
+  const int b = blockIdx.z, h = blockIdx.y;
+  const long long bh = (long long)b * g.H + h;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint32_t* coord = sm_u32;                                    // NKW tile coordinates
+  uint32_t* keys = sm_u32 + NKW * (1 + warp);                  // this warp's row
+  uint32_t* bins = sm_u32 + NKW * (1 + kRsWarps) + warp * 32 * kRsBinStride + lane * kRsBinStride;
+
+  for (int j = tid; j < NKT; j += kRsWarps * 32) {
+    int tt, ty, tx;
+    tile_xyz(g, j, tt, ty, tx);
+    coord[j] = pack_coord(tt, ty, tx);
+  }
+  __syncthreads();
+
+  const int i = blockIdx.x * kRsWarps + warp;
+  if (i >= NQT) return;
+  const long long rowid = bh * NQT + i;
+  const float* srow = S + rowid * NKTP;
+  uint32_t* mrow = a.mask + rowid * g.NW;
+  if (a.dense[(long long)b * NQT + i]) {
+    for (int w = lane; w < g.NW; w += 32) {
+      const int rem = NKT - 32 * w;
+      mrow[w] = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+    }
+    if (lane == 0) a.kv_count[rowid] = NKT;
+    return;
+  }
+  const uint32_t ci = coord[i];
+  int kind = a.window_kind, rad = a.radius, extra;
+  if (MODE == kSelectFixed) {
+    extra = a.topk;
+  } else {
+    const int2 pl = a.plan[rowid];
+    kind = 1;
+    rad = pl.x;
+    extra = pl.y;
+  }
+  int ncand = 0;
+  for (int w = 0; w < g.NW; ++w) {
+    const int j = 32 * w + lane;
+    const bool cand = j < NKT && !sel_in_window<TOK>(ci, coord[j], kind, rad);
+    keys[j] = cand ? order_key(srow[j]) : 0u;
+    ncand += __popc(__ballot_sync(0xffffffffu, cand));
+  }
+  extra = max(0, min(extra, ncand));
+
+  // keys >= t_ge are taken; of the keys equal to thr, the first need_eq in tile order
+  uint32_t t_ge, thr = 0xffffffffu;
+  int need_eq = 0;
+  if (extra == 0) {
+    t_ge = 0xffffffffu;                                         // no score maps to this key
+  } else if (extra == ncand) {
+    t_ge = 1u;                                                  // every candidate (keys >= 2)
+  } else {
+    uint32_t prefix = 0u;
+    int remaining = extra;
+    bool done = false;
+    for (int shift = 28; shift >= 0 && !done; shift -= 4) {
+      const uint32_t hi = shift == 28 ? 0u : (0xffffffffu << (shift + 4));
+#pragma unroll
+      for (int d = 0; d < 16; ++d) bins[d] = 0u;
+      for (int w = 0; w < g.NW; ++w) {
+        const uint32_t k = keys[32 * w + lane];
+        if (k != 0u && (k & hi) == prefix) ++bins[(k >> shift) & 15u];
+      }
+      __syncwarp();
+      int tot = 0;
+      if (lane < 16) {
+        const uint32_t* col = bins - lane * kRsBinStride + lane;   // bin `lane` of every lane
+        for (int l = 0; l < 32; ++l) tot += (int)col[l * kRsBinStride];
+      }
+      // suffix sums over digits 15..0 (digit d at lane d)
+      int suf = tot;
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1) {
+        const int v = __shfl_down_sync(0xffffffffu, suf, off);
+        if (lane + off < 16) suf += v;
+      }
+      const uint32_t ok = __ballot_sync(0xffffffffu, lane < 16 && suf >= remaining);
+      const int dsel = 31 - __clz(ok);                          // largest digit with enough keys at or above it
+      const int above = __shfl_sync(0xffffffffu, suf, min(dsel + 1, 31)) * (dsel < 15 ? 1 : 0);
+      const int at = __shfl_sync(0xffffffffu, tot, dsel);
+      remaining -= above;
+      prefix |= (uint32_t)dsel << shift;
+      if (at == remaining) {                                    // the whole prefix band is taken
+        t_ge = prefix;
+        done = true;
+      }
+      __syncwarp();
+    }
+    if (!done) {
+      thr = prefix;                                             // the exact key of the boundary
+      t_ge = prefix + 1u;
+      need_eq = remaining;
+    }
+    if (t_ge == 0u) t_ge = 1u;                                  // a band from key 0: every candidate
+  }
+
+  int eq_before = 0, count = 0;
+  for (int w = 0; w < g.NW; ++w) {
+    const int j = 32 * w + lane;
+    const uint32_t k = keys[j];
+    const bool inrow = j < NKT;
+    bool sel = inrow && (k == 0u || k >= t_ge);
+    const bool eq = inrow && k != 0u && k == thr && need_eq > 0;
+    const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+    const int rank = eq_before + __popc(eqb & ((1u << lane) - 1u));
+    sel = sel || (eq && rank < need_eq);
+    eq_before += __popc(eqb);
+    const uint32_t bits = __ballot_sync(0xffffffffu, sel);
+    if (lane == 0) mrow[w] = bits;
+    count += __popc(bits);
+  }
+  if (lane == 0) a.kv_count[rowid] = count;
+}
+
+template <int MODE, bool TOK>
+cudaError_t launch_select_radix(const Geom& g, const SelArgs& a, const float* S, int NKTP, cudaStream_t s) {
+  const size_t smem = sizeof(uint32_t) * ((size_t)g.NW * 32 * (1 + kRsWarps) + (size_t)kRsWarps * 32 * kRsBinStride);
+  cudaError_t e = cudaFuncSetAttribute(select_radix_kernel<MODE, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(ceil_div(g.NT, kRsWarps), g.H, g.B);
+  select_radix_kernel<MODE, TOK><<<grid, kRsWarps * 32, smem, s>>>(a, S, NKTP);
+  return cudaGetLastError();
+}
+
 template <int MODE, int KW, int WPR, bool TOK>
 cudaError_t launch_select_kw(const Geom& g, size_t smem, const SelArgs& a, const float* S, int NKTP, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(select_kernel<MODE, KW, WPR, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -592,22 +677,32 @@ cudaError_t launch_select(const Geom& g, size_t smem, const SelArgs& a, const fl
   return launch_select_kw<MODE, 32, 4, TOK>(g, smem, a, S, NKTP, s);
 }
 
+// The mask from tile-major Q and K (qt, kt: pooled here, into the workspace) or from
+// pooled means computed by the fused reorder (qt, kt null; qbar_in, kbar_in given).
 template <int D>
 cudaError_t build_mask_d(const Geom& g, const bsa_mask_params& p, const __nv_bfloat16* qt,
-                         const __nv_bfloat16* kt, const float* difficulty, uint32_t* mask,
-                         int32_t* kv_count, uint8_t* ws, cudaStream_t s) {
+                         const __nv_bfloat16* kt, const float* qbar_in, const float* kbar_in,
+                         const float* difficulty, uint32_t* mask, int32_t* kv_count, uint8_t* ws,
+                         cudaStream_t s) {
   const WsLayout L = ws_layout(g);
-  float* qbar = reinterpret_cast<float*>(ws + L.qbar);
-  float* kbar = reinterpret_cast<float*>(ws + L.kbar);
+  const float* qbar = qbar_in;
+  const float* kbar = kbar_in;
   uint8_t* dense = ws + L.dense;
   float* entropy = reinterpret_cast<float*>(ws + L.entropy);
   int2* plan = reinterpret_cast<int2*>(ws + L.plan);
 
-  const long long warps = 2LL * g.B * g.H * g.NT;
-  pool_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(g, qt, kt, qbar, kbar);
-  count_launches(1);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
+  if (qt) {
+    float* qb = reinterpret_cast<float*>(ws + L.qbar);
+    float* kb = reinterpret_cast<float*>(ws + L.kbar);
+    const long long warps = 2LL * g.B * g.H * g.NT;
+    pool_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(g, qt, kt, qb, kb);
+    count_launches(1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    qbar = qb;
+    kbar = kb;
+  }
 
   const int nd = (int)floor((double)p.dense_fraction * (double)g.NT + 0.5);
   route_kernel<<<dim3(ceil_div(g.NT, 256), g.B), 256, g.NT * sizeof(float), s>>>(g, difficulty, nd, dense);
@@ -631,10 +726,7 @@ cudaError_t build_mask_d(const Geom& g, const bsa_mask_params& p, const __nv_bfl
 
   float* S = reinterpret_cast<float*>(ws + L.scores);
   const int NKTP = (g.NT + 3) & ~3;
-  score_kernel<D><<<dim3(ceil_div(g.NT, kScoreTile), ceil_div(g.NT, kScoreTile), g.B * g.H), 256, 0, s>>>(
-      g, qbar, kbar, S, NKTP);
-  count_launches(1);
-  e = cudaGetLastError();
+  e = launch_score_tc(g, qbar, kbar, S, NKTP, reinterpret_cast<uint32_t*>(ws), s);
   if (e != cudaSuccess) return e;
 
   a.theta = p.budget_target;
@@ -656,13 +748,13 @@ cudaError_t build_mask_d(const Geom& g, const bsa_mask_params& p, const __nv_bfl
   // the budget mode always uses the decayed tile window (kind 1)
   const bool tok = p.window_kind == 2;
   if (p.budget_mode == 0)
-    e = tok ? launch_select<kSelectFixed, true>(g, sel_smem, a, S, NKTP, s)
-            : launch_select<kSelectFixed, false>(g, sel_smem, a, S, NKTP, s);
+    e = tok ? launch_select_radix<kSelectFixed, true>(g, a, S, NKTP, s)
+            : launch_select_radix<kSelectFixed, false>(g, a, S, NKTP, s);
   else if (p.budget_mode == 2)
     e = tok ? launch_select<kSelectMass, true>(g, sel_smem, a, S, NKTP, s)
             : launch_select<kSelectMass, false>(g, sel_smem, a, S, NKTP, s);
   else
-    e = launch_select<kSelectBudget, false>(g, sel_smem, a, S, NKTP, s);
+    e = launch_select_radix<kSelectBudget, false>(g, a, S, NKTP, s);
   if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();
@@ -673,8 +765,15 @@ cudaError_t build_mask_d(const Geom& g, const bsa_mask_params& p, const __nv_bfl
 cudaError_t launch_build_mask(const Geom& g, const bsa_mask_params& p, const __nv_bfloat16* qt,
                               const __nv_bfloat16* kt, const float* difficulty, uint32_t* mask,
                               int32_t* kv_count, uint8_t* ws, cudaStream_t s) {
-  if (g.d == 128) return build_mask_d<128>(g, p, qt, kt, difficulty, mask, kv_count, ws, s);
-  return build_mask_d<64>(g, p, qt, kt, difficulty, mask, kv_count, ws, s);
+  if (g.d == 128) return build_mask_d<128>(g, p, qt, kt, nullptr, nullptr, difficulty, mask, kv_count, ws, s);
+  return build_mask_d<64>(g, p, qt, kt, nullptr, nullptr, difficulty, mask, kv_count, ws, s);
+}
+
+cudaError_t launch_build_mask_pooled(const Geom& g, const bsa_mask_params& p, const float* qbar,
+                                     const float* kbar, const float* difficulty, uint32_t* mask,
+                                     int32_t* kv_count, uint8_t* ws, cudaStream_t s) {
+  if (g.d == 128) return build_mask_d<128>(g, p, nullptr, nullptr, qbar, kbar, difficulty, mask, kv_count, ws, s);
+  return build_mask_d<64>(g, p, nullptr, nullptr, qbar, kbar, difficulty, mask, kv_count, ws, s);
 }
 
 }  // namespace bsa

@@ -10,6 +10,13 @@
 //  - unreorder walks the raster output (b, n, head, chunk): contiguous writes, 256-byte
 //    runs of reads.
 // Each thread keeps 4 independent vectors in flight.
+//
+// reorder_pool does the reorder of Q or K and, in the same pass, the per-tile mean of the
+// valid tokens (VORTA summary, "average pooling" of tiles) that the mask builder scores:
+// one block per (b, tile) walks the tile's 64 slots for every (head, 16-byte chunk) of the
+// token rows, so each thread keeps the fp32 sums of its chunk in registers while the
+// vectors move. The mask builder then starts from the means instead of reading the
+// tile-major tensors a second time.
 #include "common.cuh"
 
 namespace bsa {
@@ -105,6 +112,59 @@ __global__ void __launch_bounds__(kThreads) unreorder_kernel(ReorderArgs a, cons
   }
 }
 
+constexpr int kPoolThreads = 128;
+constexpr int kPoolUnroll = 8;
+
+// One block per (b, tile j): every vector of the tile's slots, and the means.
+__global__ void __launch_bounds__(kPoolThreads) reorder_pool_kernel(ReorderArgs a, const uint4* __restrict__ x,
+                                                                    uint4* __restrict__ xt, float* __restrict__ xbar) {
+  __shared__ int tok[64];
+  __shared__ int s_nvalid;
+  const int d8 = 1 << a.d8_log2;
+  const int b = blockIdx.x / a.g.NT, j = blockIdx.x - b * a.g.NT;
+  if (threadIdx.x < 64) tok[threadIdx.x] = slot_token(a, j, threadIdx.x);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int r = 0; r < 64; ++r) n += tok[r] >= 0;
+    s_nvalid = n;
+  }
+  __syncthreads();
+  const float inv = 1.0f / (float)s_nvalid;
+  const int nv = a.g.H * d8;                       // vectors per token row
+  for (int v = threadIdx.x; v < nv; v += kPoolThreads) {
+    const int h = v >> a.d8_log2, c = v & (d8 - 1);
+    const uint4* src = x + (long long)b * a.g.N * nv + v;
+    uint4* dst = xt + ((((long long)b * a.g.H + h) * a.g.NT + j) * 64) * d8 + c;
+    float acc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+#pragma unroll 1
+    for (int r0 = 0; r0 < 64; r0 += kPoolUnroll) {
+      uint4 w[kPoolUnroll];
+#pragma unroll
+      for (int u = 0; u < kPoolUnroll; ++u) {
+        const int n = tok[r0 + u];
+        w[u] = n >= 0 ? __ldg(&src[(long long)n * nv]) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kPoolUnroll; ++u) {
+        dst[(r0 + u) * d8] = w[u];
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&w[u]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(p[k]);
+          acc[2 * k] += f.x;
+          acc[2 * k + 1] += f.y;
+        }
+      }
+    }
+    float4* m = reinterpret_cast<float4*>(xbar + ((((long long)b * a.g.H + h) * a.g.NT + j) * d8 + c) * 8);
+    m[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    m[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+  }
+}
+
 ReorderArgs make_args(const Geom& g, long long total) {
   ReorderArgs a;
   a.g = g;
@@ -137,6 +197,15 @@ cudaError_t launch_reorder(const Geom& g, const __nv_bfloat16* x, __nv_bfloat16*
   ReorderArgs a = make_args(g, total);
   reorder_kernel<<<grid_for(total), kThreads, 0, s>>>(a, reinterpret_cast<const uint4*>(x),
                                                       reinterpret_cast<uint4*>(xt));
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reorder_pool(const Geom& g, const __nv_bfloat16* x, __nv_bfloat16* xt, float* xbar,
+                                cudaStream_t s) {
+  ReorderArgs a = make_args(g, 0);
+  reorder_pool_kernel<<<g.B * g.NT, kPoolThreads, 0, s>>>(a, reinterpret_cast<const uint4*>(x),
+                                                          reinterpret_cast<uint4*>(xt), xbar);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -66,9 +66,9 @@ typedef struct bsa_geom {
  *                    (y_m - y_n)^2 + (x_m - x_n)^2 <= (radius - |t_m - t_n|)^2, in tokens;
  *                    key tile j is a window tile of query tile i when a valid token of j
  *                    supports a valid token of i. Budget modes 0 and 2 only. The mask is
- *                    tile-granular: bsa_sparse_attn_fwd attends every valid token of each
- *                    retained tile (it does not yet mask the tokens outside the support
- *                    inside window tiles)
+ *                    tile-granular; bsa_sparse_attn_fwd_token masks the tokens outside the
+ *                    support inside window tiles (bsa_sparse_attn_fwd attends every valid
+ *                    token of each retained tile)
  *   radius        window radius (>= 0): in tiles for kinds 0 and 1, in tokens (at most
  *                 32767) for kind 2; ignored when budget_mode = 1
  *   topk          extra key tiles outside the window, by pooled score, ties to the lower
@@ -134,6 +134,16 @@ int bsa_clear_error(void* ws, void* stream);
  * Bit-exact copy; no arithmetic. */
 int bsa_reorder(const bsa_geom* g, const void* x, void* xt, void* stream);
 
+/* Tile-major reorder fused with the per-tile mean of the mask builder (Token Radius
+ * Attention summary, "Efficient execution", tile-major layout; VORTA summary, "average
+ * pooling" of tiles). One pass over x does both:
+ *   x    : bf16 [B, N, H, d] raster (input, read only)
+ *   xt   : bf16 [B, H, NT, 64, d] (output, exactly as bsa_reorder writes it)
+ *   xbar : fp32 [B, H, NT, d] (output): the mean over the valid tokens of each tile, summed
+ *          in fp32 in slot order
+ * For Q and K ahead of bsa_build_mask_pooled, which then needs no second read of qt, kt. */
+int bsa_reorder_pool(const bsa_geom* g, const void* x, void* xt, float* xbar, void* stream);
+
 /* Inverse of bsa_reorder: xt bf16 [B, H, NT, 64, d] -> x bf16 [B, N, H, d]. Padding slots
  * of xt are ignored. Bit-exact. */
 int bsa_unreorder(const bsa_geom* g, const void* xt, void* x, void* stream);
@@ -154,6 +164,14 @@ int bsa_build_mask(const bsa_geom* g, const bsa_mask_params* p, const void* qt,
                    const void* kt, const float* difficulty, uint32_t* mask,
                    int32_t* kv_count, void* ws, size_t ws_bytes, void* stream);
 
+/* bsa_build_mask starting from the per-tile means of Q and K (as bsa_reorder_pool writes
+ * them) instead of the tile-major tensors: the same routing, window and selection steps,
+ * with the same arguments otherwise.
+ *   qbar, kbar : fp32 [B, H, NT, d] per-tile means of the valid tokens of Q and K */
+int bsa_build_mask_pooled(const bsa_geom* g, const bsa_mask_params* p, const float* qbar,
+                          const float* kbar, const float* difficulty, uint32_t* mask,
+                          int32_t* kv_count, void* ws, size_t ws_bytes, void* stream);
+
 /* Block-sparse attention forward (Token Radius Attention summary, execution of
  * block-sparse masks; FlashAttention-style online softmax).
  *   qt, kt, vt : bf16 [B, H, NT, 64, d] tile-major Q, K, V
@@ -172,6 +190,32 @@ int bsa_build_mask(const bsa_geom* g, const bsa_mask_params* p, const void* qt,
 int bsa_sparse_attn_fwd(const bsa_geom* g, const void* qt, const void* kt, const void* vt,
                         const uint32_t* mask, const int32_t* kv_count, float softmax_scale,
                         void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Block-sparse attention forward under a token-level circular support (window kind 2 of
+ * bsa_mask_params; Token Radius Attention summary: query-centred circular neighbourhoods,
+ * base radius applied across frames with temporal decay).
+ *   Arguments as bsa_sparse_attn_fwd, plus
+ *   dense        : device pointer, uint8 [B, NQT]; nonzero marks a dense row (see
+ *                  bsa_route_flags_offset for the flags bsa_build_mask leaves in its
+ *                  workspace)
+ *   token_radius : the support radius rho in tokens, 0 <= rho <= 32767
+ * A local row (dense == 0) sees, in each retained key tile that is a window tile of its
+ * query tile (window kind 2 with radius rho), only the key tokens in the support of each
+ * query token: |t_k - t_q| <= rho and (y_k - y_q)^2 + (x_k - x_q)^2 <= (rho - |t_k - t_q|)^2.
+ * Other retained tiles, and every tile of a dense row, are seen whole. Every query token
+ * sees at least itself, so no row is empty. Errors as bsa_sparse_attn_fwd; a null dense or
+ * a radius out of range is BSA_ERR_INVALID_ARG. */
+int bsa_sparse_attn_fwd_token(const bsa_geom* g, const void* qt, const void* kt, const void* vt,
+                              const uint32_t* mask, const int32_t* kv_count, const uint8_t* dense,
+                              int token_radius, float softmax_scale, void* out, float* lse, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/* Byte offset in the workspace at which bsa_build_mask leaves the route flags of its call
+ * (uint8 [B, NQT], 1 = dense row), valid until the workspace is given to another
+ * bsa_build_mask call. The attention calls do not touch that region, so the flags may be
+ * passed to bsa_sparse_attn_fwd_token together with the same workspace. 0 for an invalid
+ * geometry. Host only. */
+size_t bsa_route_flags_offset(const bsa_geom* g);
 
 /* Block-sparse attention forward without a workspace argument. The papers have no
  * counterpart: this entry point exists for callers that cannot allocate device memory,

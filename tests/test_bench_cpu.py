@@ -50,7 +50,7 @@ def test_valid_token_flops():
 
 def test_mask_bytes():
     g = _G(1, 12, 128, 21, 30, 52)
-    assert bench._mask_bytes(g) == 2 * 32760 * 12 * 128 * 2 + 12 * 624 * (20 + 1) * 4
+    assert bench._mask_bytes(g) == 2 * 12 * 624 * 128 * 4 + 12 * 624 * (20 + 1) * 4
 
 
 def test_reference_arm_prints_a_contract_line():
