@@ -65,4 +65,54 @@ BSA_HD bool in_window(uint32_t ci, uint32_t cj, int kind, int r) {
   return kind == 2 ? in_token_window(ci, cj, r) : in_tile_window(ci, cj, kind, r);
 }
 
+// ---- the token-level support inside window tiles (the attention side of kind 2)
+
+// Slots of key tile (tt, ty, tx), bit (a * 4 + b) * 4 + c for the token
+// (4 tt + a, 4 ty + b, 4 tx + c), whose token lies in the support of query token
+// (qt, qy, qx). Slots beyond the grid are not excluded here.
+BSA_HD uint64_t token_support_slots(int qt, int qy, int qx, int tt, int ty, int tx, int r) {
+  uint64_t m = 0;
+#ifdef __CUDA_ARCH__
+#pragma unroll
+#endif
+  for (int a = 0; a < 4; ++a) {
+    const int dt = iabs_(4 * tt + a - qt);
+    const int rr = r - dt;
+    const int R2 = dt <= r ? rr * rr : -1;
+#ifdef __CUDA_ARCH__
+#pragma unroll
+#endif
+    for (int b = 0; b < 4; ++b) {
+      const int dy = 4 * ty + b - qy;
+      const int lim = R2 - dy * dy;
+#ifdef __CUDA_ARCH__
+#pragma unroll
+#endif
+      for (int c = 0; c < 4; ++c) {
+        const int dx = 4 * tx + c - qx;
+        if (dx * dx <= lim) m |= 1ull << (16 * a + 4 * b + c);
+      }
+    }
+  }
+  return m;
+}
+
+// Largest token distance along an axis of n tokens between tiles a and b.
+BSA_HD int max_token_dist(int a, int b, int n) {
+  const int ahi = 4 * a + 3 < n - 1 ? 4 * a + 3 : n - 1;
+  const int bhi = 4 * b + 3 < n - 1 ? 4 * b + 3 : n - 1;
+  return imax_(ahi - 4 * b, bhi - 4 * a);
+}
+
+// Whether every valid token of key tile cj lies in the support of every valid token of
+// query tile ci (grid T x Hs x Ws): the condition at the largest distance along each axis,
+// since the valid tokens of a tile form a box and the condition only gets harder as any
+// distance grows. Such a tile needs no per-token mask.
+BSA_HD bool token_tiles_all_inside(uint32_t ci, uint32_t cj, int T, int Hs, int Ws, int r) {
+  const int mt = max_token_dist((int)(ci >> 20), (int)(cj >> 20), T);
+  const int my = max_token_dist((int)((ci >> 10) & 1023u), (int)((cj >> 10) & 1023u), Hs);
+  const int mx = max_token_dist((int)(ci & 1023u), (int)(cj & 1023u), Ws);
+  return mt <= r && my * my + mx * mx <= (r - mt) * (r - mt);
+}
+
 }  // namespace bsa

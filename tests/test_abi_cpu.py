@@ -127,14 +127,30 @@ def test_invalid_mask_params_rejected_on_host(lib, bad):
                               ctypes.c_void_p(0x10000), 1 << 30, None) == 1
 
 
-def test_forward_refuses_token_window():
-    """forward() does not hand a kind-2 mask to an attention that would attend whole tiles."""
-    import torch
+def test_token_attention_rejects_bad_arguments_on_host(lib):
+    """Null route flags and radii outside [0, 32767] are refused before any device call."""
     import block_sparse_attention_major_b200 as bsa
-    g = bsa.Geometry(1, 1, 64, 4, 4, 4)
-    x = torch.zeros(1, 64, 1, 64, dtype=torch.bfloat16)
-    with pytest.raises(ValueError, match="window kind 2"):
-        bsa.forward(g, bsa.MaskParams(2, 6, 1), x, x, x, torch.zeros(1, 1))
+    g = bsa.Geometry(1, 2, 64, 8, 16, 16).c()
+    al = ctypes.c_void_p(0x1000)
+    ws = ctypes.c_void_p(0x10000)
+    for dense, rho in ((None, 6), (al, -1), (al, 32768)):
+        assert lib.bsa_sparse_attn_fwd_token(ctypes.byref(g), al, al, al, al, al, dense, rho,
+                                             ctypes.c_float(0.125), al, None, ws, 1 << 30, None) == 1
+    bad = bsa.Geometry(1, 2, 96, 8, 16, 16).c()
+    assert lib.bsa_sparse_attn_fwd_token(ctypes.byref(bad), al, al, al, al, al, al, 6,
+                                         ctypes.c_float(0.125), al, None, ws, 1 << 30, None) == 1
+
+
+def test_route_flags_offset(lib):
+    """The route flags sit inside the workspace, after the pooled Q and K, and a flags
+    region of B*NQT bytes fits before the workspace ends."""
+    import block_sparse_attention_major_b200 as bsa
+    g = bsa.Geometry(2, 3, 128, 7, 13, 10)
+    off = lib.bsa_route_flags_offset(ctypes.byref(g.c()))
+    pooled = g.B * g.H * g.NT * g.d * 4
+    assert off >= 256 + 2 * pooled and off % 256 == 0
+    assert off + g.B * g.NT <= lib.bsa_workspace_bytes(ctypes.byref(g.c()), None)
+    assert lib.bsa_route_flags_offset(ctypes.byref(bsa.Geometry(1, 1, 96, 4, 4, 4).c())) == 0
 
 
 def test_binding_fails_loudly_without_library(tmp_path):
@@ -218,9 +234,21 @@ def test_binding_wrappers_marshal_every_entry_point(monkeypatch):
     bsa.sparse_attn_fwd_fixed_scratch(g, tiled, tiled, tiled, mask, cnt, None, out, lse, err)
     bsa.clear_error(ws)
     bsa.selftest_bounded_wait(err)
+    pooled = torch.zeros(g.B, g.H, g.NT, g.d)
+    bsa.reorder_pool(g, raster, tiled, pooled)
+    bsa.build_mask_pooled(g, p, pooled, pooled, diff, mask, cnt, ws)
+    dense = torch.zeros(g.B, g.NT, dtype=torch.uint8)
+    bsa.sparse_attn_fwd_token(g, tiled, tiled, tiled, mask, cnt, dense, 6, None, out, lse, ws)
     names = [c[0] for c in calls]
     assert names == ["bsa_reorder", "bsa_unreorder", "bsa_build_mask", "bsa_sparse_attn_fwd",
-                     "bsa_sparse_attn_fwd_fixed_scratch", "bsa_clear_error", "bsa_selftest_bounded_wait"]
+                     "bsa_sparse_attn_fwd_fixed_scratch", "bsa_clear_error", "bsa_selftest_bounded_wait",
+                     "bsa_reorder_pool", "bsa_build_mask_pooled", "bsa_sparse_attn_fwd_token"]
+    tk = calls[9][1]
+    assert tk[6].value == dense.data_ptr() and tk[7].value == 6 and abs(tk[8].value - 0.125) < 1e-7
+    assert [a.value for a in (tk[9], tk[10], tk[11])] == [out.data_ptr(), lse.data_ptr(), ws.data_ptr()]
+    assert [a.value for a in calls[7][1][1:4]] == [raster.data_ptr(), tiled.data_ptr(), pooled.data_ptr()]
+    assert [a.value for a in calls[8][1][2:8]] == [pooled.data_ptr(), pooled.data_ptr(), diff.data_ptr(),
+                                                  mask.data_ptr(), cnt.data_ptr(), ws.data_ptr()]
     for name, args in calls:
         assert args[-1].value == FakeStream.cuda_stream, name
     ptr = lambda t: t.data_ptr()
@@ -275,17 +303,18 @@ def test_forward_mask_reuse_skips_the_build(monkeypatch):
     p = bsa.MaskParams(1, 1, 2, 0.25)
     t = lambda *shape, dt=torch.bfloat16: torch.zeros(*shape, dtype=dt)
     b = types.SimpleNamespace(qt=t(1, 2, g.NT, 64, 64), kt=t(1, 2, g.NT, 64, 64), vt=t(1, 2, g.NT, 64, 64),
+                              qbar=t(1, 2, g.NT, 64, dt=torch.float32), kbar=t(1, 2, g.NT, 64, dt=torch.float32),
                               mask=t(1, 2, g.NT, g.NW, dt=torch.int32), kv_count=t(1, 2, g.NT, dt=torch.int32),
                               out=t(1, g.N, 2, 64), lse=t(1, 2, g.N, dt=torch.float32),
                               ws=t(4096, dt=torch.uint8))
     x = t(1, g.N, 2, 64)
     d = t(1, g.NT, dt=torch.float32)
     bsa.forward(g, p, x, x, x, d, bufs=b)
-    assert calls == ["bsa_reorder"] * 3 + ["bsa_build_mask", "bsa_sparse_attn_fwd"]
+    assert calls == ["bsa_reorder_pool"] * 2 + ["bsa_reorder", "bsa_build_mask_pooled", "bsa_sparse_attn_fwd"]
     calls.clear()
     bsa.forward(g, p, x, x, x, d, bufs=b, rebuild_mask=False)
     assert calls == ["bsa_reorder"] * 3 + ["bsa_sparse_attn_fwd"]
-    assert bsa.launches_per_forward(p, rebuild_mask=False) == bsa.launches_per_forward(p) - 4
+    assert bsa.launches_per_forward(p, rebuild_mask=False) == bsa.launches_per_forward(p) - 3
     with pytest.raises(ValueError, match="earlier call"):
         bsa.forward(g, p, x, x, x, d, rebuild_mask=False)
 

@@ -51,18 +51,26 @@ def _whole_path(w: Workload, token: bool = False):
     p = C.params(w)
     tiled = (g.B, g.H, g.NT, 64, g.d)
     raster = (g.B, g.N, g.H, g.d)
+    pooled = (g.B, g.H, g.NT, g.d)
     c = Carved([(raster, torch.bfloat16)] * 3 + [(tiled, torch.bfloat16)] * 3 +
                [((g.B, g.NT), torch.float32), ((g.B, g.H, g.NT, g.NW), torch.int32),
                 ((g.B, g.H, g.NT), torch.int32), (raster, torch.bfloat16), ((g.B, g.H, g.N), torch.float32),
-                ((bsa.workspace_bytes(g),), torch.uint8), (raster, torch.bfloat16)])
-    qd, kd, vd, qt, kt, vt, dd, mask, cnt, out, lse, ws, back = c.views
+                ((bsa.workspace_bytes(g),), torch.uint8), (raster, torch.bfloat16),
+                (pooled, torch.float32), (pooled, torch.float32)])
+    qd, kd, vd, qt, kt, vt, dd, mask, cnt, out, lse, ws, back, qbar, kbar = c.views
     for dst, src in ((qd, q), (kd, k), (vd, v), (dd, diff)):
         dst.copy_(src)
     ws.zero_()
+    # both mask paths: from the tile-major tensors, then from the fused reorder's means
     for x, xt in ((qd, qt), (kd, kt), (vd, vt)):
         bsa.reorder(g, x, xt)
     bsa.build_mask(g, p, qt, kt, dd, mask, cnt, ws)
-    if not token:
+    bsa.reorder_pool(g, qd, qt, qbar)
+    bsa.reorder_pool(g, kd, kt, kbar)
+    bsa.build_mask_pooled(g, p, qbar, kbar, dd, mask, cnt, ws)
+    if token:
+        bsa.sparse_attn_fwd_token(g, qt, kt, vt, mask, cnt, bsa.route_flags(g, ws), w.radius, None, out, lse, ws)
+    else:
         bsa.sparse_attn_fwd(g, qt, kt, vt, mask, cnt, None, out, lse, ws)
     bsa.unreorder(g, vt, back)
     torch.cuda.synchronize()
@@ -83,7 +91,7 @@ def test_no_writes_outside_tensors_degenerate_grids(grid):
                          topk=2, dense_fraction=0.3))
 
 
-def test_no_writes_outside_tensors_token_window_masks():
+def test_no_writes_outside_tensors_token_support():
     _whole_path(C.workload("token128"), token=True)
 
 

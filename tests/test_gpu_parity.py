@@ -52,6 +52,25 @@ def test_unreorder_round_trip_bit_exact(name):
     assert np.array_equal(_i16(bsa.unreorder(g, xt)), ref)
 
 
+@pytest.mark.parametrize("name", SMALL + ["wan13b"])
+def test_reorder_pool(name):
+    """The fused reorder writes the same tile-major tensor as the reorder (bit-exact) and the
+    per-tile means of the valid tokens, within fp32 summation error of the oracle's."""
+    bsa = _bsa()
+    w, q, k, _, _ = C.inputs(name)
+    g = C.geometry(w)
+    for x in (q, k):
+        xt, xbar = bsa.reorder_pool(g, x.cuda())
+        torch.cuda.synchronize()
+        assert np.array_equal(_i16(xt), O.reorder(_i16(x), w.T, w.Hs, w.Ws))
+        x64 = O.reorder(O.to_f64(x), w.T, w.Hs, w.Ws)
+        ref = O.pool(x64, w.T, w.Hs, w.Ws)
+        # 64 fp32 additions of bf16 values: error below 64 * 2^-24 of the largest magnitude
+        bound = 64 * 2.0 ** -24 * np.abs(x64).max(axis=(3, 4))[..., None] + 1e-30
+        err = np.abs(xbar.double().cpu().numpy() - ref)
+        assert (err <= bound).all(), float((err / bound).max())
+
+
 # ----------------------------------------------------------------------------- mask
 def _mask_case(name, heads=None, overrides=()):
     bsa = _bsa()
@@ -418,4 +437,134 @@ def test_forward_mask_reuse():
     ref = O.attention_tiles(qb64, kb64, vb64, used, rows, T=wb.T, Hs=wb.Hs, Ws=wb.Ws)
     st = C.compare_attention(wb, b.out, b.lse, ref)
     print(st)
+    C.assert_attention_close(st)
+
+
+# ----------------------------------------------------------------------------- score kernel
+def _ws_offsets(g):
+    """Byte offsets of the pooled means and the scores in the workspace. This mirrors the
+    library's workspace layout (256-byte aligned regions in a fixed order)."""
+    a = lambda x: (x + 255) // 256 * 256
+    off = 256
+    pooled = g.B * g.H * g.NT * g.d * 4
+    qbar = off; off = a(off + pooled)
+    kbar = off; off = a(off + pooled)
+    off = a(off + g.B * g.NT)                                   # route flags
+    off = a(off + g.B * g.H * g.NT * 4)                         # entropy
+    off = a(off + g.B * g.H * g.NT * 8)                         # budget plan
+    off = a(off + g.B * g.H * 16)                               # per-(b, h) counts
+    off = a(off + g.B * g.H * (g.NT // 4 + 2) * 32)             # work units
+    return qbar, kbar, off
+
+
+@pytest.mark.parametrize("name", ["small128", "ragged128", "wan13b"])
+def test_scores_against_exact_products(name):
+    """The tensor-core scores against the exact products of the GPU's own pooled means:
+    within 2e-6 of each row's score scale (3xTF32)."""
+    bsa = _bsa()
+    w, q, k, _, diff = C.inputs(name)
+    g = C.geometry(w)
+    qt, kt = bsa.reorder(g, q.cuda()), bsa.reorder(g, k.cuda())
+    ws = bsa.alloc_workspace(g)
+    assert ws.numel() == bsa.workspace_bytes(g)
+    bsa.build_mask(g, C.params(w), qt, kt, diff.cuda(), ws=ws)
+    torch.cuda.synchronize()
+    assert bsa.read_error(ws) == 0
+    oq, ok_, os_ = _ws_offsets(g)
+    n = g.B * g.H * g.NT * g.d
+    qbar = ws[oq:oq + 4 * n].view(torch.float32).view(g.B * g.H, g.NT, g.d).double().cpu().numpy()
+    kbar = ws[ok_:ok_ + 4 * n].view(torch.float32).view(g.B * g.H, g.NT, g.d).double().cpu().numpy()
+    nktp = (g.NT + 3) // 4 * 4
+    S = ws[os_:os_ + 4 * g.B * g.H * g.NT * nktp].view(torch.float32).view(g.B * g.H, g.NT, nktp)
+    S = S[:, :, :g.NT].double().cpu().numpy()
+    exact = np.einsum("bid,bjd->bij", qbar, kbar)
+    scale = np.abs(exact).max(axis=2, keepdims=True)
+    err = float((np.abs(S - exact) / scale).max())
+    print(name, "max relative score error", err)
+    assert err < 2e-6
+
+
+# ----------------------------------------------------------------------------- token support
+def _attn_token(w, q, k, v, mask_bool, dense, rho, rows=None):
+    """GPU attention under a token-level support, given a mask and route flags computed
+    here (never from the GPU), and the oracle's rows."""
+    bsa = _bsa()
+    g = C.geometry(w)
+    qt, kt, vt = (bsa.reorder(g, x.cuda()) for x in (q, k, v))
+    bits = O.pack_bitmask(mask_bool).view(np.int32)
+    mask = torch.from_numpy(bits.copy()).cuda()
+    cnt = torch.from_numpy(mask_bool.sum(-1).astype(np.int32)).cuda()
+    dflags = torch.from_numpy(dense.astype(np.uint8)).cuda()
+    ws = bsa.alloc_workspace(g)
+    out, lse = bsa.sparse_attn_fwd_token(g, qt, kt, vt, mask, cnt, dflags, rho, ws=ws)
+    torch.cuda.synchronize()
+    assert bsa.read_error(ws) == 0
+    if rows is None:
+        rows = [(b, h, i) for b in range(w.B) for h in range(w.H) for i in range(g.NT)]
+    qt64, kt64, vt64 = (O.reorder(O.to_f64(x), w.T, w.Hs, w.Ws) for x in (q, k, v))
+    ref = O.attention_tiles(qt64, kt64, vt64, mask_bool, rows, T=w.T, Hs=w.Hs, Ws=w.Ws, token_rho=rho,
+                            window=O.token_window(rho, w.T, w.Hs, w.Ws), dense=dense)
+    return out, lse, ref
+
+
+@pytest.mark.parametrize("name", ["token128", "token_mass"])
+def test_attention_token_support_oracle_mask(name):
+    """Token-level support inside window tiles, on the oracle's kind-2 mask and route flags."""
+    w, q, k, v, diff = C.inputs(name)
+    qt64, kt64 = (O.reorder(O.to_f64(x), w.T, w.Hs, w.Ws) for x in (q, k))
+    mref = C.oracle_mask(w, qt64, kt64, diff.numpy())
+    out, lse, ref = _attn_token(w, q, k, v, mref["mask"], mref["dense"], w.radius)
+    st = C.compare_attention(w, out, lse, ref)
+    print(name, st)
+    C.assert_attention_close(st)
+
+
+@pytest.mark.parametrize("rho", [0, 3, 6, 11])
+def test_attention_token_support_random_masks(rho):
+    """Random tile masks (window tiles and extras alike) and random route flags on a
+    ragged grid, across radii from the tile itself (0) to most of the grid."""
+    w, q, k, v, diff = C.inputs("ragged128")
+    g = C.geometry(w)
+    rng = np.random.default_rng(40 + rho)
+    m = rng.random((w.B, w.H, g.NT, g.NT)) < 0.4
+    m |= np.eye(g.NT, dtype=bool)[None, None]                 # every row keeps its own tile
+    dense = rng.random((w.B, g.NT)) < 0.2
+    m[dense[:, None, :, None].repeat(w.H, 1).repeat(g.NT, 3)] = True
+    out, lse, ref = _attn_token(w, q, k, v, m, dense, rho)
+    st = C.compare_attention(w, out, lse, ref)
+    print(rho, st)
+    C.assert_attention_close(st)
+
+
+@pytest.mark.parametrize("name,overrides", [("token128", ()), ("token_mass", ()),
+                                            ("wan13b", (("window_kind", 2), ("radius", 6)))])
+def test_forward_path_token_support(name, overrides):
+    """The whole path with window kind 2: GPU mask against the oracle, then the GPU output
+    against the oracle's token-masked attention (rows whose GPU mask differs at a flagged
+    near-tie under the GPU's own mask)."""
+    bsa = _bsa()
+    w, q, k, v, diff = C.inputs(name, overrides)
+    g = C.geometry(w)
+    b = bsa.forward(g, C.params(w), q.cuda(), k.cuda(), v.cuda(), diff.cuda())
+    torch.cuda.synchronize()
+    assert bsa.read_error(b.ws) == 0
+    heads = [0, w.H - 1] if name == "wan13b" else list(range(w.H))
+    qt64, kt64, vt64 = (O.reorder(O.to_f64(x[:, :, heads]), w.T, w.Hs, w.Ws) for x in (q, k, v))
+    mref = C.oracle_mask(w, qt64, kt64, diff.numpy())
+    gm = C.gpu_mask_bool(b.mask, g.NT)[:, heads]
+    cmp = C.compare_masks(gm, mref)
+    assert cmp["n_unflagged"] == 0, cmp
+    assert np.array_equal(bsa.route_flags(g, b.ws).cpu().numpy().astype(bool), mref["dense"])
+    if name == "wan13b":
+        rng = np.random.default_rng(29)
+        rows = [(0, int(rng.integers(2)), int(rng.integers(g.NT))) for _ in range(16)]
+    else:
+        rows = [(bb, h, i) for bb in range(w.B) for h in range(len(heads)) for i in range(g.NT)]
+    used = C.mask_for_reference(mref["mask"], gm, cmp["diff_rows"])
+    ref = O.attention_tiles(qt64, kt64, vt64, used, rows, T=w.T, Hs=w.Hs, Ws=w.Ws,
+                            token_rho=w.radius, window=O.token_window(w.radius, w.T, w.Hs, w.Ws),
+                            dense=mref["dense"])
+    ref = {(bb, heads[h], i): e for (bb, h, i), e in ref.items()}
+    st = C.compare_attention(w, b.out, b.lse, ref)
+    print(name, st, "retained", float(gm.mean()))
     C.assert_attention_close(st)

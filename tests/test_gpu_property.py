@@ -64,8 +64,13 @@ def test_forward_matches_oracle_on_random_grids(T, Hs, Ws, d, B, H, kind, radius
 @SETTINGS
 @given(T=axis, Hs=axis, Ws=axis, rho=st.integers(0, 10), topk=st.integers(0, 4),
        mass=st.booleans(), seed=st.integers(0, 2**16))
-def test_token_window_masks_match_oracle_on_random_grids(T, Hs, Ws, rho, topk, mass, seed):
+def test_token_support_matches_oracle_on_random_grids(T, Hs, Ws, rho, topk, mass, seed):
     w = Workload("gpu_property_token", B=1, H=2, d=64, T=T, Hs=Hs, Ws=Ws, seed=seed, window_kind=2,
                  radius=rho, topk=topk, dense_fraction=0.25, budget_mode=2 if mass else 0,
                  budget_target=0.5 if mass else 0.0)
-    _run(w, forward=False)
+    b, mref, cmp, (qt64, kt64, vt64) = _run(w, forward=True)
+    rows = [(0, h, i) for h in range(w.H) for i in range(w.NT)]
+    ref = O.attention_tiles(qt64, kt64, vt64, mref["used"], rows, T=T, Hs=Hs, Ws=Ws, token_rho=rho,
+                            window=O.token_window(rho, T, Hs, Ws), dense=mref["dense"])
+    st_ = C.compare_attention(w, b.out, b.lse, ref)
+    C.assert_attention_close(st_)

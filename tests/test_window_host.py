@@ -28,12 +28,17 @@ def win(tmp_path_factory):
     lib = ctypes.CDLL(so)
     lib.window_tiles.restype = ctypes.c_int
     lib.window_tiles.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p]
+    lib.support_slots.restype = ctypes.c_ulonglong
+    lib.support_slots.argtypes = [ctypes.c_int] * 7
+    lib.all_inside.restype = ctypes.c_int
+    lib.all_inside.argtypes = [ctypes.c_int] * 4 + [ctypes.c_void_p]
 
     def run(kind, r, T, Hs, Ws):
         NT = int(np.prod(O.tile_grid(T, Hs, Ws)))
         out = np.zeros((NT, NT), dtype=np.uint8)
         assert lib.window_tiles(T, Hs, Ws, kind, r, out.ctypes.data) == NT
         return out.astype(bool)
+    run.lib = lib
     return run
 
 
@@ -66,3 +71,43 @@ def test_token_support_window_extremes(win):
     assert w.all()
     w0 = win(2, 0, 8, 8, 8)
     assert np.array_equal(w0, np.eye(w0.shape[0], dtype=bool))
+
+
+@pytest.mark.parametrize("grid", [(8, 16, 16), (6, 10, 9), (13, 7, 11)])
+def test_support_slots_match_oracle(win, grid):
+    """The per-slot support mask the attention softmax uses inside window tiles, against
+    the oracle's token support on the token coordinates of the slots."""
+    T, Hs, Ws = grid
+    xy = O.slot_coords(T, Hs, Ws)
+    NT = xy.shape[0]
+    rng = np.random.default_rng(sum(grid))
+    for rho in (0, 1, 3, 6, 10):
+        W = O.token_window(rho, T, Hs, Ws)
+        for _ in range(60):
+            i, j = int(rng.integers(NT)), int(rng.integers(NT))
+            if rng.random() < 0.7:                          # mostly window pairs
+                js = np.nonzero(W[i])[0]
+                j = int(js[rng.integers(js.size)])
+            r = int(rng.integers(64))
+            got = win.lib.support_slots(T, Hs, Ws, i, r, j, rho)
+            want = O.in_token_support(xy[i, r][None, :], xy[j], rho)
+            bits = sum(1 << s_ for s_ in range(64) if want[s_])
+            assert got == bits, (rho, i, r, j)
+
+
+@pytest.mark.parametrize("grid", [(8, 16, 16), (6, 10, 9), (13, 7, 11), (5, 5, 5)])
+def test_all_inside_matches_brute_force(win, grid):
+    """Tile pairs that need no per-token mask: every valid token pair in the support."""
+    T, Hs, Ws = grid
+    xy = O.slot_coords(T, Hs, Ws)
+    valid = O.slot_valid(T, Hs, Ws)
+    NT = xy.shape[0]
+    for rho in (0, 2, 5, 6, 9, 14):
+        out = np.zeros((NT, NT), dtype=np.uint8)
+        assert win.lib.all_inside(T, Hs, Ws, rho, out.ctypes.data) == NT
+        for i in range(NT):
+            q = xy[i][valid[i]]
+            for j in range(NT):
+                k = xy[j][valid[j]]
+                want = bool(O.in_token_support(q[:, None, :], k[None, :, :], rho).all())
+                assert bool(out[i, j]) == want, (rho, i, j)
