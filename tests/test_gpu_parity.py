@@ -460,7 +460,8 @@ def _ws_offsets(g):
 @pytest.mark.parametrize("name", ["small128", "ragged128", "wan13b"])
 def test_scores_against_exact_products(name):
     """The tensor-core scores against the exact products of the GPU's own pooled means:
-    within 2e-6 of each row's score scale (3xTF32)."""
+    within 1e-5 of each row's score scale (3xTF32), a tenth of the selection's near-tie
+    band of 1e-4, so that only rows the oracle flags can select differently."""
     bsa = _bsa()
     w, q, k, _, diff = C.inputs(name)
     g = C.geometry(w)
@@ -481,7 +482,7 @@ def test_scores_against_exact_products(name):
     scale = np.abs(exact).max(axis=2, keepdims=True)
     err = float((np.abs(S - exact) / scale).max())
     print(name, "max relative score error", err)
-    assert err < 2e-6
+    assert err < 1e-5
 
 
 # ----------------------------------------------------------------------------- token support
