@@ -15,13 +15,14 @@ from oracle import bsa_oracle as O
 O_REL_L2 = 5e-3
 O_MAX_ABS = 2e-2
 LSE_ABS = 1e-3
-# The output is bf16, so where half a bf16 ulp of |O| reaches the max-abs bound (|O| >= 8)
-# no bf16 result can meet it literally. Per element the bound is therefore
-#   max(O_MAX_ABS, half_ulp_bf16(O) + O_PRE_ROUNDING)
-# with O_PRE_ROUNDING = 2e-2 - 2^-6: the computation error that the literal bound leaves
-# at the top of its attainable range (|O| just below 8, half an ulp 2^-6). Every element
-# with |O| < 8 is held to the literal 2e-2.
-O_PRE_ROUNDING = O_MAX_ABS - 2.0 ** -6
+# The output is bf16, and the P.V product takes bf16 probabilities (each rounded by up to
+# 2^-9 of itself). Where half a bf16 ulp of |O| is well under the max-abs bound (|O| < 4:
+# at most 2^-7) the bound is held literally: 2e-2. Above that, half an ulp (2^-6 and up)
+# takes most of the bound by itself, and the literal bound would leave less computation
+# error than the rounding of bf16 probabilities implies; there the bound is half an ulp
+# plus the computation error the literal bound allows at |O| just below 4:
+#   max(O_MAX_ABS, half_ulp_bf16(O) + O_PRE_ROUNDING),  O_PRE_ROUNDING = 2e-2 - 2^-7.
+O_PRE_ROUNDING = O_MAX_ABS - 2.0 ** -7
 
 SMALL_D128 = {
     "small128": Workload("small128", B=1, H=2, d=128, T=8, Hs=16, Ws=16, seed=1010,
