@@ -28,13 +28,14 @@
 //   warps 4-7  softmax of query block B
 //              (each reads S from TMEM, writes P as bf16 pairs over S, rescales its O in
 //              TMEM when a row maximum grows by more than 2^8, and runs the epilogue)
-//   warp 8     lane 0 issues the TMA loads of Q and of the K/V ring
+//   warp 8     lane 0 issues the TMA loads of Q and of the K ring
 //   warp 9     allocates TMEM; lane 0 issues every tcgen05.mma of both query blocks
 //   warp 10    takes the next unit from the work list and builds its key stream in shared
 //              memory (double buffered, one unit ahead)
-//   warp 11    idle (it completes the third warpgroup)
-// The softmax warpgroups raise their register budget to 208 and the third lowers its own to
-// 88 (setmaxnreg), which keeps a whole 128-column score block of a row in registers.
+//   warp 11    lane 0 issues the TMA loads of the V ring
+// The softmax warpgroups raise their register budget to 184 and the third lowers its own to
+// 136 (setmaxnreg); the softmax holds 64 score columns of a row at a time, reading a
+// 128-column block from TMEM twice.
 // TMEM columns: S_A at 0, S_B at 128 (128 each; P is written over S as bf16 pairs, key k of
 // the block at column k/2), O_A at 256, O_B at 256 + D. Shared memory (1024-byte aligned):
 // Q_A, Q_B, two K and two V stages, each a 128-row operand laid out as [D/64 column
@@ -68,8 +69,8 @@ namespace {
 
 constexpr int kAttnThreads = 384;
 constexpr int kRegsLaunch = 168;                   // 65536 / (3 warps per SM sub-partition x 32 x 4), rounded to 8
-constexpr int kRegsSoftmax = 208;
-constexpr int kRegsControl = 88;
+constexpr int kRegsSoftmax = 184;
+constexpr int kRegsControl = 136;
 static_assert(128 * (2 * kRegsSoftmax + kRegsControl) <= kAttnThreads * kRegsLaunch,
               "register split above the launch's pool");
 constexpr int kNS = 2;                             // K and V ring stages, two key tiles each
@@ -133,9 +134,9 @@ struct Bars {
   __device__ uint32_t drain() const { return b0 + 8 * (4 * kNS + 14); }
 };
 
-// lempty arrivals per key-stream buffer: the TMA producer, the two issuer cursors and the
-// eight softmax warps.
-constexpr int kListConsumers = 1 + 2 + 8;
+// lempty arrivals per key-stream buffer: the two TMA producers, the two issuer cursors and
+// the eight softmax warps.
+constexpr int kListConsumers = 2 + 2 + 8;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -186,46 +187,43 @@ __device__ __forceinline__ uint64_t tile_slots(int j, uint32_t flags, int t, con
   return m;
 }
 
-// Row maximum over the 64 columns at offset OFF of r (four short chains).
-template <int OFF>
-__device__ __forceinline__ float half_max_full(const uint32_t (&r)[128], float m) {
+// Row maximum over 64 score columns (four short chains).
+__device__ __forceinline__ float half_max_full(const uint32_t (&r)[64], float m) {
   float a0 = m, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
   for (int c = 0; c < 64; c += 8) {
-    a0 = max3(a0, __uint_as_float(r[OFF + c + 0]), __uint_as_float(r[OFF + c + 1]));
-    a1 = max3(a1, __uint_as_float(r[OFF + c + 2]), __uint_as_float(r[OFF + c + 3]));
-    a2 = max3(a2, __uint_as_float(r[OFF + c + 4]), __uint_as_float(r[OFF + c + 5]));
-    a3 = max3(a3, __uint_as_float(r[OFF + c + 6]), __uint_as_float(r[OFF + c + 7]));
+    a0 = max3(a0, __uint_as_float(r[c + 0]), __uint_as_float(r[c + 1]));
+    a1 = max3(a1, __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
+    a2 = max3(a2, __uint_as_float(r[c + 4]), __uint_as_float(r[c + 5]));
+    a3 = max3(a3, __uint_as_float(r[c + 6]), __uint_as_float(r[c + 7]));
   }
   return fmaxf(max3(a0, a1, a2), a3);
 }
 
-// Same over the valid slots only (bit c of `valid` set).
-template <int OFF>
-__device__ __forceinline__ float half_max_valid(const uint32_t (&r)[128], uint64_t valid, float m) {
+// Same over the slots whose bit in `valid` is set.
+__device__ __forceinline__ float half_max_valid(const uint32_t (&r)[64], uint64_t valid, float m) {
   const uint32_t lo = (uint32_t)valid, hi = (uint32_t)(valid >> 32);
   float a0 = m, a1 = -INFINITY;
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
-    a0 = fmaxf(a0, ((lo >> c) & 1u) ? __uint_as_float(r[OFF + c]) : -INFINITY);
-    a1 = fmaxf(a1, ((hi >> c) & 1u) ? __uint_as_float(r[OFF + 32 + c]) : -INFINITY);
+    a0 = fmaxf(a0, ((lo >> c) & 1u) ? __uint_as_float(r[c]) : -INFINITY);
+    a1 = fmaxf(a1, ((hi >> c) & 1u) ? __uint_as_float(r[32 + c]) : -INFINITY);
   }
   return fmaxf(a0, a1);
 }
 
-template <int OFF>
-__device__ __forceinline__ float half_max(const uint32_t (&r)[128], int use, uint64_t valid, float m) {
-  if (use == kUseFull) return half_max_full<OFF>(r, m);
-  if (use == kUsePartial) return half_max_valid<OFF>(r, valid, m);
+__device__ __forceinline__ float half_max(const uint32_t (&r)[64], int use, uint64_t valid, float m) {
+  if (use == kUseFull) return half_max_full(r, m);
+  if (use == kUsePartial) return half_max_valid(r, valid, m);
   return m;
 }
 
-// p = 2^(s*c - m) for the 64 columns at offset OFF of r (zero on slots whose bit in
-// `valid` is clear), stored to TMEM as bf16 pairs (column 2i in the low half of 32-bit
-// column i), 16 columns per store. `sum` gets the fp32 probabilities, `sum_bf` the
-// bf16-rounded ones that P.V uses.
-template <bool kMasked, int OFF>
-__device__ __forceinline__ void exp_half(const uint32_t (&r)[128], uint64_t valid, float c, float m,
+// p = 2^(s*c - m) for 64 score columns (zero on slots whose bit in `valid` is clear),
+// stored to TMEM as bf16 pairs (column 2i in the low half of 32-bit column i), 16 columns
+// per store. `sum` gets the fp32 probabilities, `sum_bf` the bf16-rounded ones that P.V
+// uses.
+template <bool kMasked>
+__device__ __forceinline__ void exp_half(const uint32_t (&r)[64], uint64_t valid, float c, float m,
                                          float& sum, float& sum_bf, uint32_t taddr) {
   const uint32_t lo = (uint32_t)valid, hi = (uint32_t)(valid >> 32);
   float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
@@ -236,10 +234,10 @@ __device__ __forceinline__ void exp_half(const uint32_t (&r)[128], uint64_t vali
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
       const int b = 16 * k + 2 * i;
-      float p0 = ex2(fmaf(__uint_as_float(r[OFF + b + 0]), c, -m));
-      float p1 = ex2(fmaf(__uint_as_float(r[OFF + b + 1]), c, -m));
-      float p2 = ex2(fmaf(__uint_as_float(r[OFF + b + 2]), c, -m));
-      float p3 = ex2(fmaf(__uint_as_float(r[OFF + b + 3]), c, -m));
+      float p0 = ex2(fmaf(__uint_as_float(r[b + 0]), c, -m));
+      float p1 = ex2(fmaf(__uint_as_float(r[b + 1]), c, -m));
+      float p2 = ex2(fmaf(__uint_as_float(r[b + 2]), c, -m));
+      float p3 = ex2(fmaf(__uint_as_float(r[b + 3]), c, -m));
       if (kMasked) {
         const uint32_t w = b < 32 ? lo : hi;
         const int sh = b & 31;
@@ -272,12 +270,18 @@ __device__ __forceinline__ void store_zero_p(uint32_t taddr) {
   for (int k = 0; k < 4; ++k) tmem_st_x8(taddr + 8 * k, z);
 }
 
-template <int OFF>
-__device__ __forceinline__ void half_exp(const uint32_t (&r)[128], int use, uint64_t valid, float c, float m,
+__device__ __forceinline__ void half_exp(const uint32_t (&r)[64], int use, uint64_t valid, float c, float m,
                                          float& sum, float& sum_bf, uint32_t taddr) {
-  if (use == kUseFull) exp_half<false, OFF>(r, 0ull, c, m, sum, sum_bf, taddr);
-  else if (use == kUsePartial) exp_half<true, OFF>(r, valid, c, m, sum, sum_bf, taddr);
+  if (use == kUseFull) exp_half<false>(r, 0ull, c, m, sum, sum_bf, taddr);
+  else if (use == kUsePartial) exp_half<true>(r, valid, c, m, sum, sum_bf, taddr);
   else store_zero_p(taddr);
+}
+
+// 64 score columns from TMEM (two 32-column loads) and the wait for them.
+__device__ __forceinline__ void load_half(uint32_t taddr, uint32_t (&r)[64]) {
+  tmem_ld_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  tmem_ld_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+  ptx::tmem_wait_ld();
 }
 
 // O *= alpha for this thread's row of the D accumulator columns, 32 columns per TMEM
@@ -348,9 +352,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = *tmem_slot;
   if (warp >= 8) {
   ptx::setmaxnreg_dec<kRegsControl>();
-  if (warp == 11) {
-    // idle
-  } else if (warp == 10) {
+  if (warp == 10) {
     // ------------------------------------------------------------ key-stream builder
     const int nunits = a.header[1];
     for (int it = 0;; ++it) {
@@ -458,14 +460,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar.lfull(buf));
     }
-  } else if (warp == 8) {
-    // ------------------------------------------------------------------ TMA producer
+  } else if (warp == 8 || warp == 11) {
+    // ------------------------------------------------------------------ TMA producers
+    // Lane 0 of warp 8 loads Q and the K ring, lane 0 of warp 11 the V ring, so that a K
+    // stage never waits behind a V stage (or the reverse).
+    const bool vprod = warp == 11;
     if (lane == 0) {
       ptx::prefetch_tensormap(&tmQ);
       ptx::prefetch_tensormap(&tmK);
       ptx::prefetch_tensormap(&tmV);
       int qn[2] = {0, 0};       // Q loads issued per query block
-      long long nk = 0, nv = 0; // stream blocks whose K / V load was issued
+      uint32_t nk = 0, nv = 0;  // stream blocks whose K / V load was issued (only the low bits matter)
       bool ok = true;
       for (int it = 0; ok; ++it) {
         const int buf = it & 1;
@@ -478,7 +483,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int q[4] = {meta[1], meta[2], meta[3], meta[4]};
         const int L = meta[5];
         const long long tile_row0 = (long long)bh * g.NT;
-        for (int x = 0; x < 2 && ok; ++x) {
+        for (int x = 0; x < 2 && ok && !vprod; ++x) {
           if (q[2 * x] < 0) continue;
           if (qn[x] > 0 && !ptx::mbar_wait(bar.qempty(x), (qn[x] - 1) & 1, abort, a.err, kWaitLimit)) {
             ok = false;
@@ -497,7 +502,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int nb = (L + 1) / 2;
         for (int c = 0; c < nb && ok; ++c) {
           const int nh = 2 * c + 1 < L ? 2 : 1;
-          {
+          if (!vprod) {
             const int s = (int)(nk % kNS);
             const uint32_t ph = ((nk / kNS) & 1) ^ 1;
             if (!ptx::mbar_wait(bar.kempty(s), ph, abort, a.err, kWaitLimit)) { ok = false; break; }
@@ -509,8 +514,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               for (int cb = 0; cb < D / 64; ++cb) ptx::tma_load_2d(dst + cb * C::kCB, &tmK, bar.kfull(s), cb * 64, row);
             }
             ++nk;
-          }
-          {
+          } else {
             const int s = (int)(nv % kNS);
             const uint32_t ph = ((nv / kNS) & 1) ^ 1;
             if (!ptx::mbar_wait(bar.vempty(s), ph, abort, a.err, kWaitLimit)) { ok = false; break; }
@@ -530,11 +534,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int zero = 0;
       for (int s = 0; s < kNS; ++s) {
         if (nk > s) {
-          const long long last = s + kNS * ((nk - 1 - s) / kNS);
+          const uint32_t last = s + kNS * ((nk - 1 - s) / kNS);
           ptx::mbar_wait(bar.kfull(s), (uint32_t)((last / kNS) & 1), &zero, a.err, kWaitLimit);
         }
         if (nv > s) {
-          const long long last = s + kNS * ((nv - 1 - s) / kNS);
+          const uint32_t last = s + kNS * ((nv - 1 - s) / kNS);
           ptx::mbar_wait(bar.vfull(s), (uint32_t)((last / kNS) & 1), &zero, a.err, kWaitLimit);
         }
       }
@@ -564,7 +568,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         bool have, done;
         int L, nb, kc, vc, pend;
         bool hasq, qready, qreleased, first_pv;
-        long long gbase;   // global index of the unit's first stream block
+        uint32_t gbase;    // index of the unit's first stream block in this CTA's stream
         int qn;            // Q loads consumed (units with this query block)
         uint32_t pn;       // P.V products issued (= pfull phases consumed)
         const uint16_t* flags;
@@ -581,7 +585,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         cur[x].pn = 0;
         cur[x].flags = nullptr;
       }
-      long long kpass[2] = {0, 0}, vpass[2] = {0, 0};
+      // stream blocks each cursor has passed (modulo 2^32: the cursors stay within a ring
+      // length of each other, so differences decide the order)
+      uint32_t kpass[2] = {0u, 0u}, vpass[2] = {0u, 0u};
       bool ok = true;
       long long idle_since = clock64();
       while (ok && !(cur[0].done && cur[1].done)) {
@@ -614,7 +620,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           // ---- K position
           if (cu.kc < cu.nb) {
             const int u = cu.hasq ? block_use(cu.flags, cu.L, cu.kc, x) : 0;
-            const long long gi = cu.gbase + cu.kc;
+            const uint32_t gi = cu.gbase + (uint32_t)cu.kc;
             const int s = (int)(gi % kNS);
             const uint32_t fph = (uint32_t)((gi / kNS) & 1);
             bool passed = false;
@@ -642,8 +648,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               }
             }
             if (passed) {
-              kpass[x] = gi + 1;
-              if (kpass[x ^ 1] >= gi + 1) ptx::mma_commit(bar.kempty(s));
+              kpass[x] = gi + 1u;
+              if ((int)(kpass[x ^ 1] - (gi + 1u)) >= 0) ptx::mma_commit(bar.kempty(s));
               ++cu.kc;
               progress = true;
               if (cu.kc == cu.nb && cu.hasq && cu.qready && !cu.qreleased) {
@@ -654,7 +660,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           // ---- V position
           if (cu.vc < cu.kc) {
-            const long long gi = cu.gbase + cu.vc;
+            const uint32_t gi = cu.gbase + (uint32_t)cu.vc;
             const int s = (int)(gi % kNS);
             const uint32_t fph = (uint32_t)((gi / kNS) & 1);
             bool passed = false;
@@ -680,8 +686,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               passed = ptx::mbar_test_wait(bar.vfull(s), fph);
             }
             if (passed) {
-              vpass[x] = gi + 1;
-              if (vpass[x ^ 1] >= gi + 1) ptx::mma_commit(bar.vempty(s));
+              vpass[x] = gi + 1u;
+              if ((int)(vpass[x ^ 1] - (gi + 1u)) >= 0) ptx::mma_commit(bar.vempty(s));
               ++cu.vc;
               progress = true;
             }
@@ -699,7 +705,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             ptx::mbar_arrive(bar.lempty(cu.it & 1));
             ++cu.it;
             cu.have = false;
-            cu.gbase += cu.nb;
+            cu.gbase += (uint32_t)cu.nb;
             progress = true;
           }
         }
@@ -768,19 +774,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             use1 == kUsePartial ? tile_slots(tiles[2 * cb + 1], f1, t, g, tq, yq, xq, a.token_rho) : ~0ull;
         if (!warp_wait(bar.sfull(x), sidx & 1, abort, a.err)) { ok = false; break; }
         ptx::tc_fence_after();
-        uint32_t r[128];
-        if (u & 1) {
-          tmem_ld_x32(s_tmem + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-          tmem_ld_x32(s_tmem + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        }
-        if (u & 2) {
-          tmem_ld_x32(s_tmem + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
-          tmem_ld_x32(s_tmem + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
-        }
-        ptx::tmem_wait_ld();
+        // The block is read from TMEM twice, 64 columns at a time: once for the maximum
+        // (second tile first, so the first tile's columns are still in registers), once
+        // for the exponentials (first tile first: its P overwrites only its own, already
+        // read, S columns; the second tile's P then overwrites the first tile's upper S
+        // columns, which are no longer needed).
+        uint32_t r[64];
         float mx = -INFINITY;
-        mx = half_max<0>(r, use0, valid0, mx);
-        mx = half_max<64>(r, use1, valid1, mx);
+        if (u & 2) {
+          load_half(s_tmem + 64, r);
+          mx = half_max(r, use1, valid1, mx);
+        }
+        if (u & 1) {
+          load_half(s_tmem + 0, r);
+          mx = half_max(r, use0, valid0, mx);
+        }
         const float mb = mx * c;                       // block maximum, log2 domain
         bool resc = false;
         if (m_run == -INFINITY) m_run = mb;            // O of this row is still zero
@@ -796,8 +804,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (resc) m_run = mb;
         }
         const float m_use = m_run == -INFINITY ? 0.0f : m_run;
-        if (u & 1) half_exp<0>(r, use0, valid0, c, m_use, l_ex, l_bf, s_tmem + 0);
-        if (u & 2) half_exp<64>(r, use1, valid1, c, m_use, l_ex, l_bf, s_tmem + 32);
+        if (u & 1) half_exp(r, use0, valid0, c, m_use, l_ex, l_bf, s_tmem + 0);
+        if (u & 2) {
+          if (u & 1) load_half(s_tmem + 64, r);       // (with the second tile alone, r holds it)
+          half_exp(r, use1, valid1, c, m_use, l_ex, l_bf, s_tmem + 32);
+        }
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();

@@ -13,8 +13,8 @@
 //
 // reorder_pool does the reorder of Q or K and, in the same pass, the per-tile mean of the
 // valid tokens (VORTA summary, "average pooling" of tiles) that the mask builder scores:
-// one block per (b, tile) walks the tile's 64 slots for every (head, 16-byte chunk) of the
-// token rows, so each thread keeps the fp32 sums of its chunk in registers while the
+// one block per (b, tile, 128 (head, 16-byte chunk) vectors of the token rows) walks the
+// tile's 64 slots, so each thread keeps the fp32 sums of its chunk in registers while the
 // vectors move. The mask builder then starts from the means instead of reading the
 // tile-major tensors a second time.
 #include "common.cuh"
@@ -113,9 +113,10 @@ __global__ void __launch_bounds__(kThreads) unreorder_kernel(ReorderArgs a, cons
 }
 
 constexpr int kPoolThreads = 128;
-constexpr int kPoolUnroll = 8;
+constexpr int kPoolUnroll = 16;
 
-// One block per (b, tile j): every vector of the tile's slots, and the means.
+// One block per (b, tile j, 128 of the token row's vectors): each thread moves one
+// (head, 16-byte chunk) vector of the tile's 64 slots and keeps its fp32 sums.
 __global__ void __launch_bounds__(kPoolThreads) reorder_pool_kernel(ReorderArgs a, const uint4* __restrict__ x,
                                                                     uint4* __restrict__ xt, float* __restrict__ xbar) {
   __shared__ int tok[64];
@@ -132,7 +133,8 @@ __global__ void __launch_bounds__(kPoolThreads) reorder_pool_kernel(ReorderArgs 
   __syncthreads();
   const float inv = 1.0f / (float)s_nvalid;
   const int nv = a.g.H * d8;                       // vectors per token row
-  for (int v = threadIdx.x; v < nv; v += kPoolThreads) {
+  const int v = blockIdx.y * kPoolThreads + threadIdx.x;
+  if (v < nv) {
     const int h = v >> a.d8_log2, c = v & (d8 - 1);
     const uint4* src = x + (long long)b * a.g.N * nv + v;
     uint4* dst = xt + ((((long long)b * a.g.H + h) * a.g.NT + j) * 64) * d8 + c;
@@ -204,8 +206,9 @@ cudaError_t launch_reorder(const Geom& g, const __nv_bfloat16* x, __nv_bfloat16*
 cudaError_t launch_reorder_pool(const Geom& g, const __nv_bfloat16* x, __nv_bfloat16* xt, float* xbar,
                                 cudaStream_t s) {
   ReorderArgs a = make_args(g, 0);
-  reorder_pool_kernel<<<g.B * g.NT, kPoolThreads, 0, s>>>(a, reinterpret_cast<const uint4*>(x),
-                                                          reinterpret_cast<uint4*>(xt), xbar);
+  const dim3 grid(g.B * g.NT, ceil_div(g.H * (g.d / 8), kPoolThreads));
+  reorder_pool_kernel<<<grid, kPoolThreads, 0, s>>>(a, reinterpret_cast<const uint4*>(x),
+                                                    reinterpret_cast<uint4*>(xt), xbar);
   count_launches(1);
   return cudaGetLastError();
 }

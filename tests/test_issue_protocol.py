@@ -1,7 +1,7 @@
 """Discrete-event model of the persistent attention kernel's pipeline protocol (CPU only).
 
-The attention kernel hands work between a key-stream builder, a TMA producer, one
-MMA-issuing thread with two cursors (query blocks A and B) and two softmax warpgroups of
+The attention kernel hands work between a key-stream builder, two TMA producers (Q and
+the K ring; the V ring), one MMA-issuing thread with two cursors (query blocks A and B) and two softmax warpgroups of
 four warps, through mbarriers that are tested by phase parity. Units follow one another
 inside a CTA without a barrier between them. This model replays that protocol on
 sequences of units taken from real masks (and on edge cases: a missing query block, query
@@ -104,7 +104,7 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
     vfull, vempty = [Bar(1) for _ in range(NS)], [Bar(1) for _ in range(NS)]
     qfull, qempty = [Bar(1), Bar(1)], [Bar(1), Bar(1)]
     sfull, pfull, odone = [Bar(1), Bar(1)], [Bar(WARPS), Bar(WARPS)], [Bar(1), Bar(1)]
-    lfull, lempty = [Bar(1), Bar(1)], [Bar(1 + 2 + 2 * WARPS), Bar(1 + 2 + 2 * WARPS)]
+    lfull, lempty = [Bar(1), Bar(1)], [Bar(2 + 2 + 2 * WARPS), Bar(2 + 2 + 2 * WARPS)]
     # ------------------------------------------------------------------ state
     lists = [None, None]                      # key-stream buffers: unit index or 'end'
     kdata, vdata, qdata = [None] * NS, [None] * NS, [None, None]
@@ -115,8 +115,9 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
     pipe = []                                 # products / commits in issue order
 
     bld = {"it": 0, "next": 0, "done": False}
-    prod = {"it": 0, "state": "list", "unit": None, "c": 0, "qn": [0, 0], "nk": 0, "nv": 0, "x": 0,
-            "done": False}
+    # two producers: K (Q of each query block, then the K ring) and V (the V ring)
+    prods = [{"kind": kind, "it": 0, "state": "list", "unit": None, "c": 0, "qn": [0, 0], "n": 0, "x": 0,
+              "done": False} for kind in ("k", "v")]
 
     def new_cursor():
         return {"it": 0, "have": False, "done": False, "unit": None, "kc": 0, "vc": 0, "pend": -1,
@@ -156,8 +157,7 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
             bld["it"] += 1
         return [act]
 
-    def producer_actions():
-        p = prod
+    def producer_actions(p):
         if p["done"]:
             return []
         if p["state"] == "list":
@@ -170,7 +170,8 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
                 if ui == "end":
                     p["done"] = True
                     return
-                p["unit"], p["state"], p["x"], p["c"] = ui, "q", 0, 0
+                p["unit"], p["x"], p["c"] = ui, 0, 0
+                p["state"] = "q" if p["kind"] == "k" else "ring"
             return [act]
         ui = p["unit"]
         qs, ent = units[ui]
@@ -178,7 +179,7 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
             x = p["x"]
             if x == 2:
                 def act():
-                    p["state"] = "k"
+                    p["state"] = "ring"
                 return [act]
             if qs[2 * x] < 0:
                 def act():
@@ -199,27 +200,16 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
                 p["it"] += 1
                 p["state"] = "list"
             return [act]
-        if p["state"] == "k":
-            s, ph = p["nk"] % NS, ((p["nk"] // NS) & 1) ^ 1
-            if not kempty[s].test(ph):
-                return []
-
-            def act():
-                tag = (ui, p["c"])
-                inflight.append((kfull[s], lambda s=s, tag=tag: kdata.__setitem__(s, tag)))
-                p["nk"] += 1
-                p["state"] = "v"
-            return [act]
-        s, ph = p["nv"] % NS, ((p["nv"] // NS) & 1) ^ 1
-        if not vempty[s].test(ph):
+        s, ph = p["n"] % NS, ((p["n"] // NS) & 1) ^ 1
+        empty, full, data = (kempty, kfull, kdata) if p["kind"] == "k" else (vempty, vfull, vdata)
+        if not empty[s].test(ph):
             return []
 
         def act():
             tag = (ui, p["c"])
-            inflight.append((vfull[s], lambda s=s, tag=tag: vdata.__setitem__(s, tag)))
-            p["nv"] += 1
+            inflight.append((full[s], lambda s=s, tag=tag: data.__setitem__(s, tag)))
+            p["n"] += 1
             p["c"] += 1
-            p["state"] = "k"
         return [act]
 
     def release(passes, empty, x, gi):
@@ -420,7 +410,8 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
 
     for _ in range(2_000_000):
         fix_ordinals()
-        acts = builder_actions() + producer_actions() + cursor_actions(0) + cursor_actions(1) + pipe_actions()
+        acts = builder_actions() + producer_actions(prods[0]) + producer_actions(prods[1]) + \
+            cursor_actions(0) + cursor_actions(1) + pipe_actions()
         for x in range(2):
             for w in range(WARPS):
                 acts += softmax_actions(x, w)
@@ -432,7 +423,7 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
                 b.arrive()
             acts.append(land)
         if not acts:
-            done = bld["done"] and prod["done"] and all(c["done"] for c in cur) and \
+            done = bld["done"] and all(p["done"] for p in prods) and all(c["done"] for c in cur) and \
                 all(s["done"] for xs in sm for s in xs) and not pipe and not inflight
             return done
         rng.choice(acts)()
