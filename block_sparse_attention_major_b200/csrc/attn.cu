@@ -78,6 +78,7 @@ constexpr long long kWaitLimit = 4000000000LL;     // SM cycles, about 2 s
 constexpr int kTmemCols = 512;
 constexpr int kUnitInts = 8;                       // {bh, q0, q1, q2, q3, cost, 0, 0}
 constexpr float kRescaleLog2 = 8.0f;               // O is rescaled only past 2^8 of growth
+constexpr unsigned kIssuerBackoffNs = 32;          // issuer pause after a pass with nothing to issue
 
 template <int D>
 struct Cfg {
@@ -141,10 +142,6 @@ constexpr int kListConsumers = 2 + 2 + 8;
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
-}
-// The two bf16 values of a packed pair, widened exactly to fp32, summed.
-__device__ __forceinline__ float pair_sum(uint32_t w) {
-  return __uint_as_float(w << 16) + __uint_as_float(w & 0xffff0000u);
 }
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -218,47 +215,70 @@ __device__ __forceinline__ float half_max(const uint32_t (&r)[64], int use, uint
   return m;
 }
 
+// Packed pairs of fp32 (sm_100a f32x2 instructions: one instruction, two lanes of work).
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void uf2(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // p = 2^(s*c - m) for 64 score columns (zero on slots whose bit in `valid` is clear),
 // stored to TMEM as bf16 pairs (column 2i in the low half of 32-bit column i), 16 columns
 // per store. `sum` gets the fp32 probabilities, `sum_bf` the bf16-rounded ones that P.V
-// uses.
+// uses (widened from the packed pairs). The scaling and the sums run as packed f32x2
+// instructions: the softmax is bound by instruction issue, not by the exponentials.
 template <bool kMasked>
 __device__ __forceinline__ void exp_half(const uint32_t (&r)[64], uint64_t valid, float c, float m,
                                          float& sum, float& sum_bf, uint32_t taddr) {
   const uint32_t lo = (uint32_t)valid, hi = (uint32_t)(valid >> 32);
-  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-  float b0 = 0.f, b1 = 0.f;
+  const uint64_t cc = f2(c, c), mm = f2(-m, -m);
+  uint64_t ex0 = f2(0.f, 0.f), ex1 = ex0, bf0 = ex0, bf1 = ex0;   // two chains each
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     uint32_t pk[8];
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) {
+    for (int i = 0; i < 8; ++i) {
       const int b = 16 * k + 2 * i;
-      float p0 = ex2(fmaf(__uint_as_float(r[b + 0]), c, -m));
-      float p1 = ex2(fmaf(__uint_as_float(r[b + 1]), c, -m));
-      float p2 = ex2(fmaf(__uint_as_float(r[b + 2]), c, -m));
-      float p3 = ex2(fmaf(__uint_as_float(r[b + 3]), c, -m));
+      float x0, x1;
+      uf2(ffma2(f2(__uint_as_float(r[b]), __uint_as_float(r[b + 1])), cc, mm), x0, x1);
+      float p0 = ex2(x0), p1 = ex2(x1);
       if (kMasked) {
         const uint32_t w = b < 32 ? lo : hi;
         const int sh = b & 31;
         p0 = ((w >> sh) & 1u) ? p0 : 0.f;
         p1 = ((w >> (sh + 1)) & 1u) ? p1 : 0.f;
-        p2 = ((w >> (sh + 2)) & 1u) ? p2 : 0.f;
-        p3 = ((w >> (sh + 3)) & 1u) ? p3 : 0.f;
       }
       pk[i] = pack_bf16x2(p0, p1);
-      pk[i + 1] = pack_bf16x2(p2, p3);
-      s0 += p0;
-      s1 += p1;
-      s2 += p2;
-      s3 += p3;
-      b0 += pair_sum(pk[i]);
-      b1 += pair_sum(pk[i + 1]);
+      const uint64_t pe = f2(p0, p1);
+      const uint64_t pb = f2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xffff0000u));
+      if (i & 1) {
+        ex1 = fadd2(ex1, pe);
+        bf1 = fadd2(bf1, pb);
+      } else {
+        ex0 = fadd2(ex0, pe);
+        bf0 = fadd2(bf0, pb);
+      }
     }
     tmem_st_x8(taddr + 8 * k, pk);
   }
-  sum += (s0 + s1) + (s2 + s3);
-  sum_bf += b0 + b1;
+  float a0, a1, a2, a3;
+  uf2(fadd2(ex0, ex1), a0, a1);
+  sum += a0 + a1;
+  uf2(fadd2(bf0, bf1), a2, a3);
+  sum_bf += a2 + a3;
 }
 
 // Zero probabilities for a tile the row does not retain (32 TMEM columns of bf16 pairs).
@@ -558,7 +578,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // second cursor passes it, so both cursors' products on it are tracked by the commit.
     // Each cursor sees every load of the ring in order, so a full barrier is never more
     // than one phase behind the block tested and the parity tests are exact. Nothing
-    // blocks: one cursor waiting must not hold up the other.
+    // blocks: one cursor waiting must not hold up the other. A cursor takes its V position
+    // before its K position, so that a query block's P.V and its next Q K^T go to the pipe
+    // back to back: the other query block's products then run while this one's softmax
+    // works (the two softmax warpgroups alternate instead of running in step).
     if (lane == 0) {
       constexpr uint32_t kIdQK128 = ptx::idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t kIdQK64 = ptx::idesc_bf16_f32(128, 64, 0, 0);
@@ -617,6 +640,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             cu.first_pv = true;
             cu.flags = reinterpret_cast<const uint16_t*>(lb + C::kListMeta + kMaxTiles * 2);
           }
+          // ---- V position
+          if (cu.vc < cu.kc) {
+            const uint32_t gi = cu.gbase + (uint32_t)cu.vc;
+            const int s = (int)(gi % kNS);
+            const uint32_t fph = (uint32_t)((gi / kNS) & 1);
+            bool passed = false;
+            if (cu.vc == cu.pend) {
+              if (ptx::mbar_test_wait(bar.pfull(x), cu.pn & 1) && ptx::mbar_test_wait(bar.vfull(s), fph)) {
+                ptx::tc_fence_after();
+                const int u = block_use(cu.flags, cu.L, cu.vc, x);
+                const uint32_t o_tmem = tmem + 256u + (uint32_t)(x * D);
+                const uint32_t p_tmem = tmem + (uint32_t)(x * 128);
+                const uint64_t vd = ptx::smem_desc_sw128(sbase + C::kVOff + s * C::kOpBytes, C::kCB, 1024);
+                const int k0 = (u & 1) ? 0 : 4, k1 = (u & 2) ? 8 : 4;
+                for (int kk = k0; kk < k1; ++kk) {
+                  ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + (uint64_t)(kk * (2048 >> 4)), kIdPV,
+                              (cu.first_pv && kk == k0) ? 0u : 1u);
+                }
+                ptx::mma_commit(bar.odone(x));
+                cu.first_pv = false;
+                ++cu.pn;
+                cu.pend = -1;
+                passed = true;
+              }
+            } else {
+              passed = ptx::mbar_test_wait(bar.vfull(s), fph);
+            }
+            if (passed) {
+              vpass[x] = gi + 1u;
+              if ((int)(vpass[x ^ 1] - (gi + 1u)) >= 0) ptx::mma_commit(bar.vempty(s));
+              ++cu.vc;
+              progress = true;
+            }
+          }
           // ---- K position
           if (cu.kc < cu.nb) {
             const int u = cu.hasq ? block_use(cu.flags, cu.L, cu.kc, x) : 0;
@@ -658,40 +715,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               }
             }
           }
-          // ---- V position
-          if (cu.vc < cu.kc) {
-            const uint32_t gi = cu.gbase + (uint32_t)cu.vc;
-            const int s = (int)(gi % kNS);
-            const uint32_t fph = (uint32_t)((gi / kNS) & 1);
-            bool passed = false;
-            if (cu.vc == cu.pend) {
-              if (ptx::mbar_test_wait(bar.pfull(x), cu.pn & 1) && ptx::mbar_test_wait(bar.vfull(s), fph)) {
-                ptx::tc_fence_after();
-                const int u = block_use(cu.flags, cu.L, cu.vc, x);
-                const uint32_t o_tmem = tmem + 256u + (uint32_t)(x * D);
-                const uint32_t p_tmem = tmem + (uint32_t)(x * 128);
-                const uint64_t vd = ptx::smem_desc_sw128(sbase + C::kVOff + s * C::kOpBytes, C::kCB, 1024);
-                const int k0 = (u & 1) ? 0 : 4, k1 = (u & 2) ? 8 : 4;
-                for (int kk = k0; kk < k1; ++kk) {
-                  ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + (uint64_t)(kk * (2048 >> 4)), kIdPV,
-                              (cu.first_pv && kk == k0) ? 0u : 1u);
-                }
-                ptx::mma_commit(bar.odone(x));
-                cu.first_pv = false;
-                ++cu.pn;
-                cu.pend = -1;
-                passed = true;
-              }
-            } else {
-              passed = ptx::mbar_test_wait(bar.vfull(s), fph);
-            }
-            if (passed) {
-              vpass[x] = gi + 1u;
-              if ((int)(vpass[x ^ 1] - (gi + 1u)) >= 0) ptx::mma_commit(bar.vempty(s));
-              ++cu.vc;
-              progress = true;
-            }
-          }
           // ---- end of the unit
           if (cu.kc == cu.nb && cu.vc == cu.nb) {
             if (cu.hasq && !cu.qreleased) {
@@ -717,6 +740,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           *abort = 1;
           report_error(a.err, BSA_KERR_WAIT_TIMEOUT);
           ok = false;
+        } else {
+          // Nothing to issue: yield the sub-partition's issue slots to the two softmax
+          // warps that share it, instead of polling the barriers back to back.
+          __nanosleep(kIssuerBackoffNs);
         }
       }
       // Never free TMEM under a running MMA: wait until everything issued has completed.
