@@ -8,12 +8,12 @@
 // Work unit: up to four query tiles of one (b, h) and of the same route class (all
 // dense, or all local), consecutive in tile order. They form two query blocks of two
 // tiles, A and B, each one M=128 tcgen05 tile. The unit's key stream is the union of the
-// four rows' retained key tiles, ascending, taken two tiles (128 keys) per stream block.
-// For each stream block a query block uses one or both of its tiles (a tile is used when
-// either of the block's two query tiles retains it) or none; it then computes
-// S = Q K^T with N = 128 (both tiles) or N = 64 (one tile) and O += P V over the used keys.
-// A key tile retained by only one of the block's two query tiles gets zero probabilities
-// in the other query tile's rows.
+// four rows' retained key tiles, ascending, one tile (64 keys) per stream block, through a
+// K ring and a V ring of four stages. For each tile a query block uses (either of its two
+// query tiles retains it) it computes S = Q K^T (N = 64) and O += P V; a tile retained by
+// only one of the block's two query tiles gets zero probabilities in the other query
+// tile's rows. Each query block has two S buffers, so the Q K^T of its next tile runs
+// while its softmax works on the current one.
 //
 // Persistent grid: one CTA per SM takes units from a device work list through an atomic
 // counter. The list (built by the scheduler kernels below) is ordered head by head, and
@@ -28,26 +28,24 @@
 //   warps 4-7  softmax of query block B
 //              (each reads S from TMEM, writes P as bf16 pairs over S, rescales its O in
 //              TMEM when a row maximum grows by more than 2^8, and runs the epilogue)
-//   warp 8     lane 0 issues the TMA loads of Q and of the K ring
-//   warp 9     allocates TMEM; lane 0 issues every tcgen05.mma of both query blocks
+//   warp 8     lane 0 issues the TMA loads of Q and of the K ring, lane 1 those of the V
+//              ring (neither ring waits behind the other)
+//   warp 9     allocates TMEM; lane 0 issues every tcgen05.mma of query block A
 //   warp 10    takes the next unit from the work list and builds its key stream in shared
 //              memory (double buffered, one unit ahead)
-//   warp 11    lane 0 issues the TMA loads of the V ring
+//   warp 11    lane 0 issues every tcgen05.mma of query block B
 // The softmax warpgroups raise their register budget to 184 and the third lowers its own to
-// 136 (setmaxnreg); the softmax holds 64 score columns of a row at a time, reading a
-// 128-column block from TMEM twice.
-// TMEM columns: S_A at 0, S_B at 128 (128 each; P is written over S as bf16 pairs, key k of
-// the block at column k/2), O_A at 256, O_B at 256 + D. Shared memory (1024-byte aligned):
-// Q_A, Q_B, two K and two V stages, each a 128-row operand laid out as [D/64 column
-// blocks][128 rows][128 B] with the 128-byte swizzle that TMA and tcgen05 share (a K or V
-// stage holds the stream block's first tile in rows 0-63, its second in rows 64-127); two
-// key-stream buffers; barriers.
+// 136 (setmaxnreg).
+// TMEM columns: S buffer b of query block x at 64 (2x + b) (64 each; P is written over S as
+// bf16 pairs, key k of the tile at column k/2), O_A at 256, O_B at 256 + D. Shared memory
+// (1024-byte aligned): Q_A, Q_B as [D/64 column blocks][128 rows][128 B], four K and four V
+// stages as [D/64][64 rows][128 B], each with the 128-byte swizzle that TMA and tcgen05
+// share; two key-stream buffers; barriers.
 //
 // Softmax numerics. Scores are scaled by softmax_scale * log2(e) with one FFMA and
 // exponentiated with ex2.approx. A row keeps a reference maximum m and is rescaled only
-// when a block's maximum exceeds m by more than 8 (then O and the row sums are multiplied
-// by 2^(m - m_new); the previous P.V has completed by then, since the pipe ran it before
-// this block's Q K^T); otherwise probabilities up to
+// when a block's maximum exceeds m by more than 8 (then, after the previous block's P.V has
+// completed, O and the row sums are multiplied by 2^(m - m_new)); otherwise probabilities up to
 // 2^8 enter P. O is normalised by the sum of the bf16-rounded probabilities that entered
 // P.V (so a row dominated by one key returns that key's value exactly); the LSE uses the
 // fp32 sum of the unrounded probabilities.
@@ -73,7 +71,7 @@ constexpr int kRegsSoftmax = 184;
 constexpr int kRegsControl = 136;
 static_assert(128 * (2 * kRegsSoftmax + kRegsControl) <= kAttnThreads * kRegsLaunch,
               "register split above the launch's pool");
-constexpr int kNS = 2;                             // K and V ring stages, two key tiles each
+constexpr int kNS = 4;                             // K and V ring stages, one key tile each
 constexpr long long kWaitLimit = 4000000000LL;     // SM cycles, about 2 s
 constexpr int kTmemCols = 512;
 constexpr int kUnitInts = 8;                       // {bh, q0, q1, q2, q3, cost, 0, 0}
@@ -82,23 +80,24 @@ constexpr unsigned kIssuerBackoffNs = 32;          // issuer pause after a pass 
 
 template <int D>
 struct Cfg {
-  static constexpr int kTileBytes = 64 * D * 2;         // one 64-token tile
-  static constexpr int kOpBytes = 2 * kTileBytes;       // one 128-row operand
-  static constexpr int kCB = 128 * 128;                 // bytes between 64-column blocks
-  static constexpr int kHalf = 64 * 128;                // rows 64-127 start here in a block
+  static constexpr int kTileBytes = 64 * D * 2;         // one 64-token tile (a K or V stage)
+  static constexpr int kQBytes = 2 * kTileBytes;        // one query block (128 rows)
+  static constexpr int kQCB = 128 * 128;                // Q: bytes between 64-column blocks
+  static constexpr int kKCB = 64 * 128;                 // K/V stage: bytes between 64-column blocks
+  static constexpr int kHalf = 64 * 128;                // rows 64-127 of a query block start here
   static constexpr int kQOff = 0;                       // Q_A, then Q_B
-  static constexpr int kKOff = 2 * kOpBytes;
-  static constexpr int kVOff = kKOff + kNS * kOpBytes;
-  static constexpr int kListOff = kVOff + kNS * kOpBytes;
+  static constexpr int kKOff = 2 * kQBytes;
+  static constexpr int kVOff = kKOff + kNS * kTileBytes;
+  static constexpr int kListOff = kVOff + kNS * kTileBytes;
   // key-stream buffer: meta (8 ints: bh or -1, q0..q3, L), tile ids (u16), flags (u16:
   // bit t = query tile t retains the tile, bit 4 = the tile has no padding slot, bit 5 + t
   // = query tile t sees the tile through its tokens' support)
   static constexpr int kListMeta = 32;
   static constexpr int kListBytes = kListMeta + kMaxTiles * 2 + kMaxTiles * 2;
   static constexpr int kBarOff = kListOff + 2 * kListBytes;
-  // kfull, kempty, vfull, vempty [kNS each]; qfull, qempty, sfull, pfull, odone [2 each];
-  // lfull, lempty [2 each]; drain
-  static constexpr int kNumBars = 4 * kNS + 5 * 2 + 2 * 2 + 1;
+  // kfull, kempty, vfull, vempty [kNS each]; qfull, qempty [2 each]; sfull, pfull, odone
+  // [query block][S buffer]; lfull, lempty [2 each]; drain [one per issuer]
+  static constexpr int kNumBars = 4 * kNS + 2 * 2 + 3 * 4 + 2 * 2 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base, abort
   static constexpr int kSmemBytes = 1024 + kMiscOff + 64;
   static_assert(kSmemBytes <= 232448, "shared memory");
@@ -127,15 +126,15 @@ struct Bars {
   __device__ uint32_t vempty(int s) const { return b0 + 8 * (3 * kNS + s); }
   __device__ uint32_t qfull(int x) const { return b0 + 8 * (4 * kNS + x); }
   __device__ uint32_t qempty(int x) const { return b0 + 8 * (4 * kNS + 2 + x); }
-  __device__ uint32_t sfull(int x) const { return b0 + 8 * (4 * kNS + 4 + x); }
-  __device__ uint32_t pfull(int x) const { return b0 + 8 * (4 * kNS + 6 + x); }
-  __device__ uint32_t odone(int x) const { return b0 + 8 * (4 * kNS + 8 + x); }
-  __device__ uint32_t lfull(int b) const { return b0 + 8 * (4 * kNS + 10 + b); }
-  __device__ uint32_t lempty(int b) const { return b0 + 8 * (4 * kNS + 12 + b); }
-  __device__ uint32_t drain() const { return b0 + 8 * (4 * kNS + 14); }
+  __device__ uint32_t sfull(int x, int b) const { return b0 + 8 * (4 * kNS + 4 + 2 * x + b); }
+  __device__ uint32_t pfull(int x, int b) const { return b0 + 8 * (4 * kNS + 8 + 2 * x + b); }
+  __device__ uint32_t odone(int x, int b) const { return b0 + 8 * (4 * kNS + 12 + 2 * x + b); }
+  __device__ uint32_t lfull(int b) const { return b0 + 8 * (4 * kNS + 16 + b); }
+  __device__ uint32_t lempty(int b) const { return b0 + 8 * (4 * kNS + 18 + b); }
+  __device__ uint32_t drain(int x) const { return b0 + 8 * (4 * kNS + 20 + x); }
 };
 
-// lempty arrivals per key-stream buffer: the two TMA producers, the two issuer cursors and
+// lempty arrivals per key-stream buffer: the two TMA producers, the two issuers and
 // the eight softmax warps.
 constexpr int kListConsumers = 2 + 2 + 8;
 
@@ -319,13 +318,6 @@ __device__ __forceinline__ void rescale_o(uint32_t o_tmem, float alpha) {
   }
 }
 
-// Which tiles of stream block c query block x uses: bit 0 the first tile, bit 1 the second.
-__device__ __forceinline__ int block_use(const uint16_t* flags, int L, int c, int x) {
-  const uint32_t f0 = flags[2 * c];
-  const uint32_t f1 = 2 * c + 1 < L ? flags[2 * c + 1] : 0u;
-  return (((f0 >> (2 * x)) & 3u) ? 1 : 0) | (((f1 >> (2 * x)) & 3u) ? 2 : 0);
-}
-
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -345,20 +337,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNS; ++s) {
       ptx::mbar_init(bar.kfull(s), 1);
-      ptx::mbar_init(bar.kempty(s), 1);
+      ptx::mbar_init(bar.kempty(s), 2);   // one release per issuer
       ptx::mbar_init(bar.vfull(s), 1);
-      ptx::mbar_init(bar.vempty(s), 1);
+      ptx::mbar_init(bar.vempty(s), 2);
     }
     for (int x = 0; x < 2; ++x) {
       ptx::mbar_init(bar.qfull(x), 1);
       ptx::mbar_init(bar.qempty(x), 1);
-      ptx::mbar_init(bar.sfull(x), 1);
-      ptx::mbar_init(bar.pfull(x), 4);        // one arrival per softmax warp
-      ptx::mbar_init(bar.odone(x), 1);
+      for (int b = 0; b < 2; ++b) {
+        ptx::mbar_init(bar.sfull(x, b), 1);
+        ptx::mbar_init(bar.pfull(x, b), 4);   // one arrival per softmax warp
+        ptx::mbar_init(bar.odone(x, b), 1);
+      }
       ptx::mbar_init(bar.lfull(x), 1);
       ptx::mbar_init(bar.lempty(x), kListConsumers);
     }
-    ptx::mbar_init(bar.drain(), 1);
+    ptx::mbar_init(bar.drain(0), 1);
+    ptx::mbar_init(bar.drain(1), 1);
     *abort = 0;
     ptx::fence_mbar_init();
   }
@@ -480,12 +475,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar.lfull(buf));
     }
-  } else if (warp == 8 || warp == 11) {
+  } else if (warp == 8) {
     // ------------------------------------------------------------------ TMA producers
-    // Lane 0 of warp 8 loads Q and the K ring, lane 0 of warp 11 the V ring, so that a K
-    // stage never waits behind a V stage (or the reverse).
-    const bool vprod = warp == 11;
-    if (lane == 0) {
+    // Lane 0 of warp 8 loads Q and the K ring, lane 1 the V ring, so that a K stage never
+    // waits behind a V stage (or the reverse).
+    const bool vprod = lane == 1;
+    if (lane <= 1) {
       ptx::prefetch_tensormap(&tmQ);
       ptx::prefetch_tensormap(&tmK);
       ptx::prefetch_tensormap(&tmV);
@@ -509,44 +504,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             ok = false;
             break;
           }
-          ptx::mbar_arrive_expect_tx(bar.qfull(x), C::kOpBytes);
+          ptx::mbar_arrive_expect_tx(bar.qfull(x), C::kQBytes);
           for (int rh = 0; rh < 2; ++rh) {
             const int tile = q[2 * x + rh] >= 0 ? q[2 * x + rh] : q[2 * x];   // a missing tile repeats the first
             const int row = (int)((tile_row0 + tile) * 64);
-            const uint32_t dst = sbase + C::kQOff + x * C::kOpBytes + rh * C::kHalf;
+            const uint32_t dst = sbase + C::kQOff + x * C::kQBytes + rh * C::kHalf;
 #pragma unroll
-            for (int cb = 0; cb < D / 64; ++cb) ptx::tma_load_2d(dst + cb * C::kCB, &tmQ, bar.qfull(x), cb * 64, row);
+            for (int cb = 0; cb < D / 64; ++cb) ptx::tma_load_2d(dst + cb * C::kQCB, &tmQ, bar.qfull(x), cb * 64, row);
           }
           ++qn[x];
         }
-        const int nb = (L + 1) / 2;
-        for (int c = 0; c < nb && ok; ++c) {
-          const int nh = 2 * c + 1 < L ? 2 : 1;
-          if (!vprod) {
-            const int s = (int)(nk % kNS);
-            const uint32_t ph = ((nk / kNS) & 1) ^ 1;
-            if (!ptx::mbar_wait(bar.kempty(s), ph, abort, a.err, kWaitLimit)) { ok = false; break; }
-            ptx::mbar_arrive_expect_tx(bar.kfull(s), nh * C::kTileBytes);
-            for (int h = 0; h < nh; ++h) {
-              const int row = (int)((tile_row0 + tiles[2 * c + h]) * 64);
-              const uint32_t dst = sbase + C::kKOff + s * C::kOpBytes + h * C::kHalf;
+        for (int c = 0; c < L && ok; ++c) {
+          const int row = (int)((tile_row0 + tiles[c]) * 64);
+          uint32_t& n = vprod ? nv : nk;
+          const int s = (int)(n % kNS);
+          const uint32_t ph = ((n / kNS) & 1) ^ 1;
+          const uint32_t empty = vprod ? bar.vempty(s) : bar.kempty(s);
+          const uint32_t full = vprod ? bar.vfull(s) : bar.kfull(s);
+          if (!ptx::mbar_wait(empty, ph, abort, a.err, kWaitLimit)) { ok = false; break; }
+          ptx::mbar_arrive_expect_tx(full, C::kTileBytes);
+          const uint32_t dst = sbase + (vprod ? C::kVOff : C::kKOff) + s * C::kTileBytes;
 #pragma unroll
-              for (int cb = 0; cb < D / 64; ++cb) ptx::tma_load_2d(dst + cb * C::kCB, &tmK, bar.kfull(s), cb * 64, row);
-            }
-            ++nk;
-          } else {
-            const int s = (int)(nv % kNS);
-            const uint32_t ph = ((nv / kNS) & 1) ^ 1;
-            if (!ptx::mbar_wait(bar.vempty(s), ph, abort, a.err, kWaitLimit)) { ok = false; break; }
-            ptx::mbar_arrive_expect_tx(bar.vfull(s), nh * C::kTileBytes);
-            for (int h = 0; h < nh; ++h) {
-              const int row = (int)((tile_row0 + tiles[2 * c + h]) * 64);
-              const uint32_t dst = sbase + C::kVOff + s * C::kOpBytes + h * C::kHalf;
-#pragma unroll
-              for (int cb = 0; cb < D / 64; ++cb) ptx::tma_load_2d(dst + cb * C::kCB, &tmV, bar.vfull(s), cb * 64, row);
-            }
-            ++nv;
-          }
+          for (int cb = 0; cb < D / 64; ++cb) ptx::tma_load_2d(dst + cb * C::kKCB, vprod ? &tmV : &tmK, full, cb * 64, row);
+          ++n;
         }
         if (ok) ptx::mbar_arrive(bar.lempty(buf));
       }
@@ -565,75 +545,67 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int x = 0; x < 2; ++x)
         if (qn[x] > 0) ptx::mbar_wait(bar.qfull(x), (qn[x] - 1) & 1, &zero, a.err, kWaitLimit);
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------------ MMA issuer
-    // Lane 0 issues every product of both query blocks. Two cursors (A and B) walk the
-    // units' stream blocks in order, each with a K position and a V position. At its K
-    // position a cursor issues S = Q K^T for a block its query block uses, once the K
-    // stage is in and its single S buffer is free (the P.V of its previous block has been
-    // issued: the tensor pipe runs one thread's products in issue order, so S may
-    // overwrite that P); at its V position it issues O += P V once its softmax has written
-    // P and the V stage is in. A block the query block does not use is passed once its
-    // stage is seen loaded. A stage is released (one commit on its empty barrier) when the
-    // second cursor passes it, so both cursors' products on it are tracked by the commit.
-    // Each cursor sees every load of the ring in order, so a full barrier is never more
-    // than one phase behind the block tested and the parity tests are exact. Nothing
-    // blocks: one cursor waiting must not hold up the other. A cursor takes its V position
-    // before its K position, so that a query block's P.V and its next Q K^T go to the pipe
-    // back to back: the other query block's products then run while this one's softmax
-    // works (the two softmax warpgroups alternate instead of running in step).
+  } else if (warp == 9 || warp == 11) {
+    // ------------------------------------------------------------------ MMA issuers
+    // Lane 0 of warp 9 issues every product of query block A, lane 0 of warp 11 those of
+    // B: each MMA issue waits for the tensor pipe to take it, so one thread for both query
+    // blocks could not keep the pipe fed. Each issuer's cursor walks the units' key streams
+    // in order with a K position and a V position; each query block has two S buffers in
+    // TMEM. At its K position a cursor issues S = Q K^T (N = 64) for a tile its query
+    // block uses into the next S buffer, once the K stage is in and that buffer is free:
+    // the P.V of the block two back has been issued (the tensor pipe runs one thread's
+    // products in issue order, so S may overwrite that P). At its V position it issues
+    // O += P V for the oldest block whose P.V is pending, once its softmax has released P
+    // and the V stage is in. A tile the query block does not use is passed once its stage
+    // is seen loaded. Each issuer releases each stage once (a commit after its product on
+    // it, or an arrive when it passed the tile); a stage is reloaded after both releases,
+    // and a commit tracks its own thread's products. Each cursor sees every load of the
+    // ring in order, so a full barrier is never more than one phase behind the tile tested
+    // and the parity tests are exact. The cursor takes its V position before its K
+    // position, so that a query block's P.V and its next Q K^T go to the pipe back to back.
+    const int x = warp == 9 ? 0 : 1;           // query block of this issuer
     if (lane == 0) {
-      constexpr uint32_t kIdQK128 = ptx::idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t kIdQK64 = ptx::idesc_bf16_f32(128, 64, 0, 0);
+      constexpr uint32_t kIdQK = ptx::idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t kIdPV = ptx::idesc_bf16_f32(128, D, 0, 1);
       struct Cursor {
         int it;            // key-stream buffer iteration
         bool have, done;
-        int L, nb, kc, vc, pend;
+        int L, kc, vc;     // unit's stream length; next K and V positions
         bool hasq, qready, qreleased, first_pv;
-        uint32_t gbase;    // index of the unit's first stream block in this CTA's stream
+        uint32_t gbase;    // index of the unit's first stream tile in this CTA's stream
         int qn;            // Q loads consumed (units with this query block)
-        uint32_t pn;       // P.V products issued (= pfull phases consumed)
+        uint32_t qk, pv;   // Q K^T and P.V products issued (all units)
+        int ent0, ent1;    // stream positions of the blocks whose P.V is pending, by S buffer
         const uint16_t* flags;
       };
-      Cursor cur[2];
-      for (int x = 0; x < 2; ++x) {
-        cur[x].it = 0;
-        cur[x].have = cur[x].done = false;
-        cur[x].L = cur[x].nb = cur[x].kc = cur[x].vc = 0;
-        cur[x].pend = -1;
-        cur[x].hasq = cur[x].qready = cur[x].qreleased = cur[x].first_pv = false;
-        cur[x].gbase = 0;
-        cur[x].qn = 0;
-        cur[x].pn = 0;
-        cur[x].flags = nullptr;
-      }
-      // stream blocks each cursor has passed (modulo 2^32: the cursors stay within a ring
-      // length of each other, so differences decide the order)
-      uint32_t kpass[2] = {0u, 0u}, vpass[2] = {0u, 0u};
+      Cursor cu;
+      cu.it = 0;
+      cu.have = cu.done = false;
+      cu.L = cu.kc = cu.vc = 0;
+      cu.hasq = cu.qready = cu.qreleased = cu.first_pv = false;
+      cu.gbase = 0;
+      cu.qn = 0;
+      cu.qk = cu.pv = 0;
+      cu.ent0 = cu.ent1 = -1;
+      cu.flags = nullptr;
       bool ok = true;
       long long idle_since = clock64();
-      while (ok && !(cur[0].done && cur[1].done)) {
+      while (ok && !cu.done) {
         bool progress = false;
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          Cursor& cu = cur[x];
-          if (cu.done) continue;
+        do {
           if (!cu.have) {
             const int buf = cu.it & 1;
-            if (!ptx::mbar_test_wait(bar.lfull(buf), (cu.it >> 1) & 1)) continue;
+            if (!ptx::mbar_test_wait(bar.lfull(buf), (cu.it >> 1) & 1)) break;
             const uint8_t* lb = smem + C::kListOff + buf * C::kListBytes;
             const int* meta = reinterpret_cast<const int*>(lb);
             progress = true;
             if (meta[0] < 0) {
               cu.done = true;
-              continue;
+              break;
             }
             cu.have = true;
             cu.L = meta[5];
-            cu.nb = (cu.L + 1) / 2;
             cu.kc = cu.vc = 0;
-            cu.pend = -1;
             cu.hasq = meta[1 + 2 * x] >= 0;
             cu.qready = false;
             cu.qreleased = false;
@@ -645,82 +617,78 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const uint32_t gi = cu.gbase + (uint32_t)cu.vc;
             const int s = (int)(gi % kNS);
             const uint32_t fph = (uint32_t)((gi / kNS) & 1);
-            bool passed = false;
-            if (cu.vc == cu.pend) {
-              if (ptx::mbar_test_wait(bar.pfull(x), cu.pn & 1) && ptx::mbar_test_wait(bar.vfull(s), fph)) {
+            bool passed = false, issued_pv = false;
+            if (cu.pv != cu.qk && cu.vc == ((cu.pv & 1) ? cu.ent1 : cu.ent0)) {
+              const int b = (int)(cu.pv & 1);
+              if (ptx::mbar_test_wait(bar.pfull(x, b), (cu.pv >> 1) & 1) && ptx::mbar_test_wait(bar.vfull(s), fph)) {
                 ptx::tc_fence_after();
-                const int u = block_use(cu.flags, cu.L, cu.vc, x);
                 const uint32_t o_tmem = tmem + 256u + (uint32_t)(x * D);
-                const uint32_t p_tmem = tmem + (uint32_t)(x * 128);
-                const uint64_t vd = ptx::smem_desc_sw128(sbase + C::kVOff + s * C::kOpBytes, C::kCB, 1024);
-                const int k0 = (u & 1) ? 0 : 4, k1 = (u & 2) ? 8 : 4;
-                for (int kk = k0; kk < k1; ++kk) {
+                const uint32_t p_tmem = tmem + (uint32_t)(64 * (2 * x + b));
+                const uint64_t vd = ptx::smem_desc_sw128(sbase + C::kVOff + s * C::kTileBytes, C::kKCB, 1024);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
                   ptx::mma_ts(o_tmem, p_tmem + kk * 8, vd + (uint64_t)(kk * (2048 >> 4)), kIdPV,
-                              (cu.first_pv && kk == k0) ? 0u : 1u);
-                }
-                ptx::mma_commit(bar.odone(x));
+                              (cu.first_pv && kk == 0) ? 0u : 1u);
+                ptx::mma_commit(bar.odone(x, b));
                 cu.first_pv = false;
-                ++cu.pn;
-                cu.pend = -1;
+                ++cu.pv;
                 passed = true;
+                issued_pv = true;
               }
             } else {
               passed = ptx::mbar_test_wait(bar.vfull(s), fph);
             }
             if (passed) {
-              vpass[x] = gi + 1u;
-              if ((int)(vpass[x ^ 1] - (gi + 1u)) >= 0) ptx::mma_commit(bar.vempty(s));
+              if (issued_pv) ptx::mma_commit(bar.vempty(s));
+              else ptx::mbar_arrive(bar.vempty(s));
               ++cu.vc;
               progress = true;
             }
           }
           // ---- K position
-          if (cu.kc < cu.nb) {
-            const int u = cu.hasq ? block_use(cu.flags, cu.L, cu.kc, x) : 0;
+          if (cu.kc < cu.L) {
+            const bool used = cu.hasq && ((cu.flags[cu.kc] >> (2 * x)) & 3u) != 0u;
             const uint32_t gi = cu.gbase + (uint32_t)cu.kc;
             const int s = (int)(gi % kNS);
             const uint32_t fph = (uint32_t)((gi / kNS) & 1);
             bool passed = false;
-            if (u == 0) {
+            if (!used) {
               passed = ptx::mbar_test_wait(bar.kfull(s), fph);
-            } else if (cu.pend < 0) {
+            } else if (cu.qk - cu.pv < 2u) {
               if (!cu.qready) cu.qready = ptx::mbar_test_wait(bar.qfull(x), cu.qn & 1);
               if (cu.qready && ptx::mbar_test_wait(bar.kfull(s), fph)) {
-                // S = Q K^T over the used tiles: N = 128 for both, N = 64 for one (its
-                // columns at 64 * tile in S).
-                const int h0 = u == 2 ? 1 : 0;
-                const uint32_t s_tmem = tmem + (uint32_t)(x * 128 + h0 * 64);
-                const uint64_t qd = ptx::smem_desc_sw128(sbase + C::kQOff + x * C::kOpBytes, 16, 1024);
-                const uint64_t kd =
-                    ptx::smem_desc_sw128(sbase + C::kKOff + s * C::kOpBytes + h0 * C::kHalf, 16, 1024);
-                const uint32_t id = u == 3 ? kIdQK128 : kIdQK64;
+                const int b = (int)(cu.qk & 1);
+                const uint32_t s_tmem = tmem + (uint32_t)(64 * (2 * x + b));
+                const uint64_t qd = ptx::smem_desc_sw128(sbase + C::kQOff + x * C::kQBytes, 16, 1024);
+                const uint64_t kd = ptx::smem_desc_sw128(sbase + C::kKOff + s * C::kTileBytes, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                  const uint32_t off = (uint32_t)(((kk >> 2) * C::kCB + (kk & 3) * 32) >> 4);
-                  ptx::mma_ss(s_tmem, qd + off, kd + off, id, kk > 0 ? 1u : 0u);
-                }
-                ptx::mma_commit(bar.sfull(x));
-                cu.pend = cu.kc;
+                for (int kk = 0; kk < D / 16; ++kk)
+                  ptx::mma_ss(s_tmem, qd + (uint64_t)(((kk >> 2) * C::kQCB + (kk & 3) * 32) >> 4),
+                              kd + (uint64_t)(((kk >> 2) * C::kKCB + (kk & 3) * 32) >> 4), kIdQK, kk > 0 ? 1u : 0u);
+                ptx::mma_commit(bar.sfull(x, b));
+                if (b) cu.ent1 = cu.kc;
+                else cu.ent0 = cu.kc;
+                ++cu.qk;
                 passed = true;
               }
             }
             if (passed) {
-              kpass[x] = gi + 1u;
-              if ((int)(kpass[x ^ 1] - (gi + 1u)) >= 0) ptx::mma_commit(bar.kempty(s));
+              if (used) ptx::mma_commit(bar.kempty(s));
+              else ptx::mbar_arrive(bar.kempty(s));
               ++cu.kc;
               progress = true;
-              if (cu.kc == cu.nb && cu.hasq && cu.qready && !cu.qreleased) {
+              if (cu.kc == cu.L && cu.hasq && cu.qready && !cu.qreleased) {
                 ptx::mma_commit(bar.qempty(x));      // the unit's last Q K^T has been issued
                 cu.qreleased = true;
               }
             }
           }
           // ---- end of the unit
-          if (cu.kc == cu.nb && cu.vc == cu.nb) {
+          if (cu.kc == cu.L && cu.vc == cu.L) {
             if (cu.hasq && !cu.qreleased) {
               // No product used Q (its rows retain nothing here): release it once loaded.
               if (!cu.qready) cu.qready = ptx::mbar_test_wait(bar.qfull(x), cu.qn & 1);
-              if (!cu.qready) continue;
+              if (!cu.qready) break;
               ptx::mma_commit(bar.qempty(x));
               cu.qreleased = true;
             }
@@ -728,10 +696,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             ptx::mbar_arrive(bar.lempty(cu.it & 1));
             ++cu.it;
             cu.have = false;
-            cu.gbase += (uint32_t)cu.nb;
+            cu.gbase += (uint32_t)cu.L;
             progress = true;
           }
-        }
+        } while (false);
         if (progress) {
           idle_since = clock64();
         } else if (*abort) {
@@ -748,8 +716,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       // Never free TMEM under a running MMA: wait until everything issued has completed.
       int zero = 0;
-      ptx::mma_commit(bar.drain());
-      ptx::mbar_wait(bar.drain(), 0, &zero, a.err, kWaitLimit);
+      ptx::mma_commit(bar.drain(x));
+      ptx::mbar_wait(bar.drain(x), 0, &zero, a.err, kWaitLimit);
     }
   }
   } else {
@@ -760,7 +728,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int rh = row >> 6;                 // which of the block's two query tiles
     const int t = 2 * x + rh;                // query tile slot in the unit
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t s_tmem = tmem + (uint32_t)(x * 128) + lane_base;
+    const uint32_t s_tmem0 = tmem + (uint32_t)(128 * x) + lane_base;   // S buffer b at + 64 b
     const uint32_t o_tmem = tmem + 256u + (uint32_t)(x * D) + lane_base;
     const float c = a.scale_log2;
     uint32_t sidx = 0;                       // blocks processed (sfull / pfull phases)
@@ -775,7 +743,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (bh < 0) break;
       const int qt = meta[1 + t];
       const int L = meta[5];
-      const int nb = (L + 1) / 2;
       int tq = 0, yq = 0, xq = 0;            // this row's token (the token support's centre)
       {
         int tt, ty, tx;
@@ -788,42 +755,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float m_run = -INFINITY, l_ex = 0.f, l_bf = 0.f;
       int nused = 0;
       bool ok = true;
-      for (int cb = 0; cb < nb; ++cb) {
-        const int u = meta[1 + 2 * x] >= 0 ? block_use(flags, L, cb, x) : 0;
-        if (!u) continue;
-        const uint32_t f0 = flags[2 * cb];
-        const uint32_t f1 = 2 * cb + 1 < L ? flags[2 * cb + 1] : 0u;
-        const int use0 = (u & 1) ? tile_use(f0, t) : kUseSkip;
-        const int use1 = (u & 2) ? tile_use(f1, t) : kUseSkip;
-        const uint64_t valid0 =
-            use0 == kUsePartial ? tile_slots(tiles[2 * cb], f0, t, g, tq, yq, xq, a.token_rho) : ~0ull;
-        const uint64_t valid1 =
-            use1 == kUsePartial ? tile_slots(tiles[2 * cb + 1], f1, t, g, tq, yq, xq, a.token_rho) : ~0ull;
-        if (!warp_wait(bar.sfull(x), sidx & 1, abort, a.err)) { ok = false; break; }
+      for (int cb = 0; cb < L; ++cb) {
+        const uint32_t f = flags[cb];
+        if (meta[1 + 2 * x] < 0 || ((f >> (2 * x)) & 3u) == 0u) continue;   // not used by this query block
+        const int use = tile_use(f, t);
+        const uint64_t valid = use == kUsePartial ? tile_slots(tiles[cb], f, t, g, tq, yq, xq, a.token_rho) : ~0ull;
+        const int b = (int)(sidx & 1);
+        const uint32_t s_tmem = s_tmem0 + 64u * (uint32_t)b;
+        if (!warp_wait(bar.sfull(x, b), (sidx >> 1) & 1, abort, a.err)) { ok = false; break; }
         ptx::tc_fence_after();
-        // The block is read from TMEM twice, 64 columns at a time: once for the maximum
-        // (second tile first, so the first tile's columns are still in registers), once
-        // for the exponentials (first tile first: its P overwrites only its own, already
-        // read, S columns; the second tile's P then overwrites the first tile's upper S
-        // columns, which are no longer needed).
         uint32_t r[64];
         float mx = -INFINITY;
-        if (u & 2) {
-          load_half(s_tmem + 64, r);
-          mx = half_max(r, use1, valid1, mx);
-        }
-        if (u & 1) {
-          load_half(s_tmem + 0, r);
-          mx = half_max(r, use0, valid0, mx);
+        if (use != kUseSkip) {
+          load_half(s_tmem, r);
+          mx = half_max(r, use, valid, mx);
         }
         const float mb = mx * c;                       // block maximum, log2 domain
         bool resc = false;
         if (m_run == -INFINITY) m_run = mb;            // O of this row is still zero
         else if (mb > m_run + kRescaleLog2) resc = true;
         if (__any_sync(0xffffffffu, resc)) {
-          // O holds exactly the unit's earlier blocks here: the issuer sent this block's
-          // Q K^T after the previous block's P.V, the pipe ran them in that order, and S of
-          // this block is complete.
+          // O must hold exactly the unit's earlier blocks: wait for the previous block's
+          // P.V (the block two back has completed: this block's Q K^T followed its P.V).
+          if (!warp_wait(bar.odone(x, (int)((sidx - 1) & 1)), ((sidx - 1) >> 1) & 1, abort, a.err)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
           const float alpha = resc ? ex2(m_run - mb) : 1.0f;
           rescale_o<D>(o_tmem, alpha);
           l_ex *= alpha;
@@ -831,15 +789,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (resc) m_run = mb;
         }
         const float m_use = m_run == -INFINITY ? 0.0f : m_run;
-        if (u & 1) half_exp(r, use0, valid0, c, m_use, l_ex, l_bf, s_tmem + 0);
-        if (u & 2) {
-          if (u & 1) load_half(s_tmem + 64, r);       // (with the second tile alone, r holds it)
-          half_exp(r, use1, valid1, c, m_use, l_ex, l_bf, s_tmem + 32);
-        }
+        half_exp(r, use, valid, c, m_use, l_ex, l_bf, s_tmem);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar.pfull(x));
+        if (lane == 0) ptx::mbar_arrive(bar.pfull(x, b));
         ++sidx;
         ++nused;
       }
@@ -857,7 +811,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (tk < g.T && y < g.Hs && xx < g.Ws) n_tok = (tk * g.Hs + y) * g.Ws + xx;
       }
       if (nused > 0) {
-        if (!warp_wait(bar.odone(x), (sidx - 1) & 1, abort, a.err)) break;
+        if (!warp_wait(bar.odone(x, (int)((sidx - 1) & 1)), ((sidx - 1) >> 1) & 1, abort, a.err)) break;
         ptx::tc_fence_after();
       }
       const float inv_l = l_bf > 0.f ? 1.0f / l_bf : 0.f;

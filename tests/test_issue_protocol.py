@@ -1,33 +1,35 @@
 """Discrete-event model of the persistent attention kernel's pipeline protocol (CPU only).
 
 The attention kernel hands work between a key-stream builder, two TMA producers (Q and
-the K ring; the V ring), one MMA-issuing thread with two cursors (query blocks A and B) and two softmax warpgroups of
-four warps, through mbarriers that are tested by phase parity. Units follow one another
+the K ring; the V ring), two MMA-issuing threads (one per query block, A and B) and two
+softmax warpgroups of four warps, through mbarriers that are tested by phase parity. Units follow one another
 inside a CTA without a barrier between them. This model replays that protocol on
 sequences of units taken from real masks (and on edge cases: a missing query block, query
 tiles that retain nothing, odd stream lengths) under random interleavings, and checks that
 it always finishes (no deadlock) and that every read sees what it should:
 
-  * each Q K^T product the Q of its own unit and the K tiles of its own stream block;
-  * each softmax warp the S of its own block;
-  * each P.V the P of its own block, the V tiles of its block, and O holding exactly the
+  * each Q K^T product the Q of its own unit and the K tile of its own stream position;
+  * each softmax warp the S of its own block, in the S buffer the block went to;
+  * each P.V the P of its own block, the V tile of its block, and O holding exactly the
     unit's earlier blocks (the unit's first P.V overwrites O);
-  * each rescale O holding exactly the unit's earlier blocks (the softmax rescales right
-    after S of its block is complete, with no wait of its own: the issuer sends Q K^T of a
-    block only after the previous block's P.V, and the pipe runs them in that order);
+  * each rescale O holding exactly the unit's earlier blocks (the softmax waits for the
+    previous block's P.V; the one before has completed, since this block's Q K^T went to
+    the pipe after it);
   * each epilogue O holding every block of the unit;
   * the next unit's first P.V only after every warp has read O in the epilogue.
 
 mbarrier semantics modelled: a phase completes when its expected arrival count is
 reached; a parity test for parity P succeeds when the current phase's parity differs from
-P (a barrier two phases behind the awaited one looks complete). The issuing thread's
-products run in its issue order, and a commit arrives once the products issued before it
-are done. TMA loads land at a random later time and write their stage when they land.
+P (a barrier two phases behind the awaited one looks complete). Each issuing thread's
+products run in its own issue order, the two threads' products interleave arbitrarily,
+and a commit arrives once the products its thread issued before it are done. TMA loads
+land at a random later time and write their stage when they land.
 
 Deliberately broken variants must be caught, which shows the checker can see the
-hazards: a stage released when the first cursor passes it, a Q K^T issued before the
-previous P.V (overwriting P), a P.V issued before its softmax released P, Q released at
-the unit's first product, and an epilogue that does not wait for the last P.V.
+hazards: a stage reloaded after one issuer's release instead of both, a Q K^T into an S buffer whose
+P.V is still pending (overwriting P), a P.V issued before its softmax released P, Q
+released at the unit's first product, a rescale without its wait, and an epilogue that
+does not wait for the last P.V.
 """
 import random
 
@@ -37,7 +39,7 @@ import pytest
 import _cases as C
 from oracle import bsa_oracle as O
 
-NS = 2          # ring stages (two key tiles each)
+NS = 4          # ring stages (one key tile each)
 WARPS = 4       # softmax warps per query block
 
 
@@ -85,34 +87,32 @@ def cost(unit):
     return sum(e[0] or e[1] for e in ent) + sum(e[2] or e[3] for e in ent)
 
 
-def block_use(ent, c, x):
-    u = 0
-    for h in range(2):
-        i = 2 * c + h
-        if i < len(ent) and (ent[i][2 * x] or ent[i][2 * x + 1]):
-            u |= 1 << h
-    return u
+def used(ent, c, x):
+    return ent[c][2 * x] or ent[c][2 * x + 1]
 
 
 def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=False,
-                 no_pfull_wait=False, no_epilogue_wait=False):
+                 no_pfull_wait=False, no_epilogue_wait=False, no_rescale_wait=False):
     """True if every unit finishes; False on deadlock; raises Stale on a wrong read."""
     rng = random.Random(seed)
     nunits = len(units)
     # ------------------------------------------------------------------ barriers
-    kfull, kempty = [Bar(1) for _ in range(NS)], [Bar(1) for _ in range(NS)]
-    vfull, vempty = [Bar(1) for _ in range(NS)], [Bar(1) for _ in range(NS)]
+    releases = 1 if early_release else 2        # stage releases before a reload: one per issuer
+    kfull, kempty = [Bar(1) for _ in range(NS)], [Bar(releases) for _ in range(NS)]
+    vfull, vempty = [Bar(1) for _ in range(NS)], [Bar(releases) for _ in range(NS)]
     qfull, qempty = [Bar(1), Bar(1)], [Bar(1), Bar(1)]
-    sfull, pfull, odone = [Bar(1), Bar(1)], [Bar(WARPS), Bar(WARPS)], [Bar(1), Bar(1)]
+    sfull = [[Bar(1), Bar(1)] for _ in range(2)]            # [query block][S buffer]
+    pfull = [[Bar(WARPS), Bar(WARPS)] for _ in range(2)]
+    odone = [[Bar(1), Bar(1)] for _ in range(2)]
     lfull, lempty = [Bar(1), Bar(1)], [Bar(2 + 2 + 2 * WARPS), Bar(2 + 2 + 2 * WARPS)]
     # ------------------------------------------------------------------ state
     lists = [None, None]                      # key-stream buffers: unit index or 'end'
     kdata, vdata, qdata = [None] * NS, [None] * NS, [None, None]
-    sbuf = [[None] * WARPS for _ in range(2)]  # per warp's rows: ('S'|'P', unit, block)
+    sbuf = [[[None] * WARPS for _ in range(2)] for _ in range(2)]  # [x][buffer][warp]: ('S'|'P', unit, block)
     obuf = [[None, 0], [None, 0]]             # (unit, blocks absorbed)
     epi_done = [[-1] * WARPS for _ in range(2)]   # last unit whose epilogue each warp finished
     inflight = []                             # TMA loads: (barrier, apply)
-    pipe = []                                 # products / commits in issue order
+    pipes = [[], []]                          # per issuer: products / commits in issue order
 
     bld = {"it": 0, "next": 0, "done": False}
     # two producers: K (Q of each query block, then the K ring) and V (the V ring)
@@ -120,22 +120,21 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
               "done": False} for kind in ("k", "v")]
 
     def new_cursor():
-        return {"it": 0, "have": False, "done": False, "unit": None, "kc": 0, "vc": 0, "pend": -1,
+        return {"it": 0, "have": False, "done": False, "unit": None, "kc": 0, "vc": 0,
                 "hasq": False, "qready": False, "qrel": False, "first": True, "gbase": 0, "qn": 0,
-                "pn": 0, "nb": 0}
+                "qk": 0, "pv": 0, "ent": [-1, -1], "nb": 0}
     cur = [new_cursor(), new_cursor()]
-    kpass, vpass = [0, 0], [0, 0]
     sm = [[{"it": 0, "state": "list", "unit": None, "c": 0, "sidx": 0, "nused": 0, "blocks": 0,
             "done": False} for _ in range(WARPS)] for _ in range(2)]
 
-    def enqueue(kind, **kw):
-        pipe.append(dict(kind=kind, **kw))
+    def enqueue(x, kind, **kw):
+        pipes[x].append(dict(kind=kind, x=x, **kw))
 
     def unit_of(buf):
         return lists[buf]
 
     def nblocks(ui):
-        return (len(units[ui][1]) + 1) // 2
+        return len(units[ui][1])
 
     # ------------------------------------------------------------------ agents
     def builder_actions():
@@ -212,10 +211,13 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
             p["c"] += 1
         return [act]
 
-    def release(passes, empty, x, gi):
-        passes[x] = gi + 1
-        if early_release or passes[x ^ 1] >= gi + 1:
-            enqueue("commit", bar=empty[gi % NS])
+    def release(empty, x, gi, issued):
+        # after a product on the stage, a commit (arrives once the product is done);
+        # a tile passed without a product is released at once
+        if issued:
+            enqueue(x, "commit", bar=empty[gi % NS])
+        else:
+            empty[gi % NS].arrive()
 
     def cursor_actions(x):
         cu = cur[x]
@@ -230,64 +232,67 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
                     if ui == "end":
                         cu["done"] = True
                         return
-                    cu.update(have=True, unit=ui, kc=0, vc=0, pend=-1, hasq=units[ui][0][2 * x] >= 0,
+                    cu.update(have=True, unit=ui, kc=0, vc=0, hasq=units[ui][0][2 * x] >= 0,
                               qready=False, qrel=False, first=True, nb=nblocks(ui))
                 acts.append(act)
             return acts
         ui = cu["unit"]
         qs, ent = units[ui]
         nb = cu["nb"]
-        if cu["kc"] < nb:
-            c = cu["kc"]
-            u = block_use(ent, c, x) if cu["hasq"] else 0
-            gi = cu["gbase"] + c
-            s, fph = gi % NS, (gi // NS) & 1
-            qok = cu["qready"] or qfull[x].test(cu["qn"] & 1)
-            if u == 0:
-                ok = kfull[s].test(fph)
-            else:
-                ok = (cu["pend"] < 0 or qk_before_pv) and qok and kfull[s].test(fph)
-            if ok:
-                def act(u=u, c=c, gi=gi, s=s, qok=qok):
-                    if u:
-                        cu["qready"] = True
-                        enqueue("qk", x=x, unit=ui, block=c, stage=s)
-                        enqueue("commit", bar=sfull[x])
-                        cu["pend"] = c
-                        if early_q and not cu["qrel"]:
-                            enqueue("commit", bar=qempty[x])
-                            cu["qrel"] = True
-                    release(kpass, kempty, x, gi)
-                    cu["kc"] += 1
-                    if cu["kc"] == nb and cu["hasq"] and cu["qready"] and not cu["qrel"]:
-                        enqueue("commit", bar=qempty[x])
-                        cu["qrel"] = True
-                acts.append(act)
         if cu["vc"] < cu["kc"]:
             c = cu["vc"]
             gi = cu["gbase"] + c
             s, fph = gi % NS, (gi // NS) & 1
-            if c == cu["pend"]:
-                ok = (no_pfull_wait or pfull[x].test(cu["pn"] & 1)) and vfull[s].test(fph)
+            pending = cu["pv"] != cu["qk"] and c == cu["ent"][cu["pv"] & 1]
+            if pending:
+                b = cu["pv"] & 1
+                ok = (no_pfull_wait or pfull[x][b].test((cu["pv"] >> 1) & 1)) and vfull[s].test(fph)
             else:
                 ok = vfull[s].test(fph)
             if ok:
-                def act(c=c, gi=gi, s=s):
-                    if c == cu["pend"]:
-                        enqueue("pv", x=x, unit=ui, block=c, stage=s, first=cu["first"],
-                                ordinal=cu["pn"])
-                        enqueue("commit", bar=odone[x])
+                def act(c=c, gi=gi, s=s, pending=pending):
+                    if pending:
+                        b = cu["pv"] & 1
+                        enqueue(x, "pv", unit=ui, block=c, stage=s, buf=b, first=cu["first"])
+                        enqueue(x, "commit", bar=odone[x][b])
                         cu["first"] = False
-                        cu["pn"] += 1
-                        cu["pend"] = -1
-                    release(vpass, vempty, x, gi)
+                        cu["pv"] += 1
+                    release(vempty, x, gi, pending)
                     cu["vc"] += 1
+                acts.append(act)
+        if cu["kc"] < nb:
+            c = cu["kc"]
+            u = used(ent, c, x) if cu["hasq"] else False
+            gi = cu["gbase"] + c
+            s, fph = gi % NS, (gi // NS) & 1
+            qok = cu["qready"] or qfull[x].test(cu["qn"] & 1)
+            if not u:
+                ok = kfull[s].test(fph)
+            else:
+                ok = (cu["qk"] - cu["pv"] < (3 if qk_before_pv else 2)) and qok and kfull[s].test(fph)
+            if ok:
+                def act(u=u, c=c, gi=gi, s=s):
+                    if u:
+                        cu["qready"] = True
+                        b = cu["qk"] & 1
+                        enqueue(x, "qk", unit=ui, block=c, stage=s, buf=b)
+                        enqueue(x, "commit", bar=sfull[x][b])
+                        cu["ent"][b] = c
+                        cu["qk"] += 1
+                        if early_q and not cu["qrel"]:
+                            enqueue(x, "commit", bar=qempty[x])
+                            cu["qrel"] = True
+                    release(kempty, x, gi, u)
+                    cu["kc"] += 1
+                    if cu["kc"] == nb and cu["hasq"] and cu["qready"] and not cu["qrel"]:
+                        enqueue(x, "commit", bar=qempty[x])
+                        cu["qrel"] = True
                 acts.append(act)
         if cu["kc"] == nb and cu["vc"] == nb:
             if not cu["hasq"] or cu["qrel"] or cu["qready"] or qfull[x].test(cu["qn"] & 1):
                 def act():
                     if cu["hasq"] and not cu["qrel"]:
-                        enqueue("commit", bar=qempty[x])
+                        enqueue(x, "commit", bar=qempty[x])
                         cu["qrel"] = True
                     if cu["hasq"]:
                         cu["qn"] += 1
@@ -298,7 +303,7 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
                 acts.append(act)
         return acts
 
-    def pipe_actions():
+    def pipe_actions(pipe):
         if not pipe:
             return []
 
@@ -313,17 +318,19 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
                     raise Stale(f"QK of unit {ui} reads Q of {qdata[x]}")
                 if kdata[s] != (ui, c):
                     raise Stale(f"QK of {(ui, c)} reads K {kdata[s]}")
+                b = op["buf"]
                 for w in range(WARPS):
-                    if sbuf[x][w] is not None and sbuf[x][w][0] == "S":
-                        raise Stale(f"S of {sbuf[x][w][1:]} overwritten before its softmax read it")
-                    sbuf[x][w] = ("S", ui, c)
+                    if sbuf[x][b][w] is not None and sbuf[x][b][w][0] == "S":
+                        raise Stale(f"S of {sbuf[x][b][w][1:]} overwritten before its softmax read it")
+                    sbuf[x][b][w] = ("S", ui, c)
             else:
                 x, ui, c, s = op["x"], op["unit"], op["block"], op["stage"]
                 if vdata[s] != (ui, c):
                     raise Stale(f"PV of {(ui, c)} reads V {vdata[s]}")
+                b = op["buf"]
                 for w in range(WARPS):
-                    if sbuf[x][w] != ("P", ui, c):
-                        raise Stale(f"PV of {(ui, c)} reads {sbuf[x][w]} (warp {w})")
+                    if sbuf[x][b][w] != ("P", ui, c):
+                        raise Stale(f"PV of {(ui, c)} reads {sbuf[x][b][w]} (warp {w})")
                 if op["first"]:
                     if any(epi_done[x][w] < (obuf[x][0] if obuf[x][0] is not None else -1)
                            for w in range(WARPS)):
@@ -355,23 +362,28 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
         qs, ent = units[ui]
         nb = nblocks(ui)
         if st["state"] == "blocks":
-            while st["c"] < nb and (qs[2 * x] < 0 or block_use(ent, st["c"], x) == 0):
+            while st["c"] < nb and (qs[2 * x] < 0 or not used(ent, st["c"], x)):
                 st["c"] += 1
             if st["c"] == nb:
                 def act():
                     lempty[st["it"] & 1].arrive()
                     st["state"] = "epi"
                 return [act]
-            if not sfull[x].test(st["sidx"] & 1):
+            b = st["sidx"] & 1
+            if not sfull[x][b].test((st["sidx"] >> 1) & 1):
                 return []
 
-            def act():
+            def act(b=b):
                 c = st["c"]
-                if sbuf[x][w] != ("S", ui, c):
-                    raise Stale(f"softmax {(ui, c)} reads {sbuf[x][w]}")
+                if sbuf[x][b][w] != ("S", ui, c):
+                    raise Stale(f"softmax {(ui, c)} reads {sbuf[x][b][w]}")
                 st["state"] = "resc" if (st["nused"] > 0 and rng.random() < 0.3) else "release"
             return [act]
         if st["state"] == "resc":
+            pb = (st["sidx"] - 1) & 1
+            if not no_rescale_wait and not odone[x][pb].test(((st["sidx"] - 1) >> 1) & 1):
+                return []
+
             def act():
                 if obuf[x] != [ui, st["nused"]]:
                     raise Stale(f"rescale in {(ui, st['c'])} sees O {obuf[x]}")
@@ -379,15 +391,17 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
             return [act]
         if st["state"] == "release":
             def act():
-                sbuf[x][w] = ("P", ui, st["c"])
-                pfull[x].arrive()
+                b = st["sidx"] & 1
+                sbuf[x][b][w] = ("P", ui, st["c"])
+                pfull[x][b].arrive()
                 st["sidx"] += 1
                 st["nused"] += 1
                 st["c"] += 1
                 st["state"] = "blocks"
             return [act]
         # epilogue
-        if st["nused"] > 0 and not no_epilogue_wait and not odone[x].test((st["sidx"] - 1) & 1):
+        pb = (st["sidx"] - 1) & 1
+        if st["nused"] > 0 and not no_epilogue_wait and not odone[x][pb].test(((st["sidx"] - 1) >> 1) & 1):
             return []
 
         def act():
@@ -402,7 +416,7 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
     unit_pv = {}
 
     def fix_ordinals():
-        for op in pipe:
+        for op in pipes[0] + pipes[1]:
             if op["kind"] == "pv" and "ordinal_in_unit" not in op:
                 key = (op["x"], op["unit"])
                 op["ordinal_in_unit"] = unit_pv.get(key, 0)
@@ -411,7 +425,7 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
     for _ in range(2_000_000):
         fix_ordinals()
         acts = builder_actions() + producer_actions(prods[0]) + producer_actions(prods[1]) + \
-            cursor_actions(0) + cursor_actions(1) + pipe_actions()
+            cursor_actions(0) + cursor_actions(1) + pipe_actions(pipes[0]) + pipe_actions(pipes[1])
         for x in range(2):
             for w in range(WARPS):
                 acts += softmax_actions(x, w)
@@ -424,7 +438,7 @@ def run_protocol(units, seed, early_release=False, qk_before_pv=False, early_q=F
             acts.append(land)
         if not acts:
             done = bld["done"] and all(p["done"] for p in prods) and all(c["done"] for c in cur) and \
-                all(s["done"] for xs in sm for s in xs) and not pipe and not inflight
+                all(s["done"] for xs in sm for s in xs) and not pipes[0] and not pipes[1] and not inflight
             return done
         rng.choice(acts)()
     raise AssertionError("model did not terminate")
@@ -509,3 +523,7 @@ def test_model_catches_pv_before_p():
 
 def test_model_catches_epilogue_without_wait():
     assert _catches(no_epilogue_wait=True)
+
+
+def test_model_catches_rescale_without_wait():
+    assert _catches(no_rescale_wait=True)
