@@ -76,7 +76,7 @@ constexpr long long kWaitLimit = 4000000000LL;     // SM cycles, about 2 s
 constexpr int kTmemCols = 512;
 constexpr int kUnitInts = 8;                       // {bh, q0, q1, q2, q3, cost, 0, 0}
 constexpr float kRescaleLog2 = 8.0f;               // O is rescaled only past 2^8 of growth
-constexpr unsigned kIssuerBackoffNs = 32;          // issuer pause after a pass with nothing to issue
+constexpr unsigned kIssuerSleepNs = 2000;          // longest suspension of an idle issuer
 
 template <int D>
 struct Cfg {
@@ -709,9 +709,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           report_error(a.err, BSA_KERR_WAIT_TIMEOUT);
           ok = false;
         } else {
-          // Nothing to issue: yield the sub-partition's issue slots to the two softmax
-          // warps that share it, instead of polling the barriers back to back.
-          __nanosleep(kIssuerBackoffNs);
+          // Nothing to issue: suspend until the barrier this issuer most likely needs next
+          // completes (at most kIssuerSleepNs), so that the two softmax warps sharing the
+          // sub-partition get its issue slots. Then every position is tested again.
+          uint32_t wb, wp;
+          if (!cu.have) {
+            wb = bar.lfull(cu.it & 1);
+            wp = (uint32_t)(cu.it >> 1) & 1u;
+          } else if (cu.vc < cu.kc) {
+            const uint32_t gi = cu.gbase + (uint32_t)cu.vc;
+            wb = bar.vfull((int)(gi % kNS));
+            wp = (gi / kNS) & 1u;
+            if (cu.pv != cu.qk && cu.vc == ((cu.pv & 1) ? cu.ent1 : cu.ent0) &&
+                !ptx::mbar_test_wait(bar.pfull(x, (int)(cu.pv & 1)), (cu.pv >> 1) & 1)) {
+              wb = bar.pfull(x, (int)(cu.pv & 1));
+              wp = (cu.pv >> 1) & 1;
+            }
+          } else if (cu.kc < cu.L && (!cu.hasq || cu.qready || ((cu.flags[cu.kc] >> (2 * x)) & 3u) == 0u)) {
+            const uint32_t gi = cu.gbase + (uint32_t)cu.kc;
+            wb = bar.kfull((int)(gi % kNS));
+            wp = (gi / kNS) & 1u;
+          } else {
+            wb = bar.qfull(x);
+            wp = (uint32_t)cu.qn & 1u;
+          }
+          ptx::mbar_try_wait_ns(wb, wp, kIssuerSleepNs);
         }
       }
       // Never free TMEM under a running MMA: wait until everything issued has completed.

@@ -510,151 +510,267 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
   if (q == 0 && lane == 0) a.kv_count[rowid] = count;
 }
 
-// ---- selection by radix (fixed top-k and budget modes): one row per warp, kRsWarps rows
-// per block. The row's order keys live in shared memory (0 for window tiles and for slots
-// past NKT). The key of the extra-th best candidate is found four bits at a time from the
-// top: each pass counts, in per-lane private shared-memory bins (no atomics), the keys
-// that carry the digits found so far, sums the 16 bins across lanes and keeps the largest
-// digit under which at least the still-needed number of keys lie. A pass that finds a
-// digit holding exactly that number ends the search (every key from that prefix up is
-// taken); otherwise the search ends at the exact key, and of the keys equal to it the
-// first in tile order are taken. The result is "highest score, ties to the lower index",
-// as the argmax and threshold search of select_kernel give it.
-constexpr int kRsWarps = 8;
-constexpr int kRsBinStride = 17;                 // per-lane bins, padded so lanes hit distinct banks
+// ---- selection by radix (fixed top-k and budget modes): one block of 128 threads per
+// row at a time, each block taking rows of one (b, h) in turn. A thread holds its KPT keys
+// of the row in registers (key j at thread j mod 128, slot j / 128); 0 marks window tiles
+// and slots past NKT. The key of the extra-th best candidate is found by narrowing a key
+// range, starting from the candidates' [min, max]: each pass splits the range into at most
+// 256 buckets of 2^shift keys (the bucket is (key - lo) >> shift, so the split follows the
+// keys' spread, not fixed digit boundaries, and lanes seldom collide on a counter), counts
+// them in per-warp shared histograms, and one warp finds the largest bucket at or above
+// which at least the still-needed number of keys lie. A bucket holding exactly that number
+// ends the search (every key from its low end up is taken); otherwise the range shrinks to
+// that bucket, by at least eight bits of width per pass, down to one key value, of which
+// the first in tile order are taken. The result is "highest score, ties to the lower
+// index", as the argmax and threshold search of select_kernel give it.
+constexpr int kRsThreads = 128;
+constexpr int kRsBlocksPerSm = 8;
 
-template <int MODE, bool TOK>
-__global__ void __launch_bounds__(kRsWarps * 32) select_radix_kernel(SelArgs a, const float* __restrict__ S,
-                                                                     int NKTP) {
+// Sum over the block's four warps; `red` holds four ints. Every thread gets the sum.
+__device__ __forceinline__ int rs_block_sum(int v, int* red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  const int s = red[0] + red[1] + red[2] + red[3];
+  __syncthreads();
+  return s;
+}
+
+template <int MODE, bool TOK, int KPT>
+__global__ void __launch_bounds__(kRsThreads, kRsBlocksPerSm) select_radix_kernel(SelArgs a, const float* __restrict__ S,
+                                                                  int NKTP) {
   extern __shared__ __align__(16) uint32_t sm_u32[];
   const Geom& g = a.g;
   const int NKT = g.NT, NQT = g.NT;
-  const int NKW = g.NW * 32;                                   // key slots per row
   const int b = blockIdx.z, h = blockIdx.y;
   const long long bh = (long long)b * g.H + h;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint32_t* coord = sm_u32;                                    // NKW tile coordinates
-  uint32_t* keys = sm_u32 + NKW * (1 + warp);                  // this warp's row
-  uint32_t* bins = sm_u32 + NKW * (1 + kRsWarps) + warp * 32 * kRsBinStride + lane * kRsBinStride;
+  float* srows = reinterpret_cast<float*>(sm_u32);            // two score rows (NKTP each)
+  uint32_t* coord = sm_u32 + 2 * NKTP;                         // NKT tile coordinates
+  uint32_t* hist = coord + ((NKT + 3) & ~3);                   // 4 warps x 256 bucket counts
+  uint32_t* eqw = hist + 1024;                                 // per mask word: keys equal to thr
+  int* red = reinterpret_cast<int*>(eqw + ((g.NW + 3) & ~3));  // sums, broadcast values, key range
 
-  for (int j = tid; j < NKT; j += kRsWarps * 32) {
+  for (int j = tid; j < NKT; j += kRsThreads) {
     int tt, ty, tx;
     tile_xyz(g, j, tt, ty, tx);
     coord[j] = pack_coord(tt, ty, tx);
   }
   __syncthreads();
 
-  const int i = blockIdx.x * kRsWarps + warp;
-  if (i >= NQT) return;
-  const long long rowid = bh * NQT + i;
-  const float* srow = S + rowid * NKTP;
-  uint32_t* mrow = a.mask + rowid * g.NW;
-  if (a.dense[(long long)b * NQT + i]) {
-    for (int w = lane; w < g.NW; w += 32) {
-      const int rem = NKT - 32 * w;
-      mrow[w] = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+  // The next row's scores are copied into shared memory (cp.async, 16 bytes per copy)
+  // while this row is selected; one commit group per row, empty for dense rows.
+  auto fetch_row = [&](int ii, int buf) {
+    if (ii < NQT && !a.dense[(long long)b * NQT + ii]) {
+      const float* src = S + (bh * NQT + ii) * NKTP;
+      const uint32_t dst = (uint32_t)__cvta_generic_to_shared(srows + buf * NKTP);
+      for (int c = tid; c < NKTP / 4; c += kRsThreads)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16u * c), "l"(src + 4 * c) : "memory");
     }
-    if (lane == 0) a.kv_count[rowid] = NKT;
-    return;
-  }
-  const uint32_t ci = coord[i];
-  int kind = a.window_kind, rad = a.radius, extra;
-  if (MODE == kSelectFixed) {
-    extra = a.topk;
-  } else {
-    const int2 pl = a.plan[rowid];
-    kind = 1;
-    rad = pl.x;
-    extra = pl.y;
-  }
-  int ncand = 0;
-  for (int w = 0; w < g.NW; ++w) {
-    const int j = 32 * w + lane;
-    const bool cand = j < NKT && !sel_in_window<TOK>(ci, coord[j], kind, rad);
-    keys[j] = cand ? order_key(srow[j]) : 0u;
-    ncand += __popc(__ballot_sync(0xffffffffu, cand));
-  }
-  extra = max(0, min(extra, ncand));
-
-  // keys >= t_ge are taken; of the keys equal to thr, the first need_eq in tile order
-  uint32_t t_ge, thr = 0xffffffffu;
-  int need_eq = 0;
-  if (extra == 0) {
-    t_ge = 0xffffffffu;                                         // no score maps to this key
-  } else if (extra == ncand) {
-    t_ge = 1u;                                                  // every candidate (keys >= 2)
-  } else {
-    uint32_t prefix = 0u;
-    int remaining = extra;
-    bool done = false;
-    for (int shift = 28; shift >= 0 && !done; shift -= 4) {
-      const uint32_t hi = shift == 28 ? 0u : (0xffffffffu << (shift + 4));
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  fetch_row(blockIdx.x, 0);
+  int buf = 0;
+  for (int i = blockIdx.x; i < NQT; i += gridDim.x, buf ^= 1) {
+    // Buffer buf ^ 1 was last read in the previous row, before its closing block sums.
+    fetch_row(i + gridDim.x, buf ^ 1);
+    asm volatile("cp.async.wait_group 1;" ::: "memory");      // this row's copy has landed
+    __syncthreads();
+    const long long rowid = bh * NQT + i;
+    const float* srow = srows + buf * NKTP;
+    uint32_t* mrow = a.mask + rowid * g.NW;
+    if (a.dense[(long long)b * NQT + i]) {                     // the same branch for the whole block
+      for (int w = tid; w < g.NW; w += kRsThreads) {
+        const int rem = NKT - 32 * w;
+        mrow[w] = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+      }
+      if (tid == 0) a.kv_count[rowid] = NKT;
+      continue;
+    }
+    const uint32_t ci = coord[i];
+    int kind = a.window_kind, rad = a.radius, extra;
+    if (MODE == kSelectFixed) {
+      extra = a.topk;
+    } else {
+      const int2 pl = a.plan[rowid];
+      kind = 1;
+      rad = pl.x;
+      extra = pl.y;
+    }
+    uint32_t key[KPT];
+    int ncand = 0;
 #pragma unroll
-      for (int d = 0; d < 16; ++d) bins[d] = 0u;
-      for (int w = 0; w < g.NW; ++w) {
-        const uint32_t k = keys[32 * w + lane];
-        if (k != 0u && (k & hi) == prefix) ++bins[(k >> shift) & 15u];
-      }
-      __syncwarp();
-      int tot = 0;
-      if (lane < 16) {
-        const uint32_t* col = bins - lane * kRsBinStride + lane;   // bin `lane` of every lane
-        for (int l = 0; l < 32; ++l) tot += (int)col[l * kRsBinStride];
-      }
-      // suffix sums over digits 15..0 (digit d at lane d)
-      int suf = tot;
-#pragma unroll
-      for (int off = 1; off < 16; off <<= 1) {
-        const int v = __shfl_down_sync(0xffffffffu, suf, off);
-        if (lane + off < 16) suf += v;
-      }
-      const uint32_t ok = __ballot_sync(0xffffffffu, lane < 16 && suf >= remaining);
-      const int dsel = 31 - __clz(ok);                          // largest digit with enough keys at or above it
-      const int above = __shfl_sync(0xffffffffu, suf, min(dsel + 1, 31)) * (dsel < 15 ? 1 : 0);
-      const int at = __shfl_sync(0xffffffffu, tot, dsel);
-      remaining -= above;
-      prefix |= (uint32_t)dsel << shift;
-      if (at == remaining) {                                    // the whole prefix band is taken
-        t_ge = prefix;
-        done = true;
-      }
-      __syncwarp();
+    for (int m = 0; m < KPT; ++m) {
+      const int j = tid + kRsThreads * m;
+      const bool cand = j < NKT && !sel_in_window<TOK>(ci, coord[j], kind, rad);
+      key[m] = cand ? order_key(srow[j]) : 0u;
+      ncand += cand ? 1 : 0;
     }
-    if (!done) {
-      thr = prefix;                                             // the exact key of the boundary
-      t_ge = prefix + 1u;
-      need_eq = remaining;
-    }
-    if (t_ge == 0u) t_ge = 1u;                                  // a band from key 0: every candidate
-  }
+    ncand = rs_block_sum(ncand, red);
+    extra = max(0, min(extra, ncand));
 
-  int eq_before = 0, count = 0;
-  for (int w = 0; w < g.NW; ++w) {
-    const int j = 32 * w + lane;
-    const uint32_t k = keys[j];
-    const bool inrow = j < NKT;
-    bool sel = inrow && (k == 0u || k >= t_ge);
-    const bool eq = inrow && k != 0u && k == thr && need_eq > 0;
-    const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
-    const int rank = eq_before + __popc(eqb & ((1u << lane) - 1u));
-    sel = sel || (eq && rank < need_eq);
-    eq_before += __popc(eqb);
-    const uint32_t bits = __ballot_sync(0xffffffffu, sel);
-    if (lane == 0) mrow[w] = bits;
-    count += __popc(bits);
+    // keys >= t_ge are taken; of the keys equal to thr, the first need_eq in tile order
+    uint32_t t_ge, thr = 0xffffffffu;
+    int need_eq = 0;
+    if (extra == 0) {
+      t_ge = 0xffffffffu;                                       // no score maps to this key
+    } else if (extra == ncand) {
+      t_ge = 1u;                                                // every candidate
+    } else {
+      // key range [lo, hi] of the candidates
+      uint32_t lo = 0xffffffffu, hi = 0u;
+#pragma unroll
+      for (int m = 0; m < KPT; ++m) {
+        if (key[m] != 0u) {
+          lo = min(lo, key[m]);
+          hi = max(hi, key[m]);
+        }
+      }
+      lo = __reduce_min_sync(0xffffffffu, lo);
+      hi = __reduce_max_sync(0xffffffffu, hi);
+      if (lane == 0) {
+        red[8 + warp] = (int)lo;
+        red[12 + warp] = (int)hi;
+      }
+      __syncthreads();
+      lo = min(min((uint32_t)red[8], (uint32_t)red[9]), min((uint32_t)red[10], (uint32_t)red[11]));
+      hi = max(max((uint32_t)red[12], (uint32_t)red[13]), max((uint32_t)red[14], (uint32_t)red[15]));
+      int remaining = extra;
+      bool done = false;
+      while (!done) {
+        // buckets of 2^shift keys over [lo, hi]: at most 256
+        const uint32_t span = hi - lo;
+        const int shift = span < 256u ? 0 : (32 - __clz(span)) - 8;
+        uint32_t* wh = hist + warp * 256;                       // this warp's histogram
+#pragma unroll
+        for (int e = 0; e < 8; ++e) hist[tid + kRsThreads * e] = 0u;
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < KPT; ++m) {
+          const uint32_t k = key[m];
+          if (k >= lo && k <= hi) atomicAdd(&wh[(k - lo) >> shift], 1u);
+        }
+        __syncthreads();
+        if (warp == 0) {
+          // lane l holds buckets 8l .. 8l+7; find the largest bucket at or above which at
+          // least `remaining` keys lie
+          uint32_t c[8];
+          int lt = 0;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int d = 8 * lane + e;
+            c[e] = hist[d] + hist[256 + d] + hist[512 + d] + hist[768 + d];
+            lt += (int)c[e];
+          }
+          int incl = lt;                                        // keys in lanes >= this one
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_down_sync(0xffffffffu, incl, off);
+            if (lane + off < 32) incl += v;
+          }
+          int sfx = incl - lt, best = -1, best_above = 0, best_at = 0;
+#pragma unroll
+          for (int e = 7; e >= 0; --e) {
+            const int above = sfx;
+            sfx += (int)c[e];
+            if (best < 0 && sfx >= remaining) {
+              best = 8 * lane + e;
+              best_above = above;
+              best_at = (int)c[e];
+            }
+          }
+          const uint32_t okl = __ballot_sync(0xffffffffu, best >= 0);
+          if (lane == 31 - __clz(okl)) {                       // the lane of the largest such bucket
+            red[4] = best;
+            red[5] = best_above;
+            red[6] = best_at;
+          }
+        }
+        __syncthreads();
+        const int dsel = red[4], above = red[5], at = red[6];
+        remaining -= above;
+        const uint32_t blo = lo + ((uint32_t)dsel << shift);
+        const uint32_t bhi = (uint32_t)min((unsigned long long)hi, (unsigned long long)blo + (1ull << shift) - 1ull);
+        if (at == remaining) {                                  // the whole bucket is taken
+          t_ge = blo;
+          done = true;
+        } else if (shift == 0) {                                // one key value: ties
+          thr = blo;
+          t_ge = blo + 1u;
+          need_eq = remaining;
+          done = true;
+        }
+        lo = blo;
+        hi = bhi;
+      }
+      if (t_ge == 0u) t_ge = 1u;                                // a band from key 0: every candidate
+    }
+
+    if (need_eq > 0) {                                          // ties at the boundary key
+#pragma unroll
+      for (int m = 0; m < KPT; ++m) {
+        const int w = warp + 4 * m;
+        const int j = tid + kRsThreads * m;
+        const uint32_t eqb = __ballot_sync(0xffffffffu, j < NKT && key[m] != 0u && key[m] == thr);
+        if (lane == 0 && w < g.NW) eqw[w] = eqb;
+      }
+      __syncthreads();
+    }
+    int count = 0;
+#pragma unroll
+    for (int m = 0; m < KPT; ++m) {
+      const int w = warp + 4 * m;                              // mask word of this slot (warp-uniform)
+      if (w < g.NW) {
+        const int j = tid + kRsThreads * m;
+        const uint32_t k = key[m];
+        const bool inrow = j < NKT;
+        bool sel = inrow && (k == 0u || k >= t_ge);
+        if (need_eq > 0 && inrow && k != 0u && k == thr) {
+          int rank = __popc(eqw[w] & ((1u << lane) - 1u));
+          for (int ww = 0; ww < w; ++ww) rank += __popc(eqw[ww]);
+          sel = rank < need_eq;
+        }
+        const uint32_t bits = __ballot_sync(0xffffffffu, sel);
+        if (lane == 0) {
+          mrow[w] = bits;
+          count += __popc(bits);
+        }
+      }
+    }
+    count = rs_block_sum(count, red);
+    if (tid == 0) a.kv_count[rowid] = count;
   }
-  if (lane == 0) a.kv_count[rowid] = count;
+  asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
+template <int MODE, bool TOK, int KPT>
+cudaError_t launch_select_radix_kpt(const Geom& g, const SelArgs& a, const float* S, int NKTP, cudaStream_t s) {
+  const size_t smem = sizeof(uint32_t) * (2 * (size_t)NKTP + (size_t)((g.NT + 3) & ~3) + 1024 +
+                                          (size_t)((g.NW + 3) & ~3) + 16);
+  cudaError_t e = cudaFuncSetAttribute(select_radix_kernel<MODE, TOK, KPT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148, per_sm = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_radix_kernel<MODE, TOK, KPT>, kRsThreads, smem);
+  if (e != cudaSuccess) return e;
+  // one wave: every block resident at once, each (b, h) with the same number of blocks
+  const int per_bh = max(1, min(g.NT, (sms * max(per_sm, 1)) / (g.B * g.H)));
+  const dim3 grid(per_bh, g.H, g.B);
+  select_radix_kernel<MODE, TOK, KPT><<<grid, kRsThreads, smem, s>>>(a, S, NKTP);
+  return cudaGetLastError();
+}
+
+// KPT = key slots per thread: the row's NW * 32 slots over 128 threads, rounded up to 8.
 template <int MODE, bool TOK>
 cudaError_t launch_select_radix(const Geom& g, const SelArgs& a, const float* S, int NKTP, cudaStream_t s) {
-  const size_t smem = sizeof(uint32_t) * ((size_t)g.NW * 32 * (1 + kRsWarps) + (size_t)kRsWarps * 32 * kRsBinStride);
-  cudaError_t e = cudaFuncSetAttribute(select_radix_kernel<MODE, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e != cudaSuccess) return e;
-  const dim3 grid(ceil_div(g.NT, kRsWarps), g.H, g.B);
-  select_radix_kernel<MODE, TOK><<<grid, kRsWarps * 32, smem, s>>>(a, S, NKTP);
-  return cudaGetLastError();
+  const int kpt = ceil_div(g.NW * 32, kRsThreads);
+  if (kpt <= 8) return launch_select_radix_kpt<MODE, TOK, 8>(g, a, S, NKTP, s);
+  if (kpt <= 16) return launch_select_radix_kpt<MODE, TOK, 16>(g, a, S, NKTP, s);
+  if (kpt <= 24) return launch_select_radix_kpt<MODE, TOK, 24>(g, a, S, NKTP, s);
+  return launch_select_radix_kpt<MODE, TOK, 32>(g, a, S, NKTP, s);
 }
 
 template <int MODE, int KW, int WPR, bool TOK>
