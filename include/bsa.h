@@ -233,8 +233,11 @@ size_t bsa_route_flags_offset(const bsa_geom* g);
  * Every call uses the same array and leaves its contents there: each call zeroes the
  * array's header on its stream before use, and calls that overlap on the GPU (other
  * streams, other host threads, same device) race on the array and must not be issued.
- * The first call on each device looks up the array's device address (with that device
- * current); make that first call before any stream capture. */
+ * Every call made outside stream capture looks the array's device address up again (with
+ * the call's device current), so the address stays valid after a device reset, which
+ * reloads the library's module. A call captured into a CUDA graph uses the address looked
+ * up by the last uncaptured call on that device (make one before the first capture), and
+ * the graph holds that address: re-capture it after a device reset. */
 int bsa_sparse_attn_fwd_fixed_scratch(const bsa_geom* g, const void* qt, const void* kt, const void* vt,
                                       const uint32_t* mask, const int32_t* kv_count, float softmax_scale,
                                       void* out, float* lse, uint32_t* kernel_errors, void* stream);

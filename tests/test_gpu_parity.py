@@ -205,6 +205,42 @@ def test_attention_mask_patterns(name, pattern):
     C.assert_attention_close(st)
 
 
+@pytest.mark.parametrize("name", ["ragged128", "tiny_ragged"])
+def test_attention_empty_rows(name):
+    """Rows of a caller mask that retain nothing: zeros in O, -inf LSE, BSA_KERR_BAD_MASK;
+    the other rows, including those sharing a work unit with the empty ones, as the oracle.
+    Query tiles 0 and 1 (one whole query block of the first unit) and a lone query tile 5
+    retain nothing."""
+    bsa = _bsa()
+    w, q, k, v, _ = C.inputs(name)
+    g = C.geometry(w)
+    NT = w.NT
+    rng = np.random.default_rng(29)
+    m = rng.random((w.B, w.H, NT, NT)) < 0.35
+    m[..., np.arange(NT), np.arange(NT)] = True
+    empty = [i for i in (0, 1, 5) if i < NT]
+    m[..., empty, :] = False
+    qt, kt, vt = (bsa.reorder(g, x.cuda()) for x in (q, k, v))
+    mask = torch.from_numpy(O.pack_bitmask(m).view(np.int32).copy()).cuda()
+    cnt = torch.from_numpy(m.sum(-1).astype(np.int32)).cuda()
+    ws = bsa.alloc_workspace(g)
+    out, lse = bsa.sparse_attn_fwd(g, qt, kt, vt, mask, cnt, ws=ws)
+    torch.cuda.synchronize()
+    assert bsa.read_error(ws) & bsa.KERR_BAD_MASK
+    rows = [(b, h, i) for b in range(w.B) for h in range(w.H) for i in range(NT) if i not in empty]
+    qt64, kt64, vt64 = (O.reorder(O.to_f64(x), w.T, w.Hs, w.Ws) for x in (q, k, v))
+    ref = O.attention_tiles(qt64, kt64, vt64, m, rows, T=w.T, Hs=w.Hs, Ws=w.Ws)
+    st = C.compare_attention(w, out, lse, ref)
+    C.assert_attention_close(st)
+    # the empty rows' valid tokens: O = 0, LSE = -inf
+    src, valid = O.slot_tokens(w.T, w.Hs, w.Ws), O.slot_valid(w.T, w.Hs, w.Ws)
+    toks = np.concatenate([src[i][valid[i]] for i in empty])
+    o = out.float().cpu().numpy()
+    l = lse.float().cpu().numpy()
+    assert np.all(o[:, toks] == 0.0)
+    assert np.all(np.isneginf(l[:, :, toks]))
+
+
 def test_attention_all_retained_equals_dense():
     """All tiles retained: equals dense softmax attention over the raster sequence."""
     bsa = _bsa()
