@@ -366,9 +366,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a, const fl
   ncand = (int)row_combine<WPR, false>((uint64_t)ncand, xb, par, q, rw);
   if (MODE == kSelectMass) extra = mass_need > 0.0f ? ncand : 0;   // refined by the mass search
   extra = max(0, min(extra, ncand));
-  // extra and ncand are row-uniform by construction; the explicit broadcast from lane 0 is
-  // kept because builds without it (nvcc 12.9, -O3) selected every candidate of budget-mode
-  // rows, a code-generation effect whose cause was not identified.
+  // extra and ncand are row-uniform by construction, yet a build of this kernel without the
+  // broadcast from lane 0 below, run in budget mode, selected wrong rows (most rows of a
+  // ragged budget case; nvcc 12.9, -O3), and converging the warp before the named
+  // barriers of row_combine did not change that; with the broadcast every mode is
+  // bit-exact. The cause is not identified. The budget and fixed modes now run on
+  // select_radix_kernel; this kernel serves the cumulative-mass mode, which passes with or
+  // without the broadcast, and keeps it.
   extra = __shfl_sync(0xffffffffu, extra, 0);
   ncand = __shfl_sync(0xffffffffu, ncand, 0);
 
