@@ -1,9 +1,12 @@
 """The selection kernel's algorithm, replayed on the CPU against the oracle's selection.
 
-The GPU select kernel does not sort. It maps fp32 scores to order-preserving unsigned keys
-and takes the best candidates in one of two ways: repeated argmax (largest key, then lowest
-tile index) when a few are needed, or a bitwise binary search for a threshold key (with an
-early exit when the count is exact) followed by taking tied keys in index order. The
+The GPU select kernels do not sort. They map fp32 scores to order-preserving unsigned keys
+and take the best candidates in one of three ways: repeated argmax (largest key, then
+lowest tile index) when a few are needed, or a bitwise binary search for a threshold key
+(with an early exit when the count is exact), or (the fixed and budget modes' radix
+kernel) a search that narrows a key range from the candidates' [min, max] through at most
+256 buckets of 2^shift keys per pass, ending early on a bucket that holds exactly the keys
+still needed; each is followed by taking tied keys in index order. The
 cumulative-mass mode searches the fp32 bits of positive pooled probabilities and counts mass
 instead of keys. This module replays those steps in NumPy, with the kernel's fp32
 arithmetic, and checks on many random rows with heavy ties that they select exactly what a
@@ -60,6 +63,43 @@ def select_by_count(keys: np.ndarray, cand: np.ndarray, extra: int) -> np.ndarra
     return cand & ((kr > thr) | (eq & (rank < need_eq)))
 
 
+def select_by_range(keys: np.ndarray, cand: np.ndarray, extra: int, bucket_bits: int = 8) -> np.ndarray:
+    """The radix kernel's selection: keys >= t_ge, plus the first need_eq keys equal to thr
+    in index order. bucket_bits = 8 is the kernel (at most 2^8 buckets per pass)."""
+    kr = np.where(cand, keys, 0).astype(np.uint64)
+    ncand = int(cand.sum())
+    extra = max(0, min(extra, ncand))
+    thr, need_eq = 0, 0
+    if extra == 0:
+        t_ge = 0xFFFFFFFF + 1                      # nothing
+    elif extra == ncand:
+        t_ge = 1
+    else:
+        lo, hi = int(kr[cand].min()), int(kr[cand].max())
+        remaining, done = extra, False
+        while not done:
+            span = hi - lo
+            shift = 0 if span < (1 << bucket_bits) else span.bit_length() - bucket_bits
+            inr = cand & (kr >= lo) & (kr <= hi)
+            bucket = (kr[inr].astype(np.int64) - lo) >> shift
+            cnt = np.bincount(bucket, minlength=1 << bucket_bits)
+            suf = np.cumsum(cnt[::-1])[::-1]
+            d = int(np.nonzero(suf >= remaining)[0].max())
+            above = int(suf[d + 1]) if d + 1 < cnt.size else 0
+            at = int(cnt[d])
+            remaining -= above
+            blo = lo + (d << shift)
+            bhi = min(hi, blo + (1 << shift) - 1)
+            if at == remaining:
+                t_ge, done = blo, True
+            elif shift == 0:
+                thr, t_ge, need_eq, done = blo, blo + 1, remaining, True
+            lo, hi = blo, bhi
+    eq = cand & (kr == thr) & (need_eq > 0)
+    rank = np.cumsum(eq) - eq
+    return cand & ((kr >= t_ge) | (eq & (rank < need_eq)))
+
+
 def select_by_mass(e: np.ndarray, cand: np.ndarray, need: np.float32) -> np.ndarray:
     """Cumulative-mass mode: e are the unnormalised fp32 pooled probabilities."""
     kr = np.where(cand, np.maximum(e.astype(np.float32).view(np.uint32), 1), 0).astype(np.uint64)
@@ -103,6 +143,59 @@ def test_count_selection_matches_sort(n):
             want = np.zeros(n, bool)
             want[O.top_outside(s.astype(np.float64), ~cand, min(extra, int(cand.sum())))] = True
             assert np.array_equal(got, want), (n, extra)
+
+
+@pytest.mark.parametrize("n", [60, 624, 2160])
+def test_range_selection_matches_sort(n):
+    rng = np.random.default_rng(7 + n)
+    for s, cand in _rows(rng, 200 if n < 1000 else 60, n):
+        for extra in (0, 1, 3, 17, 32, 33, 80, int(cand.sum()), int(cand.sum()) + 5):
+            got = select_by_range(order_key(s), cand, extra)
+            want = np.zeros(n, bool)
+            want[O.top_outside(s.astype(np.float64), ~cand, min(extra, int(cand.sum())))] = True
+            assert np.array_equal(got, want), (n, extra)
+
+
+def test_range_selection_spread_and_outliers():
+    """Scores spread over many binades and rows with a few huge outliers (the range is
+    then dominated by them, so the first pass puts nearly every key in one bucket)."""
+    rng = np.random.default_rng(11)
+    for _ in range(200):
+        n = int(rng.integers(40, 700))
+        s = (rng.standard_normal(n) * np.exp(rng.uniform(-8, 8, n))).astype(np.float32)
+        if rng.random() < 0.5:
+            s[rng.integers(0, n, 3)] = np.float32(1e30)
+        cand = rng.random(n) < 0.8
+        for extra in (1, 5, 40, int(cand.sum()) - 1):
+            got = select_by_range(order_key(s), cand, extra)
+            want = np.zeros(n, bool)
+            want[O.top_outside(s.astype(np.float64), ~cand, max(0, min(extra, int(cand.sum()))))] = True
+            assert np.array_equal(got, want)
+
+
+def test_planted_range_bucket_off_by_one_is_caught():
+    """Taking the bucket below the right one (the boundary one bucket too low) must
+    disagree with the sort somewhere."""
+    rng = np.random.default_rng(13)
+
+    def wrong(keys, cand, extra):
+        kr = np.where(cand, keys, 0).astype(np.uint64)
+        lo, hi = int(kr[cand].min()), int(kr[cand].max())
+        shift = max(0, (hi - lo).bit_length() - 8)
+        cnt = np.bincount((kr[cand].astype(np.int64) - lo) >> shift, minlength=256)
+        suf = np.cumsum(cnt[::-1])[::-1]
+        d = max(0, int(np.nonzero(suf >= extra)[0].max()) - 1)
+        return cand & (kr >= lo + (d << shift))
+
+    bad = 0
+    for s, cand in _rows(rng, 60, 624):
+        extra = 30
+        if int(cand.sum()) <= extra:
+            continue
+        want = np.zeros(s.size, bool)
+        want[O.top_outside(s.astype(np.float64), ~cand, extra)] = True
+        bad += int(not np.array_equal(wrong(order_key(s), cand, extra), want))
+    assert bad > 0
 
 
 @pytest.mark.parametrize("n", [60, 624])
