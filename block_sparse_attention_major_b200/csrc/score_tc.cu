@@ -134,24 +134,33 @@ __global__ void __launch_bounds__(kTcThreads) score_tc_kernel(const __grid_const
   }
 
   if (ok) {
-    const int i = i0 + warp * 32 + lane;                 // this thread's TMEM lane = query tile
-    float* row = S + ((long long)bh * g.NT + i) * NKTP + j0;
+    // 32 accumulator columns at a time: each thread stages its row in shared memory (the
+    // operand slices are free: every product has completed), then its warp writes its 32
+    // rows with each instruction covering four rows of 128 contiguous bytes.
+    constexpr int kStageRow = 36;                         // floats; 144-byte rows keep float4 accesses conflict-free
+    float* stage = reinterpret_cast<float*>(smem + kTcA);
     const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
 #pragma unroll 1
     for (int q = 0; q < kTcTile / 32; ++q) {
       uint32_t v[32];
       tmem_ld_x32(taddr + 32 * q, v);
       ptx::tmem_wait_ld();
-      if (i < g.NT) {
+      float4* mine = reinterpret_cast<float4*>(stage + tid * kStageRow);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int j = 32 * q + 4 * e;
-          if (j0 + j < NKTP)
-            *reinterpret_cast<float4*>(row + j) =
-                make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                            __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
-        }
+      for (int e = 0; e < 8; ++e)
+        mine[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                              __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+      __syncwarp();
+      const int jj = j0 + 32 * q + 4 * (lane & 7);
+#pragma unroll
+      for (int rr = 0; rr < 32; rr += 4) {
+        const int rloc = warp * 32 + rr + (lane >> 3);
+        const int i = i0 + rloc;
+        if (i < g.NT && jj < NKTP)
+          *reinterpret_cast<float4*>(S + ((long long)bh * g.NT + i) * NKTP + jj) =
+              *reinterpret_cast<const float4*>(stage + rloc * kStageRow + 4 * (lane & 7));
       }
+      __syncwarp();
     }
   }
 
